@@ -1,0 +1,602 @@
+// C ABI of libdflash.so: argument validation, workspace layout and the
+// kernel sequence of one draft step.  No entry point allocates memory.
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dfl {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+namespace {
+
+thread_local std::string t_err;
+
+dflash_status fail(dflash_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return s;
+}
+
+dflash_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(DFLASH_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define DFL_CUDA(call, what)                          \
+  do {                                                \
+    cudaError_t e_ = (call);                          \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+#define DFL_CHECK(cond, status, ...)                 \
+  do {                                               \
+    if (!(cond)) return fail(status, __VA_ARGS__);   \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+size_t esize(const dflash_config* c) { return c->dtype == DFLASH_BF16 ? 2 : 4; }
+
+dflash_status check_config(const dflash_config* c) {
+  DFL_CHECK(c != nullptr, DFLASH_EINVAL, "config is NULL");
+  DFL_CHECK(c->dtype == DFLASH_FP32 || c->dtype == DFLASH_BF16, DFLASH_EINVAL,
+            "dtype must be DFLASH_FP32 (0) or DFLASH_BF16 (1), got %d", c->dtype);
+  const int mult = c->dtype == DFLASH_BF16 ? 8 : 4;
+  DFL_CHECK(c->hidden > 0 && c->hidden % mult == 0, DFLASH_EINVAL,
+            "hidden must be a positive multiple of %d, got %d", mult, c->hidden);
+  DFL_CHECK(c->ffn > 0 && c->ffn % mult == 0, DFLASH_EINVAL,
+            "ffn must be a positive multiple of %d, got %d", mult, c->ffn);
+  DFL_CHECK(c->n_q_heads > 0 && c->n_kv_heads > 0 && c->n_q_heads % c->n_kv_heads == 0,
+            DFLASH_EINVAL, "n_q_heads (%d) must be a positive multiple of n_kv_heads (%d)",
+            c->n_q_heads, c->n_kv_heads);
+  DFL_CHECK(c->head_dim == 64 || c->head_dim == 128, DFLASH_EUNSUPPORTED,
+            "head_dim must be 64 or 128, got %d", c->head_dim);
+  DFL_CHECK(c->n_draft_layers >= 1 && c->n_draft_layers <= kMaxLayers, DFLASH_EINVAL,
+            "n_draft_layers must be in [1, %d], got %d", kMaxLayers, c->n_draft_layers);
+  DFL_CHECK(c->n_target_layers >= 1 && c->n_target_layers <= kMaxTargetLayers, DFLASH_EINVAL,
+            "n_target_layers must be in [1, %d], got %d", kMaxTargetLayers, c->n_target_layers);
+  DFL_CHECK(c->block >= 1 && c->block <= kMaxBlock, DFLASH_EINVAL,
+            "block must be in [1, %d], got %d", kMaxBlock, c->block);
+  DFL_CHECK(c->vocab >= 2, DFLASH_EINVAL, "vocab must be >= 2, got %d", c->vocab);
+  DFL_CHECK(c->mask_token_id >= 0 && c->mask_token_id < c->vocab, DFLASH_EINVAL,
+            "mask_token_id %d outside [0, vocab)", c->mask_token_id);
+  DFL_CHECK(std::isfinite(c->rope_theta) && c->rope_theta > 0.f, DFLASH_EINVAL,
+            "rope_theta must be positive");
+  DFL_CHECK(std::isfinite(c->rms_eps) && c->rms_eps >= 0.f, DFLASH_EINVAL,
+            "rms_eps must be >= 0");
+  DFL_CHECK(c->hidden <= fuse_hidden_limit(c->dtype, c->n_target_layers), DFLASH_EUNSUPPORTED,
+            "hidden %d too large for the fusion kernel with T=%d (max %d)", c->hidden,
+            c->n_target_layers, fuse_hidden_limit(c->dtype, c->n_target_layers));
+  return DFLASH_OK;
+}
+
+#define DFL_PTR(p, name)                                                         \
+  do {                                                                           \
+    if ((p) == nullptr) return fail(DFLASH_EINVAL, "%s is NULL", name);          \
+    if (!aligned16(p)) return fail(DFLASH_EINVAL, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+void fill_inv_freq(const dflash_config* c, double* inv) {
+  const int half = c->head_dim / 2;
+  for (int i = 0; i < half; ++i)
+    inv[i] = std::pow(static_cast<double>(c->rope_theta), -2.0 * i / c->head_dim);
+}
+
+// ------------------------------------------------------------------ layout
+struct Layout {
+  size_t h = 0, x = 0, q = 0, kb = 0, vb = 0, attn = 0, act = 0, fused = 0, partial = 0,
+         attn_ws = 0, keys = 0, blk_pos = 0, new_pos = 0, new_dst = 0, total = 0;
+};
+
+size_t partial_floats(const dflash_config* c, int64_t M, int n_rows_total_segs[], int nseg, int K) {
+  if (M <= 0) return 0;
+  GemmPlan pl = plan_gemm(c->dtype, n_rows_total_segs, nseg, M, K);
+  return static_cast<size_t>(pl.splits) * M * pl.n_cols;
+}
+
+size_t step_partial_floats(const dflash_config* c, int64_t M, int64_t n_new) {
+  const int H = c->hidden, F = c->ffn, qd = c->n_q_heads * c->head_dim,
+            kvd = c->n_kv_heads * c->head_dim;
+  size_t mx = 0;
+  int ctx[2] = {kvd, kvd};
+  int qkv[3] = {qd, kvd, kvd};
+  int o[1] = {H};
+  int gu[2] = {F, F};
+  int dn[1] = {H};
+  mx = std::max(mx, partial_floats(c, n_new, ctx, 2, H));
+  mx = std::max(mx, partial_floats(c, M, ctx, 2, H));
+  mx = std::max(mx, partial_floats(c, M, qkv, 3, H));
+  mx = std::max(mx, partial_floats(c, M, o, 1, qd));
+  mx = std::max(mx, partial_floats(c, M, gu, 2, H));
+  mx = std::max(mx, partial_floats(c, M, dn, 1, F));
+  return mx;
+}
+
+Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_new,
+                   int64_t max_ctx) {
+  (void)n_req;
+  Layout L;
+  const size_t e = esize(c);
+  const int64_t M = static_cast<int64_t>(nb) * c->block;
+  const size_t H = c->hidden, F = c->ffn, qd = static_cast<size_t>(c->n_q_heads) * c->head_dim,
+               kvd = static_cast<size_t>(c->n_kv_heads) * c->head_dim;
+  size_t off = sizeof(DevStatus);
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.h = take(M * H * 4);
+  L.x = take(M * std::max(H, F) * e);
+  L.q = take(M * qd * e);
+  L.kb = take(M * kvd * e);
+  L.vb = take(M * kvd * e);
+  L.attn = take(M * qd * e);
+  L.act = take(M * F * e);
+  L.fused = take(static_cast<size_t>(c->n_draft_layers) * n_new * H * e);
+  L.partial = take(step_partial_floats(c, M, n_new) * 4);
+  AttnPlan ap = plan_attn(c->dtype, nb, c->block, c->n_q_heads, c->n_kv_heads, c->head_dim,
+                          max_ctx);
+  L.attn_ws = take(attn_ws_bytes(ap, nb, c->block, c->n_q_heads, c->head_dim));
+  L.keys = take(M * 8);
+  L.blk_pos = take(M * 4);
+  L.new_pos = take(n_new * 4);
+  L.new_dst = take(n_new * 8);
+  L.total = off;
+  return L;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+uint32_t* status_word(void* ws) { return static_cast<uint32_t*>(ws); }
+
+dflash_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  DFL_CHECK(ws != nullptr, DFLASH_EINVAL, "workspace is NULL");
+  DFL_CHECK((reinterpret_cast<uintptr_t>(ws) & 255u) == 0, DFLASH_EINVAL,
+            "workspace must be 256-byte aligned");
+  DFL_CHECK(ws_bytes >= need, DFLASH_EINVAL, "workspace too small: %zu bytes, need %zu",
+            ws_bytes, need);
+  return DFLASH_OK;
+}
+
+// ------------------------------------------------------------------ pieces
+// x [M][H] -> partial -> k_out/v_out (RoPE on K), optional row scatter.
+dflash_status run_kv_project(const dflash_config* c, const void* x, int64_t M,
+                             const int32_t* pos, const int64_t* dst, const void* wk,
+                             const void* wv, void* k_out, void* v_out, float* partial,
+                             uint32_t* status, cudaStream_t st) {
+  if (M <= 0) return DFLASH_OK;
+  const int kvd = c->n_kv_heads * c->head_dim;
+  GemmSeg segs[2] = {{wk, kvd}, {wv, kvd}};
+  int rows[2] = {kvd, kvd};
+  GemmPlan pl = plan_gemm(c->dtype, rows, 2, M, c->hidden);
+  DFL_CUDA(launch_gemm_partial(c->dtype, segs, 2, x, M, c->hidden, pl, partial, status, st),
+           "kv projection GEMM");
+  EpiParams ep{};
+  ep.nseg = 2;
+  ep.seg[0] = {EPI_STORE, kvd, 0, 1, k_out, kvd, dst != nullptr};
+  ep.seg[1] = {EPI_STORE, kvd, kvd, 0, v_out, kvd, dst != nullptr};
+  ep.M = M;
+  ep.n_cols = pl.n_cols;
+  ep.splits = pl.splits;
+  ep.partial = partial;
+  ep.pos = pos;
+  ep.dst_row = dst;
+  ep.head_dim = c->head_dim;
+  ep.out_bf16 = c->dtype == DFLASH_BF16;
+  fill_inv_freq(c, ep.inv_freq);
+  DFL_CUDA(launch_gemm_finish(ep, st), "kv projection epilogue");
+  return DFLASH_OK;
+}
+
+dflash_status run_mlp(const dflash_config* c, int64_t M, float* h, const float* g_mlp,
+                      const void* wg, const void* wu, const void* wd, void* x, void* act,
+                      float* partial, uint32_t* status, cudaStream_t st) {
+  if (M <= 0) return DFLASH_OK;
+  const int H = c->hidden, F = c->ffn;
+  DFL_CUDA(launch_rmsnorm(c->dtype, h, M, H, g_mlp, c->rms_eps, x, st), "mlp rmsnorm");
+  GemmSeg gu[2] = {{wg, F}, {wu, F}};
+  int rows[2] = {F, F};
+  GemmPlan pl = plan_gemm(c->dtype, rows, 2, M, H);
+  DFL_CUDA(launch_gemm_partial(c->dtype, gu, 2, x, M, H, pl, partial, status, st),
+           "gate/up GEMM");
+  EpiParams ep{};
+  ep.nseg = 2;
+  ep.seg[0] = {EPI_SWIGLU, F, 0, 0, act, F, 0};
+  ep.seg[1] = {EPI_NONE, F, F, 0, nullptr, 0, 0};
+  ep.M = M;
+  ep.n_cols = pl.n_cols;
+  ep.splits = pl.splits;
+  ep.partial = partial;
+  ep.out_bf16 = c->dtype == DFLASH_BF16;
+  DFL_CUDA(launch_gemm_finish(ep, st), "SwiGLU epilogue");
+  GemmSeg dn[1] = {{wd, H}};
+  int drows[1] = {H};
+  GemmPlan pd = plan_gemm(c->dtype, drows, 1, M, F);
+  DFL_CUDA(launch_gemm_partial(c->dtype, dn, 1, act, M, F, pd, partial, status, st),
+           "down GEMM");
+  EpiParams ed{};
+  ed.nseg = 1;
+  ed.seg[0] = {EPI_RESID, H, 0, 0, h, H, 0};
+  ed.M = M;
+  ed.n_cols = pd.n_cols;
+  ed.splits = pd.splits;
+  ed.partial = partial;
+  ed.out_bf16 = c->dtype == DFLASH_BF16;
+  DFL_CUDA(launch_gemm_finish(ed, st), "down epilogue");
+  return DFLASH_OK;
+}
+
+}  // namespace
+}  // namespace dfl
+
+using namespace dfl;
+
+extern "C" {
+
+const char* dflash_version(void) { return "dflash-b200 0.1 (sm_100a)"; }
+
+const char* dflash_last_error(void) { return t_err.c_str(); }
+
+uint64_t dflash_launch_count(void) { return g_launches.load(); }
+
+size_t dflash_workspace_size(const dflash_config* cfg, int32_t n_req, int32_t n_blocks,
+                             int64_t n_ctx_new, int64_t max_ctx_len) {
+  if (check_config(cfg) != DFLASH_OK || n_req < 0 || n_blocks < 0 || n_ctx_new < 0 ||
+      max_ctx_len < 0)
+    return 0;
+  return make_layout(cfg, n_req, n_blocks, n_ctx_new, max_ctx_len).total;
+}
+
+dflash_status dflash_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  DFL_CHECK(ws != nullptr, DFLASH_EINVAL, "workspace is NULL");
+  DFL_CHECK(ws_bytes >= sizeof(DevStatus), DFLASH_EINVAL, "workspace smaller than its header");
+  DFL_CUDA(cudaMemsetAsync(ws, 0, sizeof(DevStatus), static_cast<cudaStream_t>(stream)),
+           "workspace init");
+  return DFLASH_OK;
+}
+
+dflash_status dflash_check(void* ws, void* stream) {
+  DFL_CHECK(ws != nullptr, DFLASH_EINVAL, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DFL_CUDA(cudaStreamSynchronize(st), "stream synchronize");
+  uint32_t hdr[2] = {0, 0};
+  DFL_CUDA(cudaMemcpy(hdr, ws, sizeof(hdr), cudaMemcpyDeviceToHost), "read status");
+  if (hdr[0] != 0) {
+    DFL_CUDA(cudaMemset(ws, 0, sizeof(hdr)), "clear status");
+    const char* what = hdr[0] == DFLASH_ETIMEOUT ? "a bounded device wait ran out"
+                       : hdr[0] == DFLASH_ENUMERIC ? "non-finite logit"
+                                                   : "device error";
+    return fail(static_cast<dflash_status>(hdr[0]), "%s (kernel tag %u)", what, hdr[1]);
+  }
+  return DFLASH_OK;
+}
+
+dflash_status dflash_fuse_ctx(const dflash_config* cfg, const void* states, int64_t n_rows,
+                              const float* w_fuse, const float* const* g_fuse, void* fused,
+                              void* stream) {
+  dflash_status s = check_config(cfg);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(n_rows >= 0, DFLASH_EINVAL, "n_rows must be >= 0");
+  if (n_rows == 0) return DFLASH_OK;
+  DFL_PTR(states, "states");
+  DFL_PTR(fused, "fused");
+  DFL_CHECK(w_fuse != nullptr, DFLASH_EINVAL, "w_fuse is NULL");
+  DFL_CHECK(g_fuse != nullptr, DFLASH_EINVAL, "g_fuse is NULL");
+  for (int i = 0; i < cfg->n_draft_layers; ++i) DFL_PTR(g_fuse[i], "g_fuse[i]");
+  DFL_CUDA(launch_fuse(cfg->dtype, states, n_rows, cfg->n_target_layers, cfg->hidden,
+                       cfg->n_draft_layers, w_fuse, g_fuse, fused, cfg->rms_eps,
+                       static_cast<cudaStream_t>(stream)),
+           "fusion kernel");
+  return DFLASH_OK;
+}
+
+dflash_status dflash_kv_project(const dflash_config* cfg, const void* x, int64_t M,
+                                const int32_t* pos, const int64_t* dst_row, const void* w_k,
+                                const void* w_v, void* k_out, void* v_out, void* ws,
+                                size_t ws_bytes, void* stream) {
+  dflash_status s = check_config(cfg);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(M >= 0 && M < (int64_t(1) << 31), DFLASH_EINVAL, "M out of range");
+  if (M == 0) return DFLASH_OK;
+  DFL_PTR(x, "x");
+  DFL_PTR(w_k, "w_k");
+  DFL_PTR(w_v, "w_v");
+  DFL_PTR(k_out, "k_out");
+  DFL_PTR(v_out, "v_out");
+  DFL_CHECK(pos != nullptr, DFLASH_EINVAL, "pos is NULL");
+  const int kvd = cfg->n_kv_heads * cfg->head_dim;
+  int rows[2] = {kvd, kvd};
+  GemmPlan pl = plan_gemm(cfg->dtype, rows, 2, M, cfg->hidden);
+  const size_t need = sizeof(DevStatus) + static_cast<size_t>(pl.splits) * M * pl.n_cols * 4;
+  if ((s = check_ws(ws, ws_bytes, need)) != DFLASH_OK) return s;
+  return run_kv_project(cfg, x, M, pos, dst_row, w_k, w_v, k_out, v_out,
+                        at<float>(ws, sizeof(DevStatus)), status_word(ws),
+                        static_cast<cudaStream_t>(stream));
+}
+
+dflash_status dflash_block_attn(const dflash_config* cfg, int32_t n_blocks, const void* q,
+                                const void* k_blk, const void* v_blk, const void* k_ctx,
+                                const void* v_ctx, const int64_t* ctx_off,
+                                const int32_t* block_req, int64_t max_ctx_len, void* out,
+                                void* ws, size_t ws_bytes, void* stream) {
+  dflash_status s = check_config(cfg);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(n_blocks >= 0 && max_ctx_len >= 0, DFLASH_EINVAL, "negative size");
+  if (n_blocks == 0) return DFLASH_OK;
+  DFL_PTR(q, "q");
+  DFL_PTR(k_blk, "k_blk");
+  DFL_PTR(v_blk, "v_blk");
+  DFL_PTR(out, "out");
+  DFL_CHECK(ctx_off != nullptr && block_req != nullptr, DFLASH_EINVAL,
+            "ctx_off / block_req is NULL");
+  if (max_ctx_len > 0) {
+    DFL_PTR(k_ctx, "k_ctx");
+    DFL_PTR(v_ctx, "v_ctx");
+  }
+  AttnPlan ap = plan_attn(cfg->dtype, n_blocks, cfg->block, cfg->n_q_heads, cfg->n_kv_heads,
+                          cfg->head_dim, max_ctx_len);
+  const size_t need =
+      sizeof(DevStatus) + attn_ws_bytes(ap, n_blocks, cfg->block, cfg->n_q_heads, cfg->head_dim);
+  if ((s = check_ws(ws, ws_bytes, need)) != DFLASH_OK) return s;
+  DFL_CUDA(launch_attn(cfg->dtype, ap, n_blocks, cfg->block, cfg->n_q_heads, cfg->n_kv_heads,
+                       cfg->head_dim, q, k_blk, v_blk, k_ctx, v_ctx, ctx_off, block_req, out,
+                       at<float>(ws, sizeof(DevStatus)), status_word(ws),
+                       static_cast<cudaStream_t>(stream)),
+           "attention kernel");
+  return DFLASH_OK;
+}
+
+dflash_status dflash_mlp(const dflash_config* cfg, int64_t M, float* h, const float* g_mlp,
+                         const void* w_gate, const void* w_up, const void* w_down, void* ws,
+                         size_t ws_bytes, void* stream) {
+  dflash_status s = check_config(cfg);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(M >= 0 && M < (int64_t(1) << 31), DFLASH_EINVAL, "M out of range");
+  if (M == 0) return DFLASH_OK;
+  DFL_PTR(h, "h");
+  DFL_PTR(g_mlp, "g_mlp");
+  DFL_PTR(w_gate, "w_gate");
+  DFL_PTR(w_up, "w_up");
+  DFL_PTR(w_down, "w_down");
+  const size_t e = esize(cfg);
+  const int H = cfg->hidden, F = cfg->ffn;
+  int gu[2] = {F, F}, dn[1] = {H};
+  GemmPlan p1 = plan_gemm(cfg->dtype, gu, 2, M, H), p2 = plan_gemm(cfg->dtype, dn, 1, M, F);
+  const size_t part = std::max(static_cast<size_t>(p1.splits) * M * p1.n_cols,
+                               static_cast<size_t>(p2.splits) * M * p2.n_cols) * 4;
+  const size_t off_x = sizeof(DevStatus);
+  const size_t off_act = align256(off_x + M * H * e);
+  const size_t off_part = align256(off_act + M * F * e);
+  if ((s = check_ws(ws, ws_bytes, off_part + part)) != DFLASH_OK) return s;
+  return run_mlp(cfg, M, h, g_mlp, w_gate, w_up, w_down, at<void>(ws, off_x),
+                 at<void>(ws, off_act), at<float>(ws, off_part), status_word(ws),
+                 static_cast<cudaStream_t>(stream));
+}
+
+dflash_status dflash_lmhead_argmax(const dflash_config* cfg, int64_t M, const void* x,
+                                   const void* w_lm, int32_t* tok, float* max_logit, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  dflash_status s = check_config(cfg);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(M >= 0 && M < (int64_t(1) << 31), DFLASH_EINVAL, "M out of range");
+  if (M == 0) return DFLASH_OK;
+  DFL_PTR(x, "x");
+  DFL_PTR(w_lm, "w_lm");
+  DFL_CHECK(tok != nullptr, DFLASH_EINVAL, "tok is NULL");
+  if ((s = check_ws(ws, ws_bytes, sizeof(DevStatus) + M * 8)) != DFLASH_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* keys = at<unsigned long long>(ws, sizeof(DevStatus));
+  DFL_CUDA(launch_lmhead_argmax(cfg->dtype, w_lm, cfg->vocab, x, M, cfg->hidden, keys,
+                                status_word(ws), st),
+           "LM head argmax");
+  DFL_CUDA(launch_argmax_finish(keys, M, cfg->block, nullptr, nullptr, tok, max_logit, st),
+           "argmax finish");
+  return DFLASH_OK;
+}
+
+dflash_status dflash_accept(int32_t R, int32_t K, int32_t B, const int32_t* draft,
+                            const int32_t* target, int32_t* n_acc, int32_t* best_k,
+                            int32_t* out_tok, void* stream) {
+  DFL_CHECK(R >= 0, DFLASH_EINVAL, "R must be >= 0");
+  DFL_CHECK(K >= 1 && K <= 32, DFLASH_EINVAL, "K must be in [1, 32], got %d", K);
+  DFL_CHECK(B >= 1 && B <= kMaxBlock, DFLASH_EINVAL, "B must be in [1, %d], got %d", kMaxBlock, B);
+  if (R == 0) return DFLASH_OK;
+  DFL_CHECK(draft && target && n_acc && best_k && out_tok, DFLASH_EINVAL,
+            "a pointer argument is NULL");
+  DFL_CUDA(launch_accept(R, K, B, draft, target, n_acc, best_k, out_tok,
+                         static_cast<cudaStream_t>(stream)),
+           "accept kernel");
+  return DFLASH_OK;
+}
+
+dflash_status dflash_d2sd_candidates(int32_t R, int32_t B, int32_t K, int32_t mask_token_id,
+                                     const int32_t* base_tokens, const float* conf,
+                                     int32_t* known_len, int32_t* cand_tokens,
+                                     int32_t* block_req, void* stream) {
+  DFL_CHECK(R >= 0, DFLASH_EINVAL, "R must be >= 0");
+  DFL_CHECK(B >= 2 && B <= kMaxBlock, DFLASH_EINVAL, "B must be in [2, %d], got %d", kMaxBlock, B);
+  DFL_CHECK(K >= 1 && K <= B - 1, DFLASH_EINVAL, "K must be in [1, B-1], got %d", K);
+  if (R == 0) return DFLASH_OK;
+  DFL_CHECK(base_tokens && conf && known_len && cand_tokens, DFLASH_EINVAL,
+            "a pointer argument is NULL");
+  DFL_CUDA(launch_d2sd(R, B, K, mask_token_id, base_tokens, conf, known_len, cand_tokens,
+                       block_req, static_cast<cudaStream_t>(stream)),
+           "D2SD cut kernel");
+  return DFLASH_OK;
+}
+
+dflash_status dflash_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t limit_ns,
+                                           void* stream) {
+  dflash_status s = check_ws(ws, ws_bytes, sizeof(DevStatus));
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(limit_ns > 0 && limit_ns <= 2000000000ll, DFLASH_EINVAL,
+            "limit_ns must be in (0, 2e9]");
+  DFL_CUDA(launch_wait_selftest(status_word(ws), limit_ns, static_cast<cudaStream_t>(stream)),
+           "wait self test");
+  return DFLASH_OK;
+}
+
+dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
+                                const dflash_step_args* a, void* ws, size_t ws_bytes,
+                                void* stream) {
+  dflash_status s = check_config(c);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(w != nullptr && a != nullptr, DFLASH_EINVAL, "weights / args is NULL");
+  DFL_CHECK(a->n_req >= 1 && a->n_blocks >= 1, DFLASH_EINVAL, "n_req and n_blocks must be >= 1");
+  DFL_CHECK(a->n_ctx_new >= 0 && a->max_ctx_len >= 0, DFLASH_EINVAL, "negative context size");
+  DFL_CHECK(a->n_ctx_new < (int64_t(1) << 31), DFLASH_EINVAL, "n_ctx_new too large");
+  const int64_t M = static_cast<int64_t>(a->n_blocks) * c->block;
+  DFL_CHECK(a->block_req && a->block_tokens && a->ctx_off && a->draft_tokens, DFLASH_EINVAL,
+            "block_req / block_tokens / ctx_off / draft_tokens is NULL");
+  DFL_CHECK(a->k_cache && a->v_cache, DFLASH_EINVAL, "k_cache / v_cache is NULL");
+  if (a->n_ctx_new > 0) DFL_PTR(a->new_states, "new_states");
+  DFL_CHECK(w->w_fuse && w->layers, DFLASH_EINVAL, "w_fuse / layers is NULL");
+  DFL_PTR(w->embed, "embed");
+  DFL_PTR(w->lm_head, "lm_head");
+  DFL_PTR(w->g_final, "g_final");
+  const int D = c->n_draft_layers;
+  for (int i = 0; i < D; ++i) {
+    const dflash_layer_weights& l = w->layers[i];
+    DFL_PTR(l.w_q, "w_q");
+    DFL_PTR(l.w_kt, "w_kt");
+    DFL_PTR(l.w_vt, "w_vt");
+    DFL_PTR(l.w_kd, "w_kd");
+    DFL_PTR(l.w_vd, "w_vd");
+    DFL_PTR(l.w_o, "w_o");
+    DFL_PTR(l.w_gate, "w_gate");
+    DFL_PTR(l.w_up, "w_up");
+    DFL_PTR(l.w_down, "w_down");
+    DFL_PTR(l.g_fuse, "g_fuse");
+    DFL_PTR(l.g_attn, "g_attn");
+    DFL_PTR(l.g_mlp, "g_mlp");
+    if (a->max_ctx_len > 0) {
+      DFL_PTR(a->k_cache[i], "k_cache[i]");
+      DFL_PTR(a->v_cache[i], "v_cache[i]");
+    }
+  }
+  if (a->target_tokens) {
+    DFL_CHECK(a->n_cand >= 1 && a->n_cand <= 32 && a->n_blocks == a->n_req * a->n_cand,
+              DFLASH_EINVAL, "verification needs n_blocks == n_req * n_cand (n_cand in [1,32])");
+    DFL_CHECK(a->n_acc && a->best_k && a->out_tok, DFLASH_EINVAL,
+              "n_acc / best_k / out_tok is NULL");
+  }
+  const Layout L = make_layout(c, a->n_req, a->n_blocks, a->n_ctx_new, a->max_ctx_len);
+  if ((s = check_ws(ws, ws_bytes, L.total)) != DFLASH_OK) return s;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = status_word(ws);
+  const int dt = c->dtype;
+  const int H = c->hidden, qd = c->n_q_heads * c->head_dim, kvd = c->n_kv_heads * c->head_dim;
+  const size_t e = esize(c);
+  float* h = at<float>(ws, L.h);
+  void* x = at<void>(ws, L.x);
+  void* q = at<void>(ws, L.q);
+  void* kb = at<void>(ws, L.kb);
+  void* vb = at<void>(ws, L.vb);
+  void* attn = at<void>(ws, L.attn);
+  void* act = at<void>(ws, L.act);
+  uint8_t* fused = at<uint8_t>(ws, L.fused);
+  float* partial = at<float>(ws, L.partial);
+  int32_t* blk_pos = at<int32_t>(ws, L.blk_pos);
+  int32_t* new_pos = at<int32_t>(ws, L.new_pos);
+  int64_t* new_dst = at<int64_t>(ws, L.new_dst);
+  auto* keys = at<unsigned long long>(ws, L.keys);
+
+  DFL_CUDA(launch_prep_rows(a->n_req, a->n_blocks, c->block, a->block_req, a->ctx_off,
+                            a->new_off, a->ctx_cached, a->n_ctx_new, blk_pos, new_pos, new_dst,
+                            st),
+           "row bookkeeping");
+  if (a->n_ctx_new > 0) {
+    const float* gf[kMaxLayers];
+    for (int i = 0; i < D; ++i) gf[i] = w->layers[i].g_fuse;
+    DFL_CUDA(launch_fuse(dt, a->new_states, a->n_ctx_new, c->n_target_layers, H, D, w->w_fuse,
+                         gf, fused, c->rms_eps, st),
+             "fusion kernel");
+  }
+  DFL_CUDA(launch_embed(dt, w->embed, H, a->n_blocks, c->block, a->block_tokens, a->known_len,
+                        c->mask_token_id, h, st),
+           "slot embedding");
+  const AttnPlan ap = plan_attn(dt, a->n_blocks, c->block, c->n_q_heads, c->n_kv_heads,
+                                c->head_dim, a->max_ctx_len);
+  for (int i = 0; i < D; ++i) {
+    const dflash_layer_weights& l = w->layers[i];
+    // context K/V of the new rows through W^t, into the caches
+    if (a->n_ctx_new > 0) {
+      s = run_kv_project(c, fused + static_cast<size_t>(i) * a->n_ctx_new * H * e, a->n_ctx_new,
+                         new_pos, new_dst, l.w_kt, l.w_vt, a->k_cache[i], a->v_cache[i],
+                         partial, status, st);
+      if (s != DFLASH_OK) return s;
+    }
+    // block: RMSNorm -> Q (RoPE), K^d (RoPE), V^d
+    DFL_CUDA(launch_rmsnorm(dt, h, M, H, l.g_attn, c->rms_eps, x, st), "attention rmsnorm");
+    {
+      GemmSeg segs[3] = {{l.w_q, qd}, {l.w_kd, kvd}, {l.w_vd, kvd}};
+      int rows[3] = {qd, kvd, kvd};
+      GemmPlan pl = plan_gemm(dt, rows, 3, M, H);
+      DFL_CUDA(launch_gemm_partial(dt, segs, 3, x, M, H, pl, partial, status, st), "QKV GEMM");
+      EpiParams ep{};
+      ep.nseg = 3;
+      ep.seg[0] = {EPI_STORE, qd, 0, 1, q, qd, 0};
+      ep.seg[1] = {EPI_STORE, kvd, qd, 1, kb, kvd, 0};
+      ep.seg[2] = {EPI_STORE, kvd, qd + kvd, 0, vb, kvd, 0};
+      ep.M = M;
+      ep.n_cols = pl.n_cols;
+      ep.splits = pl.splits;
+      ep.partial = partial;
+      ep.pos = blk_pos;
+      ep.head_dim = c->head_dim;
+      ep.out_bf16 = dt == DFLASH_BF16;
+      fill_inv_freq(c, ep.inv_freq);
+      DFL_CUDA(launch_gemm_finish(ep, st), "QKV epilogue");
+    }
+    DFL_CUDA(launch_attn(dt, ap, a->n_blocks, c->block, c->n_q_heads, c->n_kv_heads,
+                         c->head_dim, q, kb, vb, a->k_cache[i], a->v_cache[i], a->ctx_off,
+                         a->block_req, attn, at<float>(ws, L.attn_ws), status, st),
+             "attention");
+    {
+      GemmSeg segs[1] = {{l.w_o, H}};
+      int rows[1] = {H};
+      GemmPlan pl = plan_gemm(dt, rows, 1, M, qd);
+      DFL_CUDA(launch_gemm_partial(dt, segs, 1, attn, M, qd, pl, partial, status, st),
+               "O GEMM");
+      EpiParams ep{};
+      ep.nseg = 1;
+      ep.seg[0] = {EPI_RESID, H, 0, 0, h, H, 0};
+      ep.M = M;
+      ep.n_cols = pl.n_cols;
+      ep.splits = pl.splits;
+      ep.partial = partial;
+      ep.out_bf16 = dt == DFLASH_BF16;
+      DFL_CUDA(launch_gemm_finish(ep, st), "O epilogue");
+    }
+    s = run_mlp(c, M, h, l.g_mlp, l.w_gate, l.w_up, l.w_down, x, act, partial, status, st);
+    if (s != DFLASH_OK) return s;
+  }
+  DFL_CUDA(launch_rmsnorm(dt, h, M, H, w->g_final, c->rms_eps, x, st), "final rmsnorm");
+  DFL_CUDA(launch_lmhead_argmax(dt, w->lm_head, c->vocab, x, M, H, keys, status, st),
+           "LM head argmax");
+  DFL_CUDA(launch_argmax_finish(keys, M, c->block, a->block_tokens, a->known_len,
+                                a->draft_tokens, a->max_logit, st),
+           "argmax finish");
+  if (a->target_tokens) {
+    DFL_CUDA(launch_accept(a->n_req, a->n_cand, c->block, a->draft_tokens, a->target_tokens,
+                           a->n_acc, a->best_k, a->out_tok, st),
+             "accept kernel");
+  }
+  return DFLASH_OK;
+}
+
+}  // extern "C"

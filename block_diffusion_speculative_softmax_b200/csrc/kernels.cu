@@ -1,0 +1,439 @@
+// Bandwidth- and latency-bound kernels of the draft step.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dfl {
+
+// ===========================================================================
+// Adaptive layer fusion + RMSNorm (DFLARE summary, section 2.1)
+//
+// One CTA per context row.  Thread t owns one 16-byte vector of columns and
+// keeps that vector of all T target layers in registers, so the T states
+// are read from HBM exactly once; all D draft layers' fused rows are
+// produced from them:  u_i = sum_j alpha_ij h_j,  f_i = u_i * rsqrt(mean
+// (u_i^2) + eps) * g_i  with alpha_i = softmax(W_fuse[i]).
+// ===========================================================================
+struct FuseGains {
+  const float* g[kMaxLayers];
+};
+
+// VW = 16: one 128-bit load per target layer; VW = 8 halves the registers
+// for large T.
+template <typename T, int VW> struct VecN;
+template <typename T> struct VecN<T, 16> : Vec16<T> {};
+template <> struct VecN<__nv_bfloat16, 8> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* out) {
+    uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+    float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
+    out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
+  }
+  __device__ __forceinline__ static void store(__nv_bfloat16* p, const float* in) {
+    uint2 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+    h[0] = __floats2bfloat162_rn(in[0], in[1]);
+    h[1] = __floats2bfloat162_rn(in[2], in[3]);
+    *reinterpret_cast<uint2*>(p) = u;
+  }
+};
+template <> struct VecN<float, 8> {
+  static constexpr int N = 2;
+  __device__ __forceinline__ static void load(const float* p, float* out) {
+    float2 u = __ldg(reinterpret_cast<const float2*>(p));
+    out[0] = u.x; out[1] = u.y;
+  }
+  __device__ __forceinline__ static void store(float* p, const float* in) {
+    *reinterpret_cast<float2*>(p) = make_float2(in[0], in[1]);
+  }
+};
+
+constexpr int kFuseThreads = 512;
+
+template <typename T, int MAXT, int VW>
+__global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(const T* __restrict__ states,
+                                                                 int64_t N, int nT, int H, int D,
+                                                                 const float* __restrict__ w_fuse,
+                                                                 const FuseGains gains,
+                                                                 T* __restrict__ fused, float eps) {
+  using V = VecN<T, VW>;
+  constexpr int VE = V::N;
+  __shared__ float alpha[kMaxLayers][kMaxTargetLayers];
+  __shared__ float red[32][kMaxLayers];
+  __shared__ float scale[kMaxLayers];
+  const int tid = threadIdx.x;
+  if (tid < D) {
+    float mx = -INFINITY;
+    for (int j = 0; j < nT; ++j) mx = fmaxf(mx, w_fuse[tid * nT + j]);
+    float s = 0.f;
+    for (int j = 0; j < nT; ++j) {
+      const float e = expf(w_fuse[tid * nT + j] - mx);
+      alpha[tid][j] = e;
+      s += e;
+    }
+    for (int j = 0; j < nT; ++j) alpha[tid][j] /= s;
+  }
+  __syncthreads();
+  const int nvec = H / VE;
+  const bool active = tid < nvec;
+  const int col = tid * VE;
+  for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
+    float h[MAXT][VE];
+    if (active) {
+      const T* src = states + (static_cast<size_t>(n) * nT) * H + col;
+#pragma unroll
+      for (int j = 0; j < MAXT; ++j)
+        if (j < nT) V::load(src + static_cast<size_t>(j) * H, h[j]);
+    }
+    float ss[kMaxLayers];
+#pragma unroll
+    for (int i = 0; i < kMaxLayers; ++i) ss[i] = 0.f;
+    if (active) {
+#pragma unroll
+      for (int i = 0; i < kMaxLayers; ++i) {
+        if (i >= D) break;
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < VE; ++e) {
+          float u = 0.f;
+#pragma unroll
+          for (int j = 0; j < MAXT; ++j)
+            if (j < nT) u = fmaf(alpha[i][j], h[j][e], u);
+          acc = fmaf(u, u, acc);
+        }
+        ss[i] = acc;
+      }
+    }
+    // block reduction of the D sums of squares
+    const int warp = tid >> 5, lane = tid & 31, nwarps = (blockDim.x + 31) >> 5;
+#pragma unroll
+    for (int i = 0; i < kMaxLayers; ++i) {
+      if (i >= D) break;
+      const float v = warp_sum(ss[i]);
+      if (lane == 0) red[warp][i] = v;
+    }
+    __syncthreads();
+    if (tid < D) {
+      float s = 0.f;
+      for (int w = 0; w < nwarps; ++w) s += red[w][tid];
+      scale[tid] = rsqrtf(s / static_cast<float>(H) + eps);
+    }
+    __syncthreads();
+    if (active) {
+      for (int i = 0; i < D; ++i) {
+        const float sc = scale[i];
+        const float* g = gains.g[i] + col;
+        float o[VE];
+#pragma unroll
+        for (int e = 0; e < VE; ++e) {
+          float u = 0.f;
+#pragma unroll
+          for (int j = 0; j < MAXT; ++j)
+            if (j < nT) u = fmaf(alpha[i][j], h[j][e], u);
+          o[e] = u * sc * __ldg(g + e);
+        }
+        V::store(fused + (static_cast<size_t>(i) * N + n) * H + col, o);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <typename T, int MAXT, int VW>
+static void fuse_go(const void* states, int64_t N, int nT, int H, int D, const float* w_fuse,
+                    const FuseGains& g, void* fused, float eps, cudaStream_t st) {
+  const int nvec = H / VecN<T, VW>::N;
+  const int threads = ((nvec + 31) / 32) * 32;
+  const int grid = static_cast<int>(std::min<int64_t>(N, 1 << 20));
+  fuse_rows_kernel<T, MAXT, VW><<<grid, threads, 0, st>>>(
+      static_cast<const T*>(states), N, nT, H, D, w_fuse, g, static_cast<T*>(fused), eps);
+}
+
+// Largest hidden size each variant covers with kFuseThreads threads.
+template <typename T>
+static int fuse_max_hidden(int nT) {
+  const int ve16 = 16 / static_cast<int>(sizeof(T));
+  return kFuseThreads * (nT <= 9 ? ve16 : ve16 / 2);
+}
+
+template <typename T>
+static cudaError_t launch_fuse_t(const void* states, int64_t N, int nT, int H, int D,
+                                 const float* w_fuse, const FuseGains& g, void* fused, float eps,
+                                 cudaStream_t st) {
+  if (H > fuse_max_hidden<T>(nT)) return cudaErrorInvalidValue;
+  if (nT <= 4) fuse_go<T, 4, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+  else if (nT <= 5) fuse_go<T, 5, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+  else if (nT <= 8) fuse_go<T, 8, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+  else if (nT <= 9) fuse_go<T, 9, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+  else fuse_go<T, 16, 8>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+  count_launch();
+  return cudaGetLastError();
+}
+
+int fuse_hidden_limit(int dtype, int nT) {
+  return dtype == DFLASH_BF16 ? fuse_max_hidden<__nv_bfloat16>(nT) : fuse_max_hidden<float>(nT);
+}
+
+cudaError_t launch_fuse(int dtype, const void* states, int64_t N, int nT, int H, int D,
+                        const float* w_fuse, const float* const* g_fuse, void* fused, float eps,
+                        cudaStream_t st) {
+  if (N <= 0) return cudaSuccess;
+  FuseGains g{};
+  for (int i = 0; i < D; ++i) g.g[i] = g_fuse[i];
+  if (dtype == DFLASH_BF16)
+    return launch_fuse_t<__nv_bfloat16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+  return launch_fuse_t<float>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+}
+
+// ===========================================================================
+// Slot embeddings: h[b*B + s] = embed[s < known_len[b] ? tok[b][s] : mask]
+// ===========================================================================
+template <typename T>
+__global__ void embed_kernel(const T* __restrict__ embed, int H, int B,
+                             const int32_t* __restrict__ block_tokens,
+                             const int32_t* __restrict__ known_len, int mask_id,
+                             float* __restrict__ h) {
+  const int m = blockIdx.x;
+  const int b = m / B, s = m % B;
+  const int kl = known_len ? known_len[b] : 1;
+  const int tok = s < kl ? block_tokens[m] : mask_id;
+  const T* src = embed + static_cast<size_t>(tok) * H;
+  for (int c = threadIdx.x; c < H; c += blockDim.x)
+    h[static_cast<size_t>(m) * H + c] = to_f(src[c]);
+}
+
+cudaError_t launch_embed(int dtype, const void* embed, int H, int nb, int B,
+                         const int32_t* block_tokens, const int32_t* known_len, int mask_id,
+                         float* h, cudaStream_t st) {
+  if (nb <= 0) return cudaSuccess;
+  if (dtype == DFLASH_BF16)
+    embed_kernel<__nv_bfloat16><<<nb * B, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(embed), H, B, block_tokens, known_len, mask_id, h);
+  else
+    embed_kernel<float><<<nb * B, 256, 0, st>>>(static_cast<const float*>(embed), H, B,
+                                                block_tokens, known_len, mask_id, h);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ===========================================================================
+// RMSNorm of the fp32 residual stream into the GEMM input dtype
+// ===========================================================================
+template <typename T>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ h, int H,
+                                                      const float* __restrict__ g, float eps,
+                                                      T* __restrict__ x) {
+  __shared__ float red[8];
+  const int64_t m = blockIdx.x;
+  const float* row = h + m * H;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < H; c += blockDim.x) ss = fmaf(row[c], row[c], ss);
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = rsqrtf(v / static_cast<float>(H) + eps);
+  }
+  __syncthreads();
+  const float sc = red[0];
+  for (int c = threadIdx.x; c < H; c += blockDim.x) x[m * H + c] = from_f<T>(row[c] * sc * g[c]);
+}
+
+cudaError_t launch_rmsnorm(int dtype, const float* h, int64_t M, int H, const float* g, float eps,
+                           void* x, cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  if (dtype == DFLASH_BF16)
+    rmsnorm_kernel<__nv_bfloat16><<<static_cast<unsigned>(M), 256, 0, st>>>(
+        h, H, g, eps, static_cast<__nv_bfloat16*>(x));
+  else
+    rmsnorm_kernel<float><<<static_cast<unsigned>(M), 256, 0, st>>>(h, H, g, eps,
+                                                                    static_cast<float*>(x));
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ===========================================================================
+// Row bookkeeping: RoPE positions of block slots and of new context rows,
+// and the cache row each new context row is written to.
+// ===========================================================================
+__global__ void prep_rows_kernel(int R, int nb, int B, const int32_t* __restrict__ block_req,
+                                 const int64_t* __restrict__ ctx_off,
+                                 const int64_t* __restrict__ new_off,
+                                 const int32_t* __restrict__ ctx_cached, int64_t n_new,
+                                 int32_t* __restrict__ blk_pos, int32_t* __restrict__ new_pos,
+                                 int64_t* __restrict__ new_dst) {
+  const int64_t tid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t m = tid; m < static_cast<int64_t>(nb) * B; m += stride) {
+    const int r = block_req[m / B];
+    blk_pos[m] = static_cast<int32_t>(ctx_off[r + 1] - ctx_off[r] + m % B);
+  }
+  const int64_t* off = new_off ? new_off : ctx_off;
+  for (int64_t n = tid; n < n_new; n += stride) {
+    int lo = 0, hi = R - 1;       // last r with off[r] <= n
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (off[mid] <= n) lo = mid; else hi = mid - 1;
+    }
+    const int64_t p = (ctx_cached ? ctx_cached[lo] : 0) + (n - off[lo]);
+    new_pos[n] = static_cast<int32_t>(p);
+    new_dst[n] = ctx_off[lo] + p;
+  }
+}
+
+cudaError_t launch_prep_rows(int R, int nb, int B, const int32_t* block_req,
+                             const int64_t* ctx_off, const int64_t* new_off,
+                             const int32_t* ctx_cached, int64_t n_new, int32_t* blk_pos,
+                             int32_t* new_pos, int64_t* new_dst, cudaStream_t st) {
+  const int64_t work = std::max<int64_t>(static_cast<int64_t>(nb) * B, n_new);
+  if (work <= 0) return cudaSuccess;
+  const int grid = static_cast<int>(std::min<int64_t>((work + 255) / 256, kNumSMs * 8));
+  prep_rows_kernel<<<grid, 256, 0, st>>>(R, nb, B, block_req, ctx_off, new_off, ctx_cached,
+                                         n_new, blk_pos, new_pos, new_dst);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ===========================================================================
+// argmax keys -> tokens (+ max logit); known slots keep their input token
+// ===========================================================================
+__global__ void argmax_finish_kernel(const unsigned long long* __restrict__ keys, int64_t M,
+                                     int B, const int32_t* __restrict__ block_tokens,
+                                     const int32_t* __restrict__ known_len,
+                                     int32_t* __restrict__ tok, float* __restrict__ max_logit) {
+  const int64_t m = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (m >= M) return;
+  const unsigned long long k = keys[m];
+  int32_t t = static_cast<int32_t>(key_index(k));
+  if (block_tokens) {
+    const int64_t b = m / B;
+    const int kl = known_len ? known_len[b] : 1;
+    if (m % B < kl) t = block_tokens[m];
+  }
+  tok[m] = t;
+  if (max_logit) max_logit[m] = key_value(k);
+}
+
+cudaError_t launch_argmax_finish(const unsigned long long* keys, int64_t M, int B,
+                                 const int32_t* block_tokens, const int32_t* known_len,
+                                 int32_t* tok, float* max_logit, cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  argmax_finish_kernel<<<static_cast<unsigned>((M + 255) / 256), 256, 0, st>>>(
+      keys, M, B, block_tokens, known_len, tok, max_logit);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ===========================================================================
+// Greedy acceptance: one warp per request; lane j compares draft[k][j]
+// with target[k][j-1] and a ballot gives the accepted prefix of candidate k
+// as the run of ones starting at slot 1.
+// ===========================================================================
+__global__ void accept_kernel(int R, int K, int B, const int32_t* __restrict__ draft,
+                              const int32_t* __restrict__ target, int32_t* __restrict__ n_acc,
+                              int32_t* __restrict__ best_k, int32_t* __restrict__ out_tok) {
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= R) return;
+  int best_n = -1, best = 0;
+  for (int k = 0; k < K; ++k) {
+    const int32_t* d = draft + (static_cast<size_t>(r) * K + k) * B;
+    const int32_t* t = target + (static_cast<size_t>(r) * K + k) * B;
+    const bool eq = lane >= 1 && lane < B && d[lane] == t[lane - 1];
+    const uint32_t bits = __ballot_sync(0xffffffffu, eq) >> 1;   // bit j-1 <-> slot j
+    const int n = __ffs(~bits) - 1;                               // leading run of ones
+    if (n > best_n) { best_n = n; best = k; }
+  }
+  const int32_t* d = draft + (static_cast<size_t>(r) * K + best) * B;
+  const int32_t* t = target + (static_cast<size_t>(r) * K + best) * B;
+  if (lane < B) {
+    int32_t v = -1;
+    if (lane < best_n) v = d[lane + 1];
+    else if (lane == best_n) v = t[best_n];
+    out_tok[static_cast<size_t>(r) * B + lane] = v;
+  }
+  if (lane == 0) {
+    n_acc[r] = best_n;
+    best_k[r] = best;
+  }
+}
+
+cudaError_t launch_accept(int R, int K, int B, const int32_t* draft, const int32_t* target,
+                          int32_t* n_acc, int32_t* best_k, int32_t* out_tok, cudaStream_t st) {
+  if (R <= 0) return cudaSuccess;
+  const int wpb = 4;
+  accept_kernel<<<(R + wpb - 1) / wpb, wpb * 32, 0, st>>>(R, K, B, draft, target, n_acc, best_k,
+                                                          out_tok);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ===========================================================================
+// D2SD cuts: one warp per request; lane j (1 <= j < B) ranks its confidence
+// against every other slot (ties: lower slot first); ranks < K are the cuts,
+// ordered by slot through a ballot prefix count.
+// ===========================================================================
+__global__ void d2sd_kernel(int R, int B, int K, int mask_id, const int32_t* __restrict__ base,
+                            const float* __restrict__ conf, int32_t* __restrict__ known_len,
+                            int32_t* __restrict__ cand, int32_t* __restrict__ block_req) {
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= R) return;
+  const float c = (lane >= 1 && lane < B) ? conf[static_cast<size_t>(r) * B + lane] : 0.f;
+  int rank = 0;
+  for (int i = 1; i < B; ++i) {
+    const float ci = __shfl_sync(0xffffffffu, c, i);
+    if (lane >= 1 && lane < B && (ci < c || (ci == c && i < lane))) ++rank;
+  }
+  const bool sel = lane >= 1 && lane < B && rank < K;
+  const uint32_t mask = __ballot_sync(0xffffffffu, sel);
+  if (sel) {
+    const int k = __popc(mask & ((1u << lane) - 1u));   // order by slot
+    known_len[static_cast<size_t>(r) * K + k] = lane;
+    if (block_req) block_req[static_cast<size_t>(r) * K + k] = r;
+  }
+  // candidate tokens: slot s of candidate k is base[s] if s < p_k else mask
+  const int32_t tok = lane < B ? base[static_cast<size_t>(r) * B + lane] : 0;
+  uint32_t rest = mask;
+  for (int k = 0; k < K; ++k) {
+    const int p = __ffs(rest) - 1;
+    rest &= rest - 1;
+    if (lane < B) cand[(static_cast<size_t>(r) * K + k) * B + lane] = lane < p ? tok : mask_id;
+  }
+}
+
+cudaError_t launch_d2sd(int R, int B, int K, int mask_id, const int32_t* base, const float* conf,
+                        int32_t* known_len, int32_t* cand, int32_t* block_req, cudaStream_t st) {
+  if (R <= 0) return cudaSuccess;
+  const int wpb = 4;
+  d2sd_kernel<<<(R + wpb - 1) / wpb, wpb * 32, 0, st>>>(R, B, K, mask_id, base, conf, known_len,
+                                                        cand, block_req);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ===========================================================================
+// Failure-detection self test: wait on a barrier that nothing completes.
+// ===========================================================================
+__global__ void wait_selftest_kernel(uint32_t* status, int64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, status, 99, static_cast<uint64_t>(limit_ns));
+  __syncthreads();
+}
+
+cudaError_t launch_wait_selftest(uint32_t* status, int64_t limit_ns, cudaStream_t st) {
+  wait_selftest_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace dfl

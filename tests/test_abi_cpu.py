@@ -1,0 +1,117 @@
+"""The C ABI without a GPU: libdflash.so loads, exports every function that
+include/dflash.h declares, and rejects bad arguments on the host before any
+CUDA call (these tests run on machines with no CUDA driver)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from block_diffusion_speculative_softmax_b200 import build as B
+from block_diffusion_speculative_softmax_b200 import dflash as DF
+from block_diffusion_speculative_softmax_b200 import synth
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "dflash.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return DF.load()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dflash_\w+)\s*\(", text)))
+
+
+def test_header_functions_are_exported(lib):
+    names = header_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in dflash.h but not exported"
+
+
+def test_binding_covers_exactly_the_header(lib):
+    assert sorted(DF.SIGNATURES) == header_functions()
+
+
+def test_version_and_counter(lib):
+    assert "sm_100a" in DF.dflash_version()
+    assert DF.dflash_launch_count() == 0
+
+
+def _cfg(**over):
+    c = DF.config_from(synth.get_config("qwen3_4b"))
+    for k, v in over.items():
+        setattr(c, k, v)
+    return c
+
+
+def test_workspace_size_valid_and_invalid(lib):
+    n = DF.dflash_workspace_size(_cfg(), 1, 1, 2048, 2048)
+    assert n > 0
+    assert n % 256 == 0
+    # more rows need more workspace
+    assert DF.dflash_workspace_size(_cfg(), 1, 1, 4096, 4096) > n
+    assert lib.dflash_workspace_size(C.byref(_cfg(head_dim=96)), 1, 1, 16, 16) == 0
+    assert lib.dflash_workspace_size(None, 1, 1, 16, 16) == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("dtype", 7, DF.EINVAL), ("head_dim", 96, DF.EUNSUPPORTED), ("block", 33, DF.EINVAL),
+    ("block", 0, DF.EINVAL), ("n_q_heads", 12, DF.EINVAL), ("hidden", 2561, DF.EINVAL),
+    ("mask_token_id", 151936, DF.EINVAL), ("n_draft_layers", 17, DF.EINVAL),
+    ("rope_theta", 0.0, DF.EINVAL), ("hidden", 16384, DF.EUNSUPPORTED)])
+def test_bad_config_rejected_before_any_launch(lib, field, value, status):
+    cfg = _cfg(**{field: value})
+    g = (C.c_void_p * 16)(*([16] * 16))
+    st = lib.dflash_fuse_ctx(C.byref(cfg), C.c_void_p(16), 4, C.c_void_p(16), g,
+                             C.c_void_p(16), None)
+    assert st == status
+    assert lib.dflash_last_error()
+    assert DF.dflash_launch_count() == 0
+
+
+def test_bad_pointers_and_sizes_rejected(lib):
+    cfg = _cfg()
+    # null / misaligned pointers
+    st = lib.dflash_lmhead_argmax(C.byref(cfg), 4, None, C.c_void_p(16), C.c_void_p(16), None,
+                                  C.c_void_p(256), 1 << 20, None)
+    assert st == DF.EINVAL and b"x is NULL" in lib.dflash_last_error()
+    st = lib.dflash_lmhead_argmax(C.byref(cfg), 4, C.c_void_p(24), C.c_void_p(16),
+                                  C.c_void_p(16), None, C.c_void_p(256), 1 << 20, None)
+    assert st == DF.EINVAL and b"aligned" in lib.dflash_last_error()
+    # workspace too small
+    st = lib.dflash_lmhead_argmax(C.byref(cfg), 4, C.c_void_p(16), C.c_void_p(16),
+                                  C.c_void_p(16), None, C.c_void_p(256), 64, None)
+    assert st == DF.EINVAL and b"workspace too small" in lib.dflash_last_error()
+    # accept: K and B out of range
+    assert lib.dflash_accept(1, 0, 8, *([C.c_void_p(16)] * 5), None) == DF.EINVAL
+    assert lib.dflash_accept(1, 1, 33, *([C.c_void_p(16)] * 5), None) == DF.EINVAL
+    assert lib.dflash_accept(1, 1, 8, None, *([C.c_void_p(16)] * 4), None) == DF.EINVAL
+    # D2SD: K must be in [1, B-1]
+    assert lib.dflash_d2sd_candidates(1, 16, 16, 5, *([C.c_void_p(16)] * 5), None) == DF.EINVAL
+    assert lib.dflash_d2sd_candidates(1, 1, 1, 5, *([C.c_void_p(16)] * 5), None) == DF.EINVAL
+    # self test: limit must be bounded
+    assert lib.dflash_selftest_wait_timeout(C.c_void_p(256), 4096, 10 ** 10, None) == DF.EINVAL
+    # empty work is a no-op, not an error
+    assert lib.dflash_accept(0, 1, 8, None, None, None, None, None, None) == DF.OK
+    assert DF.dflash_launch_count() == 0
+
+
+def test_draft_step_argument_checks(lib):
+    cfg = _cfg()
+    w = DF.Weights()
+    a = DF.StepArgs()
+    st = lib.dflash_draft_step(C.byref(cfg), C.byref(w), C.byref(a), C.c_void_p(256), 1 << 30,
+                               None)
+    assert st == DF.EINVAL and b"n_req" in lib.dflash_last_error()
+    a.n_req, a.n_blocks = 2, 3
+    a.target_tokens = 16
+    a.n_cand = 1
+    st = lib.dflash_draft_step(C.byref(cfg), C.byref(w), C.byref(a), C.c_void_p(256), 1 << 30,
+                               None)
+    assert st == DF.EINVAL
+    assert DF.dflash_launch_count() == 0
