@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the step eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--profile", action="store_true",
+                    help="eager steps inside an NVTX range 'dflash_step' (for ncu launch lists)")
+    ap.add_argument("--op", choices=["lmhead", "mlp", "ctxproj", "attn", "fuse"],
+                    help="time one entry point alone at the workload's shapes")
     return ap.parse_args()
 
 
@@ -132,25 +136,29 @@ class Clocks:
 
 
 # ---------------------------------------------------------------- distributed
-def dist_init(n):
+def dist_init(backend: str = "nccl"):
+    """One process per GPU (torchrun env).  Returns (rank, world, local_rank)."""
     import torch
     import torch.distributed as dist
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws > 1:
         lr = int(os.environ.get("LOCAL_RANK", "0"))
-        torch.cuda.set_device(lr)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", lr))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(lr)
+            kw["device_id"] = torch.device("cuda", lr)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
         return dist.get_rank(), ws, lr
     return 0, 1, 0
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Every rank gets the maximum of x over ranks (one all-reduce)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -232,7 +240,7 @@ def run_reference(args):
 # ---------------------------------------------------------------- our arm
 def run_ours(args):
     import torch
-    rank, world, lr = dist_init(args.gpus)
+    rank, world, lr = dist_init("nccl")
     from block_diffusion_speculative_softmax_b200 import build as B
     if rank == 0:
         B.build()
@@ -311,6 +319,7 @@ def run_ours(args):
     if not args.no_e2e:
         e2e = end_to_end(args, wl, DF, stream, world, blocks_per_step)
 
+    used_graph = graph is not None
     if graph is not None:
         del graph
     cpu = None
@@ -330,7 +339,7 @@ def run_ours(args):
                        "draft_layers": cfg.n_draft_layers, "target_layers": cfg.n_target_layers,
                        "hidden": cfg.hidden, "vocab": cfg.vocab,
                        "parallelism": f"replicas{world}",
-                       "cuda_graph": graph is not None or not args.no_graph,
+                       "cuda_graph": used_graph,
                        "l2": "inputs larger than L2 (weights %.2f GB streamed per step)"
                              % (wl.w.nbytes() / 1e9)},
             "gpu_launches": launches_per_step * args.steps,
@@ -412,10 +421,135 @@ def end_to_end(args, wl, DF, stream, world, blocks_per_step):
             "api": "dflash_draft_step via the Python binding, eager launches"}
 
 
+# ---------------------------------------------------------------- profiling modes
+def run_profile(args):
+    """Setup, W eager warm-up steps, then K eager steps inside the NVTX range
+    'dflash_step' (ncu --nvtx --nvtx-include dflash_step/ captures exactly
+    the kernels of those K steps)."""
+    import torch
+    from block_diffusion_speculative_softmax_b200 import build as B
+    B.build()
+    from block_diffusion_speculative_softmax_b200 import dflash as DF
+    from block_diffusion_speculative_softmax_b200 import synth, workload
+    cfg = synth.get_config(args.config)
+    wl = workload.Workload(cfg, seed=args.seed, mode=args.mode)
+    wl.step(verify=False)
+    torch.cuda.synchronize()
+    wl.plant_targets()
+    for _ in range(args.warmup):
+        wl.step(verify=True)
+    torch.cuda.synchronize()
+    c0 = DF.dflash_launch_count()
+    torch.cuda.nvtx.range_push("dflash_step")
+    for _ in range(args.steps):
+        wl.step(verify=True)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    wl.check()
+    print(json.dumps({"mode": "profile", "workload": cfg.name, "steps": args.steps,
+                      "launches": DF.dflash_launch_count() - c0}), flush=True)
+
+
+def run_op(args):
+    """One entry point alone at the workload's shapes: W warm-up + K timed
+    calls between CUDA events on the launching stream; achieved bandwidth
+    (or FLOP rate) from the algorithmic bytes (FLOPs) of one call."""
+    import torch
+    from block_diffusion_speculative_softmax_b200 import build as B
+    B.build()
+    from block_diffusion_speculative_softmax_b200 import dflash as DF
+    from block_diffusion_speculative_softmax_b200 import synth
+    cfg = synth.get_config(args.config)
+    cc = DF.config_from(cfg)
+    dt = DF.torch_dtype(cc)
+    e = 2 if cfg.dtype == "bf16" else 4
+    hbm, tfb, tfs, src = load_peaks()
+    H, F, V, T, D = cfg.hidden, cfg.ffn, cfg.vocab, cfg.n_target_layers, cfg.n_draft_layers
+    kvd, qd = cfg.kv_dim, cfg.q_dim
+    nb = cfg.n_req * cfg.n_cand
+    M = nb * cfg.block
+    lens = synth.ctx_lengths(cfg, args.seed)
+    N = int(sum(lens))
+    g = torch.Generator(device="cuda").manual_seed(args.seed)
+
+    def rnd(*shape, scale=1.0, dtype=dt):
+        return (torch.randn(*shape, device="cuda", generator=g) * scale).to(dtype)
+
+    ws = DF.alloc_workspace(DF.dflash_workspace_size(cc, cfg.n_req, nb, N, max(lens)))
+    flops = 0.0
+    if args.op == "lmhead":
+        x, w = rnd(M, H), rnd(V, H, scale=0.02)
+        tok = torch.empty(M, dtype=torch.int32, device="cuda")
+        call = lambda: DF.dflash_lmhead_argmax(cc, x, w, tok, None, ws)
+        algo = V * H * e + M * H * e + M * 4
+        kernel = "gemm_kernel<16,6,ARGMAX> (LM head)"
+    elif args.op == "mlp":
+        h = rnd(M, H, dtype=torch.float32)
+        gm = torch.ones(H, device="cuda")
+        wg, wu, wd = rnd(F, H, scale=0.02), rnd(F, H, scale=0.02), rnd(H, F, scale=0.02)
+        call = lambda: DF.dflash_mlp(cc, h, gm, wg, wu, wd, ws)
+        algo = 3 * F * H * e + 2 * M * H * 4
+        kernel = "rmsnorm + gemm_kernel x2 + finish x2 (SwiGLU MLP)"
+    elif args.op == "ctxproj":
+        x = rnd(N, H)
+        pos = torch.arange(N, dtype=torch.int32, device="cuda")
+        wk, wv = rnd(kvd, H, scale=0.02), rnd(kvd, H, scale=0.02)
+        ko, vo = torch.empty(N, kvd, dtype=dt, device="cuda"), torch.empty(N, kvd, dtype=dt,
+                                                                           device="cuda")
+        call = lambda: DF.dflash_kv_project(cc, x, pos, None, wk, wv, ko, vo, ws)
+        algo = N * H * e + 2 * kvd * H * e + 2 * N * kvd * e
+        flops = 2.0 * N * H * 2 * kvd
+        kernel = "gemm_kernel<256,4> + finish (context K/V projection, RoPE)"
+    elif args.op == "attn":
+        q, kb, vb = rnd(M, qd), rnd(M, kvd), rnd(M, kvd)
+        kc, vc = rnd(N, kvd), rnd(N, kvd)
+        off = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int64,
+                           device="cuda")
+        req = torch.arange(nb, dtype=torch.int32, device="cuda") // cfg.n_cand
+        out = torch.empty(M, qd, dtype=dt, device="cuda")
+        call = lambda: DF.dflash_block_attn(cc, nb, q, kb, vb, kc, vc, off, req, max(lens), out,
+                                            ws)
+        algo = 2 * N * kvd * e + 2 * M * qd * e + 2 * M * kvd * e
+        flops = 4.0 * cfg.n_cand * N * cfg.block * qd
+        kernel = "attn_mma_kernel + combine (split-KV block attention)"
+    else:  # fuse
+        st = rnd(N, T, H)
+        wf = torch.randn(D, T, device="cuda", generator=g)
+        gl = [torch.ones(H, device="cuda") for _ in range(D)]
+        fused = torch.empty(D, N, H, dtype=dt, device="cuda")
+        call = lambda: DF.dflash_fuse_ctx(cc, st, wf, gl, fused)
+        algo = N * T * H * e + D * N * H * e
+        kernel = "fuse_rows_kernel (fusion + RMSNorm, all draft layers)"
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        call()
+    e1.record()
+    e1.synchronize()
+    DF.dflash_check(ws)
+    sec = e0.elapsed_time(e1) / args.steps / 1e3
+    line = {"mode": "op", "op": args.op, "kernel": kernel, "workload": cfg.name,
+            "us_per_call": sec * 1e6, "algorithmic_bytes": algo,
+            "achieved_gbs": algo / sec / 1e9, "hbm_peak_gbs": hbm, "hbm_frac": algo / sec / 1e9 / hbm,
+            "peak_source": src, "steps": args.steps, "warmup": args.warmup}
+    if flops:
+        line.update({"flops": flops, "achieved_tflops": flops / sec / 1e12,
+                     "tensor_peak_tflops": tfb, "tensor_frac": flops / sec / 1e12 / tfb})
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.op:
+        run_op(args)
+    elif args.profile:
+        run_profile(args)
     else:
         run_ours(args)
 

@@ -136,6 +136,244 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_simt_kernel(const AttnPa
   }
 }
 
+// ---------------------------------------------------------------------------
+// bf16 tensor-core variant: 4 warps x 16 query rows, 64-key tiles streamed
+// into a double-buffered shared-memory ring by cp.async (16-byte chunks,
+// XOR-swizzled per row so ldmatrix is conflict-free), S = Q K^T and
+// O += P V on mma.sync m16n8k16 with fp32 accumulation, P kept in
+// registers, online softmax in the exp2 domain.
+// ---------------------------------------------------------------------------
+constexpr int kMmaRows = 64;
+constexpr int kMmaKeys = 64;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const uint32_t d = smem_u32(dst);
+  const int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                          uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) attn_mma_kernel(const AttnParams p) {
+  constexpr int CH = D / 8;                 // 16-byte chunks per key row
+  constexpr int NT = kMmaKeys / 8;          // n-tiles of S per key tile
+  constexpr int KS = D / 16;                // k-steps of Q K^T
+  constexpr int DT = D / 8;                 // n-tiles of O
+  extern __shared__ __align__(128) uint8_t smraw[];
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smraw);        // [2][64][D]
+  __nv_bfloat16* sV = sK + 2 * kMmaKeys * D;                          // [2][64][D]
+  const int b = blockIdx.x / p.Hkv, g = blockIdx.x % p.Hkv;
+  const int split = blockIdx.y;
+  const int r = p.block_req[b];
+  const int64_t c_begin = p.ctx_off[r];
+  const int64_t L = p.ctx_off[r + 1] - c_begin;
+  const int64_t k_lo = static_cast<int64_t>(split) * p.chunk;
+  const int n_ctx = static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(L, k_lo + p.chunk) - k_lo));
+  const int total = n_ctx + (split == 0 ? p.B : 0);
+  const int nrows_all = p.B * p.G;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int rbase = blockIdx.z * kMmaRows + warp * 16;
+  const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(p.q);
+  const __nv_bfloat16* KC = static_cast<const __nv_bfloat16*>(p.kc);
+  const __nv_bfloat16* VC = static_cast<const __nv_bfloat16*>(p.vc);
+  const __nv_bfloat16* KB = static_cast<const __nv_bfloat16*>(p.kb);
+  const __nv_bfloat16* VB = static_cast<const __nv_bfloat16*>(p.vb);
+
+  auto load_tile = [&](int t, int buf) {
+    for (int c = tid; c < kMmaKeys * CH; c += 128) {
+      const int kk = c / CH, ch = c % CH;
+      const int key = t * kMmaKeys + kk;
+      const __nv_bfloat16* sk = KC;
+      const __nv_bfloat16* sv = VC;
+      size_t off = 0;
+      const bool valid = key < total;
+      if (key < n_ctx) {
+        off = (static_cast<size_t>(c_begin + k_lo + key) * p.Hkv + g) * D + ch * 8;
+      } else if (valid) {
+        sk = KB;
+        sv = VB;
+        off = ((static_cast<size_t>(b) * p.B + (key - n_ctx)) * p.Hkv + g) * D + ch * 8;
+      } else {
+        sk = KB;   // any valid address; zero bytes are read
+        sv = VB;
+      }
+      const int sw = (ch ^ (kk & 7)) * 8;
+      cp_async16(sK + (buf * kMmaKeys + kk) * D + sw, sk + off, valid);
+      cp_async16(sV + (buf * kMmaKeys + kk) * D + sw, sv + off, valid);
+    }
+    cp_async_commit();
+  };
+
+  const int ntiles = (total + kMmaKeys - 1) / kMmaKeys;
+  if (ntiles > 0) load_tile(0, 0);
+
+  // Q fragments of this warp's 16 rows (rows past B*G read as zero)
+  uint32_t qf[KS][4];
+  {
+    const __nv_bfloat16* qrow[2] = {nullptr, nullptr};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int rr = rbase + gq + 8 * h;
+      if (rr < nrows_all) {
+        const int s = rr / p.G, j = rr % p.G;
+        qrow[h] = Q + ((static_cast<size_t>(b) * p.B + s) * p.Hq + g * p.G + j) * D;
+      }
+    }
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int col = ks * 16 + 2 * tq;
+        qf[ks][h] = qrow[h] ? *reinterpret_cast<const uint32_t*>(qrow[h] + col) : 0u;
+        qf[ks][h + 2] = qrow[h] ? *reinterpret_cast<const uint32_t*>(qrow[h] + col + 8) : 0u;
+      }
+    }
+  }
+
+  constexpr float kLog2e = 1.4426950408889634f;
+  const float sl2 = p.scale * kLog2e;
+  float o[DT][4];
+#pragma unroll
+  for (int i = 0; i < DT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  for (int t = 0; t < ntiles; ++t) {
+    const int buf = t & 1;
+    if (t + 1 < ntiles) {
+      load_tile(t + 1, buf ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint32_t kbase = smem_u32(sK + buf * kMmaKeys * D);
+    const uint32_t vbase = smem_u32(sV + buf * kMmaKeys * D);
+    // S = Q K^T  (16 rows x 64 keys per warp)
+    float sc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+      for (int k2 = 0; k2 < KS; k2 += 2) {
+        const int kk = nt * 8 + (lane & 7);
+        const int ch = k2 * 2 + (lane >> 3);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kbase + (kk * D + ((ch ^ (kk & 7)) * 8)) * 2, b0, b1, b2, b3);
+        mma_bf16(sc[nt], qf[k2], b0, b1);
+        mma_bf16(sc[nt], qf[k2 + 1], b2, b3);
+      }
+    }
+    // online softmax (rows gq and gq + 8 of the warp's 16)
+    const int key0 = t * kMmaKeys;
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool ok = key0 + nt * 8 + 2 * tq + e < total;
+        sc[nt][e] = ok ? sc[nt][e] * sl2 : -INFINITY;
+        sc[nt][e + 2] = ok ? sc[nt][e + 2] * sl2 : -INFINITY;
+        mx0 = fmaxf(mx0, sc[nt][e]);
+        mx1 = fmaxf(mx1, sc[nt][e + 2]);
+      }
+    }
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float c0 = exp2f(m0 - mn0), c1 = exp2f(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    l0 *= c0;
+    l1 *= c1;
+#pragma unroll
+    for (int i = 0; i < DT; ++i) {
+      o[i][0] *= c0; o[i][1] *= c0;
+      o[i][2] *= c1; o[i][3] *= c1;
+    }
+    uint32_t pf[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const float p0 = exp2f(sc[nt][0] - mn0), p1 = exp2f(sc[nt][1] - mn0);
+      const float p2 = exp2f(sc[nt][2] - mn1), p3 = exp2f(sc[nt][3] - mn1);
+      l0 += p0 + p1;
+      l1 += p2 + p3;
+      pf[nt][0] = pack_bf16(p0, p1);
+      pf[nt][1] = pack_bf16(p2, p3);
+    }
+    // O += P V
+#pragma unroll
+    for (int kk = 0; kk < kMmaKeys / 16; ++kk) {
+      const uint32_t a[4] = {pf[2 * kk][0], pf[2 * kk][1], pf[2 * kk + 1][0], pf[2 * kk + 1][1]};
+#pragma unroll
+      for (int dt = 0; dt < DT; dt += 2) {
+        const int mi = lane >> 3;
+        const int key = kk * 16 + (mi & 1) * 8 + (lane & 7);
+        const int ch = dt + (mi >> 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vbase + (key * D + ((ch ^ (key & 7)) * 8)) * 2, b0, b1, b2, b3);
+        mma_bf16(o[dt], a, b0, b1);
+        mma_bf16(o[dt + 1], a, b2, b3);
+      }
+    }
+    __syncthreads();
+  }
+  // partial results: unnormalised O, running max (natural-log units), sum
+#pragma unroll
+  for (int off = 1; off < 4; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+  constexpr float kLn2 = 0.6931471805599453f;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int rr = rbase + gq + 8 * h;
+    if (rr >= nrows_all) continue;
+    const int s = rr / p.G, j = rr % p.G;
+    const size_t pr = (static_cast<size_t>(b) * p.B + s) * p.Hq + g * p.G + j;
+    float* po = p.part_o + (pr * p.splits + split) * D;
+#pragma unroll
+    for (int dt = 0; dt < DT; ++dt)
+      *reinterpret_cast<float2*>(po + dt * 8 + 2 * tq) = make_float2(o[dt][2 * h], o[dt][2 * h + 1]);
+    if (tq == 0) {
+      const float mm = h ? m1 : m0;
+      p.part_ml[(pr * p.splits + split) * 2 + 0] = mm == -INFINITY ? -INFINITY : mm * kLn2;
+      p.part_ml[(pr * p.splits + split) * 2 + 1] = h ? l1 : l0;
+    }
+  }
+}
+
 // out[pr][dd] = sum_s o_s e^{m_s - M} / sum_s l_s e^{m_s - M}
 template <typename T>
 __global__ void attn_combine_kernel(const float* __restrict__ part_o,
@@ -170,8 +408,8 @@ static cudaError_t allow_smem() {
     const int bytes = 200 * 1024;
     const void* ks[4] = {reinterpret_cast<const void*>(attn_simt_kernel<float, 64>),
                          reinterpret_cast<const void*>(attn_simt_kernel<float, 128>),
-                         reinterpret_cast<const void*>(attn_simt_kernel<__nv_bfloat16, 64>),
-                         reinterpret_cast<const void*>(attn_simt_kernel<__nv_bfloat16, 128>)};
+                         reinterpret_cast<const void*>(attn_mma_kernel<64>),
+                         reinterpret_cast<const void*>(attn_mma_kernel<128>)};
     for (const void* k : ks) {
       cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
       if (e != cudaSuccess && err == cudaSuccess) err = e;
@@ -181,10 +419,9 @@ static cudaError_t allow_smem() {
 }
 
 AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d, int64_t max_ctx_len) {
-  (void)dtype;
   (void)d;
   AttnPlan p{};
-  p.rows_per_cta = kAttnWarps * kAttnRowsPerWarp;
+  p.rows_per_cta = dtype == DFLASH_BF16 ? kMmaRows : kAttnWarps * kAttnRowsPerWarp;
   const int G = Hq / Hkv;
   p.row_chunks = (B * G + p.rows_per_cta - 1) / p.rows_per_cta;
   const int64_t base = static_cast<int64_t>(nb) * Hkv * p.row_chunks;
@@ -227,17 +464,22 @@ cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq, 
   p.part_o = ws;
   p.part_ml = ws + static_cast<size_t>(n_rows) * plan.splits * d;
   dim3 grid(nb * Hkv, plan.splits, plan.row_chunks);
-  const size_t smem = (static_cast<size_t>(plan.rows_per_cta) * d +
-                       kAttnKeyTile * (d + 1) + kAttnKeyTile * d) * sizeof(float);
   cudaError_t e = cudaSuccess;
+  if (dtype == DFLASH_BF16) {
+    if ((e = allow_smem()) != cudaSuccess) return e;
+    const size_t smem = 2 * 2 * static_cast<size_t>(kMmaKeys) * d * sizeof(__nv_bfloat16);
+    if (d == 64)
+      attn_mma_kernel<64><<<grid, 128, smem, st>>>(p);
+    else
+      attn_mma_kernel<128><<<grid, 128, smem, st>>>(p);
+  } else {
+    const size_t smem = (static_cast<size_t>(plan.rows_per_cta) * d +
+                         kAttnKeyTile * (d + 1) + kAttnKeyTile * d) * sizeof(float);
 #define DFL_ATTN(T, DD)                                                                    \
   do {                                                                                     \
     if ((e = allow_smem()) != cudaSuccess) return e;                                       \
     attn_simt_kernel<T, DD><<<grid, kAttnWarps * 32, smem, st>>>(p);                       \
   } while (0)
-  if (dtype == DFLASH_BF16) {
-    if (d == 64) DFL_ATTN(__nv_bfloat16, 64); else DFL_ATTN(__nv_bfloat16, 128);
-  } else {
     if (d == 64) DFL_ATTN(float, 64); else DFL_ATTN(float, 128);
   }
 #undef DFL_ATTN

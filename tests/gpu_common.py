@@ -40,6 +40,8 @@ def token_report(gpu_tok, logits, dtype: str, tol: float = None):
     within that margin of the maximum.  Returns (n_exact, n_near, bad_rows)."""
     tol = TOL[dtype] if tol is None else tol
     gpu_tok = np.asarray(gpu_tok).reshape(-1)
+    if gpu_tok.shape[0] == 0:
+        return 0, 0, []
     logits = np.asarray(logits, dtype=np.float64).reshape(gpu_tok.shape[0], -1)
     n_exact = n_near = 0
     bad = []
