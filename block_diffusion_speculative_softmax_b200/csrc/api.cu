@@ -86,40 +86,88 @@ dflash_status check_config(const dflash_config* c) {
     if (!aligned16(p)) return fail(DFLASH_EINVAL, "%s is not 16-byte aligned", name); \
   } while (0)
 
-void fill_inv_freq(const dflash_config* c, double* inv) {
-  const int half = c->head_dim / 2;
-  for (int i = 0; i < half; ++i)
-    inv[i] = std::pow(static_cast<double>(c->rope_theta), -2.0 * i / c->head_dim);
+// ------------------------------------------------------------------ jobs
+GemmJob job_base(const dflash_config* c, const void* x, int64_t M, int K) {
+  GemmJob j;
+  j.x = x;
+  j.M = M;
+  j.K = K;
+  j.dtype = c->dtype;
+  j.head_dim = c->head_dim;
+  j.theta = c->rope_theta;
+  return j;
+}
+
+// K/V projection of context rows (W^t) or block rows (W^d): K with RoPE.
+GemmJob job_kv(const dflash_config* c, const void* x, int64_t M, const int32_t* pos,
+               const int64_t* dst, const void* wk, const void* wv, void* k_out, void* v_out) {
+  const int kvd = c->n_kv_heads * c->head_dim;
+  GemmJob j = job_base(c, x, M, c->hidden);
+  j.nseg = 2;
+  j.seg[0] = {wk, nullptr, kvd, EPI_STORE, 1, k_out, kvd, dst != nullptr};
+  j.seg[1] = {wv, nullptr, kvd, EPI_STORE, 0, v_out, kvd, dst != nullptr};
+  j.pos = pos;
+  j.dst = dst;
+  return j;
+}
+
+GemmJob job_qkv(const dflash_config* c, const dflash_layer_weights& l, const void* x, int64_t M,
+                const int32_t* pos, void* q, void* kb, void* vb) {
+  const int qd = c->n_q_heads * c->head_dim, kvd = c->n_kv_heads * c->head_dim;
+  GemmJob j = job_base(c, x, M, c->hidden);
+  j.nseg = 3;
+  j.seg[0] = {l.w_q, nullptr, qd, EPI_STORE, 1, q, qd, 0};
+  j.seg[1] = {l.w_kd, nullptr, kvd, EPI_STORE, 1, kb, kvd, 0};
+  j.seg[2] = {l.w_vd, nullptr, kvd, EPI_STORE, 0, vb, kvd, 0};
+  j.pos = pos;
+  return j;
+}
+
+GemmJob job_resid(const dflash_config* c, const void* w, const void* x, int64_t M, int K,
+                  float* h) {
+  GemmJob j = job_base(c, x, M, K);
+  j.nseg = 1;
+  j.seg[0] = {w, nullptr, c->hidden, EPI_RESID, 0, h, c->hidden, 0};
+  return j;
+}
+
+GemmJob job_swiglu(const dflash_config* c, const void* wg, const void* wu, const void* x,
+                   int64_t M, void* act) {
+  GemmJob j = job_base(c, x, M, c->hidden);
+  j.nseg = 1;
+  j.seg[0] = {wg, wu, c->ffn, EPI_SWIGLU, 0, act, c->ffn, 0};
+  return j;
 }
 
 // ------------------------------------------------------------------ layout
 struct Layout {
   size_t h = 0, x = 0, q = 0, kb = 0, vb = 0, attn = 0, act = 0, fused = 0, partial = 0,
-         attn_ws = 0, keys = 0, blk_pos = 0, new_pos = 0, new_dst = 0, total = 0;
+         attn_ws = 0, zero = 0, keys = 0, counters = 0, blk_pos = 0, new_pos = 0, new_dst = 0,
+         total = 0;
+  size_t zero_bytes = 0;   // [keys | counters], zeroed at the start of a step
 };
 
-size_t partial_floats(const dflash_config* c, int64_t M, int n_rows_total_segs[], int nseg, int K) {
-  if (M <= 0) return 0;
-  GemmPlan pl = plan_gemm(c->dtype, n_rows_total_segs, nseg, M, K);
-  return static_cast<size_t>(pl.splits) * M * pl.n_cols;
-}
+struct Needs {
+  size_t partial_floats = 0;
+  size_t counters = 0;
+  void take(const GemmPlan& p) {
+    partial_floats = std::max(partial_floats, p.partial_floats);
+    counters = std::max(counters, p.counters);
+  }
+};
 
-size_t step_partial_floats(const dflash_config* c, int64_t M, int64_t n_new) {
-  const int H = c->hidden, F = c->ffn, qd = c->n_q_heads * c->head_dim,
-            kvd = c->n_kv_heads * c->head_dim;
-  size_t mx = 0;
-  int ctx[2] = {kvd, kvd};
-  int qkv[3] = {qd, kvd, kvd};
-  int o[1] = {H};
-  int gu[2] = {F, F};
-  int dn[1] = {H};
-  mx = std::max(mx, partial_floats(c, n_new, ctx, 2, H));
-  mx = std::max(mx, partial_floats(c, M, ctx, 2, H));
-  mx = std::max(mx, partial_floats(c, M, qkv, 3, H));
-  mx = std::max(mx, partial_floats(c, M, o, 1, qd));
-  mx = std::max(mx, partial_floats(c, M, gu, 2, H));
-  mx = std::max(mx, partial_floats(c, M, dn, 1, F));
-  return mx;
+Needs step_needs(const dflash_config* c, int64_t M, int64_t n_new) {
+  Needs n;
+  dflash_layer_weights l{};
+  if (n_new > 0) n.take(plan_gemm(job_kv(c, nullptr, n_new, nullptr, nullptr, 0, 0, 0, 0)));
+  if (M > 0) {
+    n.take(plan_gemm(job_kv(c, nullptr, M, nullptr, nullptr, 0, 0, 0, 0)));
+    n.take(plan_gemm(job_qkv(c, l, nullptr, M, nullptr, 0, 0, 0)));
+    n.take(plan_gemm(job_resid(c, nullptr, nullptr, M, c->n_q_heads * c->head_dim, 0)));
+    n.take(plan_gemm(job_swiglu(c, nullptr, nullptr, nullptr, M, 0)));
+    n.take(plan_gemm(job_resid(c, nullptr, nullptr, M, c->ffn, 0)));
+  }
+  return n;
 }
 
 Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_new,
@@ -136,6 +184,9 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
     off = align256(off + bytes);
     return at;
   };
+  const Needs nd = step_needs(c, M, n_new);
+  AttnPlan ap = plan_attn(c->dtype, nb, c->block, c->n_q_heads, c->n_kv_heads, c->head_dim,
+                          max_ctx);
   L.h = take(M * H * 4);
   L.x = take(M * std::max(H, F) * e);
   L.q = take(M * qd * e);
@@ -144,11 +195,13 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
   L.attn = take(M * qd * e);
   L.act = take(M * F * e);
   L.fused = take(static_cast<size_t>(c->n_draft_layers) * n_new * H * e);
-  L.partial = take(step_partial_floats(c, M, n_new) * 4);
-  AttnPlan ap = plan_attn(c->dtype, nb, c->block, c->n_q_heads, c->n_kv_heads, c->head_dim,
-                          max_ctx);
+  L.partial = take(nd.partial_floats * 4);
   L.attn_ws = take(attn_ws_bytes(ap, nb, c->block, c->n_q_heads, c->head_dim));
+  const size_t ncount = std::max(nd.counters, attn_counters(ap, nb, c->n_kv_heads));
+  L.zero = off;
   L.keys = take(M * 8);
+  L.counters = take(ncount * 4);
+  L.zero_bytes = off - L.zero;
   L.blk_pos = take(M * 4);
   L.new_pos = take(n_new * 4);
   L.new_dst = take(n_new * 8);
@@ -171,71 +224,10 @@ dflash_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   return DFLASH_OK;
 }
 
-// ------------------------------------------------------------------ pieces
-// x [M][H] -> partial -> k_out/v_out (RoPE on K), optional row scatter.
-dflash_status run_kv_project(const dflash_config* c, const void* x, int64_t M,
-                             const int32_t* pos, const int64_t* dst, const void* wk,
-                             const void* wv, void* k_out, void* v_out, float* partial,
-                             uint32_t* status, cudaStream_t st) {
-  if (M <= 0) return DFLASH_OK;
-  const int kvd = c->n_kv_heads * c->head_dim;
-  GemmSeg segs[2] = {{wk, kvd}, {wv, kvd}};
-  int rows[2] = {kvd, kvd};
-  GemmPlan pl = plan_gemm(c->dtype, rows, 2, M, c->hidden);
-  DFL_CUDA(launch_gemm_partial(c->dtype, segs, 2, x, M, c->hidden, pl, partial, status, st),
-           "kv projection GEMM");
-  EpiParams ep{};
-  ep.nseg = 2;
-  ep.seg[0] = {EPI_STORE, kvd, 0, 1, k_out, kvd, dst != nullptr};
-  ep.seg[1] = {EPI_STORE, kvd, kvd, 0, v_out, kvd, dst != nullptr};
-  ep.M = M;
-  ep.n_cols = pl.n_cols;
-  ep.splits = pl.splits;
-  ep.partial = partial;
-  ep.pos = pos;
-  ep.dst_row = dst;
-  ep.head_dim = c->head_dim;
-  ep.out_bf16 = c->dtype == DFLASH_BF16;
-  fill_inv_freq(c, ep.inv_freq);
-  DFL_CUDA(launch_gemm_finish(ep, st), "kv projection epilogue");
-  return DFLASH_OK;
-}
-
-dflash_status run_mlp(const dflash_config* c, int64_t M, float* h, const float* g_mlp,
-                      const void* wg, const void* wu, const void* wd, void* x, void* act,
-                      float* partial, uint32_t* status, cudaStream_t st) {
-  if (M <= 0) return DFLASH_OK;
-  const int H = c->hidden, F = c->ffn;
-  DFL_CUDA(launch_rmsnorm(c->dtype, h, M, H, g_mlp, c->rms_eps, x, st), "mlp rmsnorm");
-  GemmSeg gu[2] = {{wg, F}, {wu, F}};
-  int rows[2] = {F, F};
-  GemmPlan pl = plan_gemm(c->dtype, rows, 2, M, H);
-  DFL_CUDA(launch_gemm_partial(c->dtype, gu, 2, x, M, H, pl, partial, status, st),
-           "gate/up GEMM");
-  EpiParams ep{};
-  ep.nseg = 2;
-  ep.seg[0] = {EPI_SWIGLU, F, 0, 0, act, F, 0};
-  ep.seg[1] = {EPI_NONE, F, F, 0, nullptr, 0, 0};
-  ep.M = M;
-  ep.n_cols = pl.n_cols;
-  ep.splits = pl.splits;
-  ep.partial = partial;
-  ep.out_bf16 = c->dtype == DFLASH_BF16;
-  DFL_CUDA(launch_gemm_finish(ep, st), "SwiGLU epilogue");
-  GemmSeg dn[1] = {{wd, H}};
-  int drows[1] = {H};
-  GemmPlan pd = plan_gemm(c->dtype, drows, 1, M, F);
-  DFL_CUDA(launch_gemm_partial(c->dtype, dn, 1, act, M, F, pd, partial, status, st),
-           "down GEMM");
-  EpiParams ed{};
-  ed.nseg = 1;
-  ed.seg[0] = {EPI_RESID, H, 0, 0, h, H, 0};
-  ed.M = M;
-  ed.n_cols = pd.n_cols;
-  ed.splits = pd.splits;
-  ed.partial = partial;
-  ed.out_bf16 = c->dtype == DFLASH_BF16;
-  DFL_CUDA(launch_gemm_finish(ed, st), "down epilogue");
+dflash_status run_job(const GemmJob& j, float* partial, uint32_t* counters, uint32_t* status,
+                      cudaStream_t st, const char* what) {
+  const GemmPlan pl = plan_gemm(j);
+  DFL_CUDA(launch_gemm(j, pl, partial, counters, status, st), what);
   return DFLASH_OK;
 }
 
@@ -317,14 +309,17 @@ dflash_status dflash_kv_project(const dflash_config* cfg, const void* x, int64_t
   DFL_PTR(k_out, "k_out");
   DFL_PTR(v_out, "v_out");
   DFL_CHECK(pos != nullptr, DFLASH_EINVAL, "pos is NULL");
-  const int kvd = cfg->n_kv_heads * cfg->head_dim;
-  int rows[2] = {kvd, kvd};
-  GemmPlan pl = plan_gemm(cfg->dtype, rows, 2, M, cfg->hidden);
-  const size_t need = sizeof(DevStatus) + static_cast<size_t>(pl.splits) * M * pl.n_cols * 4;
+  const GemmJob j = job_kv(cfg, x, M, pos, dst_row, w_k, w_v, k_out, v_out);
+  const GemmPlan pl = plan_gemm(j);
+  const size_t off_cnt = align256(sizeof(DevStatus) + pl.partial_floats * 4);
+  const size_t need = off_cnt + pl.counters * 4;
   if ((s = check_ws(ws, ws_bytes, need)) != DFLASH_OK) return s;
-  return run_kv_project(cfg, x, M, pos, dst_row, w_k, w_v, k_out, v_out,
-                        at<float>(ws, sizeof(DevStatus)), status_word(ws),
-                        static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DFL_CUDA(launch_zero(at<void>(ws, off_cnt), pl.counters * 4, st), "counter reset");
+  DFL_CUDA(launch_gemm(j, pl, at<float>(ws, sizeof(DevStatus)), at<uint32_t>(ws, off_cnt),
+                       status_word(ws), st),
+           "kv projection GEMM");
+  return DFLASH_OK;
 }
 
 dflash_status dflash_block_attn(const dflash_config* cfg, int32_t n_blocks, const void* q,
@@ -348,13 +343,16 @@ dflash_status dflash_block_attn(const dflash_config* cfg, int32_t n_blocks, cons
   }
   AttnPlan ap = plan_attn(cfg->dtype, n_blocks, cfg->block, cfg->n_q_heads, cfg->n_kv_heads,
                           cfg->head_dim, max_ctx_len);
-  const size_t need =
-      sizeof(DevStatus) + attn_ws_bytes(ap, n_blocks, cfg->block, cfg->n_q_heads, cfg->head_dim);
-  if ((s = check_ws(ws, ws_bytes, need)) != DFLASH_OK) return s;
+  const size_t off_cnt = align256(
+      sizeof(DevStatus) + attn_ws_bytes(ap, n_blocks, cfg->block, cfg->n_q_heads, cfg->head_dim));
+  const size_t ncnt = attn_counters(ap, n_blocks, cfg->n_kv_heads);
+  if ((s = check_ws(ws, ws_bytes, off_cnt + ncnt * 4)) != DFLASH_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DFL_CUDA(launch_zero(at<void>(ws, off_cnt), ncnt * 4, st), "counter reset");
   DFL_CUDA(launch_attn(cfg->dtype, ap, n_blocks, cfg->block, cfg->n_q_heads, cfg->n_kv_heads,
                        cfg->head_dim, q, k_blk, v_blk, k_ctx, v_ctx, ctx_off, block_req, out,
-                       at<float>(ws, sizeof(DevStatus)), status_word(ws),
-                       static_cast<cudaStream_t>(stream)),
+                       at<float>(ws, sizeof(DevStatus)), at<uint32_t>(ws, off_cnt),
+                       status_word(ws), st),
            "attention kernel");
   return DFLASH_OK;
 }
@@ -373,17 +371,25 @@ dflash_status dflash_mlp(const dflash_config* cfg, int64_t M, float* h, const fl
   DFL_PTR(w_down, "w_down");
   const size_t e = esize(cfg);
   const int H = cfg->hidden, F = cfg->ffn;
-  int gu[2] = {F, F}, dn[1] = {H};
-  GemmPlan p1 = plan_gemm(cfg->dtype, gu, 2, M, H), p2 = plan_gemm(cfg->dtype, dn, 1, M, F);
-  const size_t part = std::max(static_cast<size_t>(p1.splits) * M * p1.n_cols,
-                               static_cast<size_t>(p2.splits) * M * p2.n_cols) * 4;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t off_x = sizeof(DevStatus);
   const size_t off_act = align256(off_x + M * H * e);
+  const GemmJob j1 = job_swiglu(cfg, w_gate, w_up, at<void>(ws, off_x), M, at<void>(ws, off_act));
+  const GemmJob j2 = job_resid(cfg, w_down, at<void>(ws, off_act), M, F, h);
+  const GemmPlan p1 = plan_gemm(j1), p2 = plan_gemm(j2);
   const size_t off_part = align256(off_act + M * F * e);
-  if ((s = check_ws(ws, ws_bytes, off_part + part)) != DFLASH_OK) return s;
-  return run_mlp(cfg, M, h, g_mlp, w_gate, w_up, w_down, at<void>(ws, off_x),
-                 at<void>(ws, off_act), at<float>(ws, off_part), status_word(ws),
-                 static_cast<cudaStream_t>(stream));
+  const size_t off_cnt =
+      align256(off_part + std::max(p1.partial_floats, p2.partial_floats) * 4);
+  const size_t ncnt = std::max(p1.counters, p2.counters);
+  if ((s = check_ws(ws, ws_bytes, off_cnt + ncnt * 4)) != DFLASH_OK) return s;
+  float* part = at<float>(ws, off_part);
+  uint32_t* cnt = at<uint32_t>(ws, off_cnt);
+  DFL_CUDA(launch_zero(cnt, ncnt * 4, st), "counter reset");
+  DFL_CUDA(launch_rmsnorm(cfg->dtype, h, M, H, g_mlp, cfg->rms_eps, at<void>(ws, off_x), st),
+           "mlp rmsnorm");
+  DFL_CUDA(launch_gemm(j1, p1, part, cnt, status_word(ws), st), "gate/up GEMM");
+  DFL_CUDA(launch_gemm(j2, p2, part, cnt, status_word(ws), st), "down GEMM");
+  return DFLASH_OK;
 }
 
 dflash_status dflash_lmhead_argmax(const dflash_config* cfg, int64_t M, const void* x,
@@ -399,6 +405,7 @@ dflash_status dflash_lmhead_argmax(const dflash_config* cfg, int64_t M, const vo
   if ((s = check_ws(ws, ws_bytes, sizeof(DevStatus) + M * 8)) != DFLASH_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto* keys = at<unsigned long long>(ws, sizeof(DevStatus));
+  DFL_CUDA(launch_zero(keys, M * 8, st), "argmax key reset");
   DFL_CUDA(launch_lmhead_argmax(cfg->dtype, w_lm, cfg->vocab, x, M, cfg->hidden, keys,
                                 status_word(ws), st),
            "LM head argmax");
@@ -499,7 +506,7 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t* status = status_word(ws);
   const int dt = c->dtype;
-  const int H = c->hidden, qd = c->n_q_heads * c->head_dim, kvd = c->n_kv_heads * c->head_dim;
+  const int H = c->hidden, qd = c->n_q_heads * c->head_dim;
   const size_t e = esize(c);
   float* h = at<float>(ws, L.h);
   void* x = at<void>(ws, L.x);
@@ -514,10 +521,12 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
   int32_t* new_pos = at<int32_t>(ws, L.new_pos);
   int64_t* new_dst = at<int64_t>(ws, L.new_dst);
   auto* keys = at<unsigned long long>(ws, L.keys);
+  uint32_t* counters = at<uint32_t>(ws, L.counters);
 
+  // positions, cache rows, and zeroed argmax keys / tile counters
   DFL_CUDA(launch_prep_rows(a->n_req, a->n_blocks, c->block, a->block_req, a->ctx_off,
                             a->new_off, a->ctx_cached, a->n_ctx_new, blk_pos, new_pos, new_dst,
-                            st),
+                            at<uint32_t>(ws, L.zero), static_cast<int64_t>(L.zero_bytes / 4), st),
            "row bookkeeping");
   if (a->n_ctx_new > 0) {
     const float* gf[kMaxLayers];
@@ -535,55 +544,30 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
     const dflash_layer_weights& l = w->layers[i];
     // context K/V of the new rows through W^t, into the caches
     if (a->n_ctx_new > 0) {
-      s = run_kv_project(c, fused + static_cast<size_t>(i) * a->n_ctx_new * H * e, a->n_ctx_new,
-                         new_pos, new_dst, l.w_kt, l.w_vt, a->k_cache[i], a->v_cache[i],
-                         partial, status, st);
+      s = run_job(job_kv(c, fused + static_cast<size_t>(i) * a->n_ctx_new * H * e, a->n_ctx_new,
+                         new_pos, new_dst, l.w_kt, l.w_vt, a->k_cache[i], a->v_cache[i]),
+                  partial, counters, status, st, "context K/V GEMM");
       if (s != DFLASH_OK) return s;
     }
     // block: RMSNorm -> Q (RoPE), K^d (RoPE), V^d
     DFL_CUDA(launch_rmsnorm(dt, h, M, H, l.g_attn, c->rms_eps, x, st), "attention rmsnorm");
-    {
-      GemmSeg segs[3] = {{l.w_q, qd}, {l.w_kd, kvd}, {l.w_vd, kvd}};
-      int rows[3] = {qd, kvd, kvd};
-      GemmPlan pl = plan_gemm(dt, rows, 3, M, H);
-      DFL_CUDA(launch_gemm_partial(dt, segs, 3, x, M, H, pl, partial, status, st), "QKV GEMM");
-      EpiParams ep{};
-      ep.nseg = 3;
-      ep.seg[0] = {EPI_STORE, qd, 0, 1, q, qd, 0};
-      ep.seg[1] = {EPI_STORE, kvd, qd, 1, kb, kvd, 0};
-      ep.seg[2] = {EPI_STORE, kvd, qd + kvd, 0, vb, kvd, 0};
-      ep.M = M;
-      ep.n_cols = pl.n_cols;
-      ep.splits = pl.splits;
-      ep.partial = partial;
-      ep.pos = blk_pos;
-      ep.head_dim = c->head_dim;
-      ep.out_bf16 = dt == DFLASH_BF16;
-      fill_inv_freq(c, ep.inv_freq);
-      DFL_CUDA(launch_gemm_finish(ep, st), "QKV epilogue");
-    }
+    if ((s = run_job(job_qkv(c, l, x, M, blk_pos, q, kb, vb), partial, counters, status, st,
+                     "QKV GEMM")) != DFLASH_OK)
+      return s;
     DFL_CUDA(launch_attn(dt, ap, a->n_blocks, c->block, c->n_q_heads, c->n_kv_heads,
                          c->head_dim, q, kb, vb, a->k_cache[i], a->v_cache[i], a->ctx_off,
-                         a->block_req, attn, at<float>(ws, L.attn_ws), status, st),
+                         a->block_req, attn, at<float>(ws, L.attn_ws), counters, status, st),
              "attention");
-    {
-      GemmSeg segs[1] = {{l.w_o, H}};
-      int rows[1] = {H};
-      GemmPlan pl = plan_gemm(dt, rows, 1, M, qd);
-      DFL_CUDA(launch_gemm_partial(dt, segs, 1, attn, M, qd, pl, partial, status, st),
-               "O GEMM");
-      EpiParams ep{};
-      ep.nseg = 1;
-      ep.seg[0] = {EPI_RESID, H, 0, 0, h, H, 0};
-      ep.M = M;
-      ep.n_cols = pl.n_cols;
-      ep.splits = pl.splits;
-      ep.partial = partial;
-      ep.out_bf16 = dt == DFLASH_BF16;
-      DFL_CUDA(launch_gemm_finish(ep, st), "O epilogue");
-    }
-    s = run_mlp(c, M, h, l.g_mlp, l.w_gate, l.w_up, l.w_down, x, act, partial, status, st);
-    if (s != DFLASH_OK) return s;
+    if ((s = run_job(job_resid(c, l.w_o, attn, M, qd, h), partial, counters, status, st,
+                     "O GEMM")) != DFLASH_OK)
+      return s;
+    DFL_CUDA(launch_rmsnorm(dt, h, M, H, l.g_mlp, c->rms_eps, x, st), "mlp rmsnorm");
+    if ((s = run_job(job_swiglu(c, l.w_gate, l.w_up, x, M, act), partial, counters, status, st,
+                     "gate/up GEMM")) != DFLASH_OK)
+      return s;
+    if ((s = run_job(job_resid(c, l.w_down, act, M, c->ffn, h), partial, counters, status, st,
+                     "down GEMM")) != DFLASH_OK)
+      return s;
   }
   DFL_CUDA(launch_rmsnorm(dt, h, M, H, w->g_final, c->rms_eps, x, st), "final rmsnorm");
   DFL_CUDA(launch_lmhead_argmax(dt, w->lm_head, c->vocab, x, M, H, keys, status, st),

@@ -36,6 +36,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: wait for the previous kernel on the stream
+// (and the visibility of its writes) / let the next one start its prologue.
+// Both are no-ops for a kernel launched without the PDL attribute.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Scalar conversions
 // ---------------------------------------------------------------------------
 template <typename T> __device__ __forceinline__ float to_f(T v);

@@ -12,14 +12,29 @@
 //   warp 0 lane 0 : TMA producer (weight tile + token tile per stage)
 //   warp 1 lane 0 : tcgen05.mma issuer, commits each stage back to the ring
 //   warp 2        : TMEM allocation / release
-//   warps 0-3     : epilogue (TMEM -> registers -> global), one TMEM lane
-//                   (= one weight row) per thread
+//   warps 0-3     : epilogue, one TMEM lane (= one tile row) per thread
 //
-// Split-K writes fp32 partial sums that a fixed-order finish kernel reduces
-// (deterministic).  The LM-head variant keeps a per-CTA running (max, index)
-// and merges it with one 64-bit atomicMax per token, so logits never reach
-// global memory.  fp32 models run on a SIMT FFMA kernel with the same
-// partial layout (tensor-core tf32 would miss a 1e-4 tolerance).
+// The epilogue is fused: the accumulator tile is staged in shared memory
+// (the drained pipeline ring) and the segment's op is applied there --
+// RoPE (pairs i, i + d/2 of a head live in the same tile), scatter into a
+// KV cache, residual add, or SwiGLU (a SwiGLU tile stacks 64 rows of W_gate
+// over the same 64 rows of W_up, so silu(g) * u is formed inside one CTA).
+// With split-K every split writes its fp32 partial tile and the LAST CTA to
+// arrive at the tile's counter sums the splits in fixed order (so results
+// are deterministic), applies the op and re-arms the counter.
+//
+// Kernels are launched with programmatic dependent launch: the producer
+// streams the first ring stages of WEIGHTS (which no earlier kernel writes)
+// before griddepcontrol.wait, so a GEMM's pipeline fill overlaps the tail of
+// the kernel before it; activations, partials, counters and outputs are
+// only touched after the wait.
+//
+// The LM-head variant keeps a per-CTA (max, index) per token and merges it
+// with one 64-bit atomicMax, so logits never reach global memory.  fp32
+// models run on a SIMT FFMA kernel (partials + finish kernel): tensor-core
+// tf32 would miss a 1e-4 tolerance.
+#include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "common.cuh"
@@ -27,28 +42,49 @@
 
 namespace dfl {
 
+namespace {
+int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+}  // namespace
+
 // ===========================================================================
 // tcgen05 kernel
 // ===========================================================================
 namespace tc {
 
-constexpr int BM = 128;          // weight rows per tile (UMMA M)
+constexpr int BM = 128;          // tile rows (UMMA M)
 constexpr int BK = 64;           // bf16 per k-block: one 128-byte swizzle row
 constexpr int UK = 16;           // K per tcgen05.mma (kind::f16)
 constexpr int A_BYTES = BM * BK * 2;
+constexpr int SROW = BM + 4;     // fp32 staging row (tokens x tile rows)
+
+struct Seg {
+  int tile_begin;     // first row tile of the segment
+  int map;            // index of its (first) weight tensor map
+  int rows;           // output features
+  int pair;           // SwiGLU pair: 64 features per tile (gate rows over up rows)
+  int op;
+  int rope;
+  int use_dst;
+  int64_t out_stride;
+  void* out;
+};
 
 struct Params {
-  CUtensorMap tm_w0, tm_w1, tm_w2;  // weights of up to three segments
+  CUtensorMap tm[4];                // weights (a SwiGLU pair uses two maps)
   CUtensorMap tm_x;                 // activations [M][K]
-  int seg_tile_begin[kMaxSegs + 1]; // row-tile ranges of the segments
-  int seg_rows[kMaxSegs];
-  int seg_col0[kMaxSegs];
+  Seg seg[kMaxSegs];
   int nseg;
   int M;
   int kb_total;
   int kb_per_split;
-  int n_cols;
-  float* partial;                   // [splits][M][n_cols]
+  int splits;
+  int row_tiles;
+  float* partial;                   // [tiles][splits][BN][BM]
+  uint32_t* counters;               // [tiles]
+  const int32_t* pos;
+  const int64_t* dst;
+  int head_dim;
+  double inv_freq[64];
   unsigned long long* keys;         // argmax mode: [M]
   uint32_t* status;
 };
@@ -60,6 +96,7 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
   constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;
   constexpr uint32_t IDESC = idesc_bf16(BM, BN);
   static_assert(STAGE % 1024 == 0, "stages must stay 1024-byte aligned");
+  static_assert(ARGMAX || BN * SROW * 4 <= STAGES * STAGE, "staging tile must fit the ring");
 
   extern __shared__ uint8_t dsmem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -69,24 +106,28 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
   __shared__ __align__(8) uint64_t acc_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
+  __shared__ int s_last;
   __shared__ unsigned long long red[ARGMAX ? 4 : 1][ARGMAX ? BN : 1];
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
 
-  // Which weight segment this row tile belongs to.
+  // Which segment this row tile belongs to.
   const int tile = blockIdx.x;
-  int seg = 0;
-  while (seg + 1 < p.nseg && tile >= p.seg_tile_begin[seg + 1]) ++seg;
-  const int row0 = (tile - p.seg_tile_begin[seg]) * BM;
-  const int seg_rows = p.seg_rows[seg];
+  int sg = 0;
+  while (sg + 1 < p.nseg && tile >= p.seg[sg + 1].tile_begin) ++sg;
+  const Seg& S = p.seg[sg];
+  const int pair = S.pair;
+  const int row0 = (tile - S.tile_begin) * (pair ? BM / 2 : BM);   // first output feature
   const int tok0 = blockIdx.y * BN;
   const int kb0 = blockIdx.z * p.kb_per_split;
   const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
   const int nkb = kb1 - kb0;
-  const CUtensorMap* tmw = seg == 0 ? &p.tm_w0 : (seg == 1 ? &p.tm_w1 : &p.tm_w2);
+  const CUtensorMap* tma = &p.tm[S.map];
+  const CUtensorMap* tmb = pair ? &p.tm[S.map + 1] : nullptr;
 
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
@@ -94,7 +135,8 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
     mbar_init(&acc_bar, 1);
     abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(tmw);
+    tma_prefetch_desc(tma);
+    if (tmb) tma_prefetch_desc(tmb);
     tma_prefetch_desc(&p.tm_x);
   }
   if (warp == 2) tmem_alloc(&tmem_slot, TMEM_COLS);
@@ -102,22 +144,41 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  if (tid == 0) pdl_launch();
+
+  auto load_w = [&](int i, uint8_t* sa) {
+    const int kc = (kb0 + i) * BK;
+    if (pair) {
+      tma_load_2d(sa, tma, &full_bar[i % STAGES], kc, row0);
+      tma_load_2d(sa + A_BYTES / 2, tmb, &full_bar[i % STAGES], kc, row0);
+    } else {
+      tma_load_2d(sa, tma, &full_bar[i % STAGES], kc, row0);
+    }
+  };
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
-    int issued = 0;
-    for (int i = 0; i < nkb; ++i) {
+    // weights of the first stages before the dependency wait (no earlier
+    // kernel writes weights), activations after it
+    const int npre = min(STAGES, nkb);
+    for (int i = 0; i < npre; ++i) {
+      mbar_arrive_expect_tx(&full_bar[i], STAGE);
+      load_w(i, smem + i * STAGE);
+    }
+    pdl_wait();
+    for (int i = 0; i < npre; ++i)
+      tma_load_2d(smem + i * STAGE + A_BYTES, &p.tm_x, &full_bar[i], (kb0 + i) * BK, tok0);
+    int issued = npre;
+    for (int i = npre; i < nkb; ++i) {
       const int s = i % STAGES;
-      if (i >= STAGES) {
-        if (!mbar_wait(&empty_bar[s], ((i / STAGES) & 1) ^ 1, p.status, 11)) {
-          abort_flag = 1;
-          break;
-        }
+      if (!mbar_wait(&empty_bar[s], ((i / STAGES) & 1) ^ 1, p.status, 11)) {
+        abort_flag = 1;
+        break;
       }
       if (abort_flag) break;
       uint8_t* sa = smem + s * STAGE;
       mbar_arrive_expect_tx(&full_bar[s], STAGE);
-      tma_load_2d(sa, tmw, &full_bar[s], (kb0 + i) * BK, row0);
+      load_w(i, sa);
       tma_load_2d(sa + A_BYTES, &p.tm_x, &full_bar[s], (kb0 + i) * BK, tok0);
       ++issued;
     }
@@ -153,29 +214,21 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
   // ---------------- epilogue
   const bool ok = mbar_wait(&acc_bar, 0, p.status, 14);
   tc_fence_after();
+  pdl_wait();
   const bool live = ok && !abort_flag;
-  const int row = row0 + warp * 32 + lane;
   const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  if (live) {
+
+  if constexpr (ARGMAX) {
+    const int row = row0 + tid;
+    if (live) {
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 16) {
-      float v[16];
-      tmem_ld16(lane_addr + c, v);
-      if constexpr (!ARGMAX) {
-        if (row < seg_rows) {
-          float* dst = p.partial + (static_cast<size_t>(blockIdx.z) * p.M) * p.n_cols +
-                       p.seg_col0[seg] + row;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int t = tok0 + c + j;
-            if (t < p.M) dst[static_cast<size_t>(t) * p.n_cols] = v[j];
-          }
-        }
-      } else {
+      for (int c = 0; c < BN; c += 16) {
+        float v[16];
+        tmem_ld16(lane_addr + c, v);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           unsigned long long key = 0ull;
-          if (row < seg_rows && tok0 + c + j < p.M) {
+          if (row < S.rows && tok0 + c + j < p.M) {
             if (!isfinite(v[j])) report(p.status, DFLASH_ENUMERIC, 15);
             key = argmax_key(v[j], static_cast<uint32_t>(row));
           }
@@ -184,16 +237,104 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
         }
       }
     }
-  }
-  if constexpr (ARGMAX) {
     __syncthreads();
     if (live) {
-      for (int j = threadIdx.x; j < BN; j += blockDim.x) {
+      for (int j = tid; j < BN; j += blockDim.x) {
         unsigned long long k = red[0][j];
 #pragma unroll
         for (int w = 1; w < 4; ++w) k = red[w][j] > k ? red[w][j] : k;
         const int t = tok0 + j;
         if (t < p.M && k != 0ull) atomicMax(p.keys + t, k);
+      }
+    }
+  } else {
+    float* st = reinterpret_cast<float*>(smem);        // staging [BN][SROW]
+    const int tile_lin = blockIdx.y * p.row_tiles + blockIdx.x;
+    bool do_op = live;
+    if (live) {
+      if (p.splits == 1) {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          float v[16];
+          tmem_ld16(lane_addr + c, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) st[(c + j) * SROW + tid] = v[j];
+        }
+      } else {
+        float* mine = p.partial +
+                      (static_cast<size_t>(tile_lin) * p.splits + blockIdx.z) * BN * BM;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          float v[16];
+          tmem_ld16(lane_addr + c, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) mine[(c + j) * BM + tid] = v[j];
+        }
+        __threadfence();
+      }
+    }
+    if (p.splits > 1) {
+      __syncthreads();
+      if (tid == 0) {
+        const uint32_t prev = live ? atomicAdd(p.counters + tile_lin, 1u) : 0u;
+        s_last = live && prev == static_cast<uint32_t>(p.splits - 1);
+      }
+      __syncthreads();
+      do_op = s_last != 0;
+      if (do_op) {
+        __threadfence();
+        const float* base = p.partial + static_cast<size_t>(tile_lin) * p.splits * BN * BM;
+#pragma unroll 1
+        for (int j = 0; j < BN; ++j) {
+          float acc = 0.f;
+          for (int s = 0; s < p.splits; ++s) acc += __ldcg(base + (s * BN + j) * BM + tid);
+          st[j * SROW + tid] = acc;
+        }
+        if (tid == 0) p.counters[tile_lin] = 0u;
+      }
+    }
+    __syncthreads();
+    if (do_op) {
+      if (S.op == EPI_SWIGLU) {
+        const int r = tid & 63;
+        const int f = row0 + r;
+        for (int j = tid >> 6; j < BN; j += 2) {
+          const int t = tok0 + j;
+          if (f < S.rows && t < p.M) {
+            const float g = st[j * SROW + r], u = st[j * SROW + r + 64];
+            const float a = g / (1.f + __expf(-g)) * u;
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out);
+            o[static_cast<int64_t>(t) * S.out_stride + f] = __float2bfloat16_rn(a);
+          }
+        }
+      } else {
+        const int f = row0 + tid;
+        const int d = p.head_dim, half = d >> 1;
+        const int i = tid % d;
+        const int prt = i < half ? tid + half : tid - half;
+        const int fi = i < half ? i : i - half;
+        const double invf = S.rope ? p.inv_freq[fi] : 0.0;
+#pragma unroll 1
+        for (int j = 0; j < BN; ++j) {
+          const int t = tok0 + j;
+          if (f >= S.rows || t >= p.M) continue;
+          float v = st[j * SROW + tid];
+          if (S.op == EPI_RESID) {
+            float* h = static_cast<float*>(S.out) + static_cast<int64_t>(t) * S.out_stride + f;
+            *h += v;
+            continue;
+          }
+          if (S.rope) {
+            const float pv = st[j * SROW + prt];
+            double ang = static_cast<double>(p.pos[t]) * invf;
+            ang -= 6.283185307179586 * rint(ang * 0.15915494309189535);
+            float sn, cs;
+            sincosf(static_cast<float>(ang), &sn, &cs);
+            v = i < half ? v * cs - pv * sn : v * cs + pv * sn;
+          }
+          const int64_t orow = S.use_dst ? p.dst[t] : t;
+          static_cast<__nv_bfloat16*>(S.out)[orow * S.out_stride + f] = __float2bfloat16_rn(v);
+        }
       }
     }
   }
@@ -215,9 +356,7 @@ cudaError_t launch(const Params& p, dim3 grid, cudaStream_t st) {
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  gemm_kernel<BN, STAGES, ARGMAX><<<grid, 128, SMEM, st>>>(p);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(gemm_kernel<BN, STAGES, ARGMAX>, grid, dim3(128), SMEM, st, p);
 }
 
 // Ring depth per token tile: small tiles keep two CTAs per SM resident.
@@ -245,17 +384,18 @@ inline int ctas_per_sm(int bn) { return bn <= 64 ? 2 : 1; }
 }  // namespace tc
 
 // ===========================================================================
-// SIMT kernel (fp32 models): 64 weight rows x 32 tokens per CTA
+// SIMT kernel (fp32 models): 64 weight rows x 32 tokens per CTA, fp32
+// partials reduced by a finish kernel
 // ===========================================================================
 namespace simt {
 
 constexpr int TR = 64, TT = 32, TK = 32;
 
 struct Params {
-  const void* w[kMaxSegs];
-  int seg_tile_begin[kMaxSegs + 1];
-  int seg_rows[kMaxSegs];
-  int seg_col0[kMaxSegs];
+  const void* w[2 * kMaxSegs];
+  int seg_tile_begin[2 * kMaxSegs + 1];
+  int seg_rows[2 * kMaxSegs];
+  int seg_col0[2 * kMaxSegs];
   int nseg;
   const void* x;
   int M, K;
@@ -266,8 +406,8 @@ struct Params {
   uint32_t* status;
 };
 
-template <typename T, bool ARGMAX>
-__global__ void __launch_bounds__(256) gemm_kernel(const Params p) {
+template <bool ARGMAX>
+__global__ void __launch_bounds__(256) gemm_kernel(const __grid_constant__ Params p) {
   __shared__ float ws[TK][TR + 1];
   __shared__ float xs[TK][TT + 1];
   __shared__ unsigned long long red[16][TT];
@@ -276,24 +416,26 @@ __global__ void __launch_bounds__(256) gemm_kernel(const Params p) {
   while (seg + 1 < p.nseg && tile >= p.seg_tile_begin[seg + 1]) ++seg;
   const int row0 = (tile - p.seg_tile_begin[seg]) * TR;
   const int rows = p.seg_rows[seg];
-  const T* W = static_cast<const T*>(p.w[seg]);
-  const T* X = static_cast<const T*>(p.x);
+  const float* W = static_cast<const float*>(p.w[seg]);
+  const float* X = static_cast<const float*>(p.x);
   const int tok0 = blockIdx.y * TT;
   const int k0 = blockIdx.z * p.k_per_split;
   const int k1 = min(p.K, k0 + p.k_per_split);
   const int tid = threadIdx.x;
   const int ty = tid >> 4, tx = tid & 15;   // rows ty + 16i, tokens tx + 16j
+  pdl_wait();
+  if (tid == 0) pdl_launch();
   float acc[4][2] = {};
   for (int kk = k0; kk < k1; kk += TK) {
     for (int e = tid; e < TR * TK; e += 256) {
       const int r = e / TK, k = e % TK;
       const int gr = row0 + r, gk = kk + k;
-      ws[k][r] = (gr < rows && gk < k1) ? to_f(W[static_cast<size_t>(gr) * p.K + gk]) : 0.f;
+      ws[k][r] = (gr < rows && gk < k1) ? W[static_cast<size_t>(gr) * p.K + gk] : 0.f;
     }
     for (int e = tid; e < TT * TK; e += 256) {
       const int t = e / TK, k = e % TK;
       const int gt = tok0 + t, gk = kk + k;
-      xs[k][t] = (gt < p.M && gk < k1) ? to_f(X[static_cast<size_t>(gt) * p.K + gk]) : 0.f;
+      xs[k][t] = (gt < p.M && gk < k1) ? X[static_cast<size_t>(gt) * p.K + gk] : 0.f;
     }
     __syncthreads();
 #pragma unroll 8
@@ -344,6 +486,71 @@ __global__ void __launch_bounds__(256) gemm_kernel(const Params p) {
   }
 }
 
+// Fixed-order split reduction + epilogue op over [splits][M][n_cols].
+struct FinishSeg {
+  int op, rows, col0, rope, use_dst, up_col0;
+  int64_t out_stride;
+  void* out;
+};
+struct FinishParams {
+  FinishSeg seg[kMaxSegs];
+  int nseg;
+  int out_cols;
+  int64_t M;
+  int n_cols;
+  int splits;
+  const float* partial;
+  const int32_t* pos;
+  const int64_t* dst;
+  int head_dim;
+  double inv_freq[64];
+};
+
+__global__ void __launch_bounds__(256) finish_kernel(const __grid_constant__ FinishParams p) {
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
+  const int64_t total = p.M * p.out_cols;
+  const size_t split_stride = static_cast<size_t>(p.M) * p.n_cols;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = idx / p.out_cols;
+    int c = static_cast<int>(idx - m * p.out_cols);
+    int s = 0;
+    while (c >= p.seg[s].rows) c -= p.seg[s++].rows;
+    const FinishSeg& sg = p.seg[s];
+    const float* src = p.partial + static_cast<size_t>(m) * p.n_cols + sg.col0;
+    float v = 0.f;
+    for (int k = 0; k < p.splits; ++k) v += src[k * split_stride + c];
+    if (sg.op == EPI_RESID) {
+      float* h = static_cast<float*>(sg.out) + m * sg.out_stride + c;
+      *h = *h + v;
+      continue;
+    }
+    if (sg.op == EPI_SWIGLU) {
+      const float* up = p.partial + static_cast<size_t>(m) * p.n_cols + sg.up_col0;
+      float u = 0.f;
+      for (int k = 0; k < p.splits; ++k) u += up[k * split_stride + c];
+      static_cast<float*>(sg.out)[m * sg.out_stride + c] = v / (1.f + expf(-v)) * u;
+      continue;
+    }
+    if (sg.rope) {
+      const int d = p.head_dim, half = d >> 1;
+      const int i = c % d;
+      const int pc = i < half ? c + half : c - half;
+      float pv = 0.f;
+      for (int k = 0; k < p.splits; ++k) pv += src[k * split_stride + pc];
+      const int fi = i < half ? i : i - half;
+      double ang = static_cast<double>(p.pos[m]) * p.inv_freq[fi];
+      ang -= 6.283185307179586 * rint(ang * 0.15915494309189535);
+      float sn, cs;
+      sincosf(static_cast<float>(ang), &sn, &cs);
+      v = i < half ? v * cs - pv * sn : v * cs + pv * sn;
+    }
+    const int64_t orow = sg.use_dst ? p.dst[m] : m;
+    static_cast<float*>(sg.out)[orow * sg.out_stride + c] = v;
+  }
+}
+
 }  // namespace simt
 
 // ===========================================================================
@@ -369,7 +576,9 @@ EncodeFn get_encode() {
   return fn;
 }
 
-int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+void fill_inv_freq(double theta, int d, double* inv) {
+  for (int i = 0; i < d / 2 && i < 64; ++i) inv[i] = std::pow(theta, -2.0 * i / d);
+}
 
 }  // namespace
 
@@ -388,104 +597,169 @@ bool encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner,
   return r == CUDA_SUCCESS;
 }
 
-GemmPlan plan_gemm(int dtype, const int* seg_rows, int nseg, int64_t M, int K) {
+GemmPlan plan_gemm(const GemmJob& job) {
   GemmPlan pl{};
-  pl.n_cols = 0;
-  int row_tiles = 0;
-  const int tr = dtype == DFLASH_BF16 ? tc::BM : simt::TR;
-  for (int s = 0; s < nseg; ++s) {
-    pl.n_cols += seg_rows[s];
-    row_tiles += ceil_div(seg_rows[s], tr);
-  }
-  int kb_total, target;
-  if (dtype == DFLASH_BF16) {
+  const int64_t M = job.M;
+  int n_cols = 0;
+  if (job.dtype == DFLASH_BF16) {
+    for (int s = 0; s < job.nseg; ++s)
+      pl.row_tiles += job.seg[s].op == EPI_SWIGLU ? ceil_div(job.seg[s].rows, tc::BM / 2)
+                                                  : ceil_div(job.seg[s].rows, tc::BM);
     pl.bn = tc::pick_bn(M);
-    kb_total = ceil_div(K, tc::BK);
-    target = kNumSMs * tc::ctas_per_sm(pl.bn);
-  } else {
-    pl.bn = simt::TT;
-    kb_total = ceil_div(K, simt::TK);
-    target = kNumSMs * 4;
+    pl.tok_tiles = ceil_div(M, pl.bn);
+    const int kb_total = ceil_div(job.K, tc::BK);
+    const int tiles = pl.row_tiles * pl.tok_tiles;
+    int splits = 1;
+    if (pl.bn <= 64) {
+      // weight streaming: about two CTAs per SM in flight
+      const int target = kNumSMs * tc::ctas_per_sm(pl.bn);
+      if (tiles < target) splits = std::min(kb_total, ceil_div(target, tiles));
+    } else if (tiles * 2 < kNumSMs) {
+      // tensor-bound: split only when fewer than half the SMs have a tile
+      splits = std::min(kb_total, ceil_div(kNumSMs, tiles));
+    }
+    splits = std::max(1, std::min(splits, 32));
+    pl.kb_per_split = ceil_div(kb_total, splits);
+    pl.splits = ceil_div(kb_total, pl.kb_per_split);
+    pl.partial_floats = pl.splits > 1 ? static_cast<size_t>(tiles) * pl.splits * pl.bn * tc::BM
+                                      : 0;
+    pl.counters = pl.splits > 1 ? tiles : 0;
+    return pl;
   }
-  const int tiles = row_tiles * ceil_div(M, pl.bn);
-  int splits = 1;
-  if (tiles < target) splits = std::min(kb_total, ceil_div(target, tiles));
+  for (int s = 0; s < job.nseg; ++s) {
+    const int mats = job.seg[s].op == EPI_SWIGLU ? 2 : 1;
+    n_cols += mats * job.seg[s].rows;
+    pl.row_tiles += mats * ceil_div(job.seg[s].rows, simt::TR);
+  }
+  pl.bn = simt::TT;
+  pl.tok_tiles = ceil_div(M, pl.bn);
+  const int kb_total = ceil_div(job.K, simt::TK);
+  const int tiles = pl.row_tiles * pl.tok_tiles;
+  const int target = kNumSMs * 4;
+  int splits = tiles < target ? std::min(kb_total, ceil_div(target, tiles)) : 1;
   splits = std::max(1, std::min(splits, 32));
   pl.kb_per_split = ceil_div(kb_total, splits);
   pl.splits = ceil_div(kb_total, pl.kb_per_split);
+  pl.partial_floats = static_cast<size_t>(pl.splits) * M * n_cols;
+  pl.counters = 0;
   return pl;
 }
 
-cudaError_t launch_gemm_partial(int dtype, const GemmSeg* segs, int nseg, const void* X,
-                                int64_t M, int K, const GemmPlan& pl, float* partial,
-                                uint32_t* status, cudaStream_t st) {
-  if (M <= 0) return cudaSuccess;
-  if (dtype == DFLASH_BF16) {
-    tc::Params p{};
-    CUtensorMap* maps[3] = {&p.tm_w0, &p.tm_w1, &p.tm_w2};
-    int tiles = 0;
-    for (int s = 0; s < nseg; ++s) {
-      if (!encode_tmap_bf16_2d(maps[s], segs[s].w, K, segs[s].rows, tc::BK, tc::BM))
-        return cudaErrorInvalidValue;
-      p.seg_tile_begin[s] = tiles;
-      p.seg_rows[s] = segs[s].rows;
-      p.seg_col0[s] = s == 0 ? 0 : p.seg_col0[s - 1] + segs[s - 1].rows;
-      tiles += ceil_div(segs[s].rows, tc::BM);
-    }
-    p.seg_tile_begin[nseg] = tiles;
-    if (!encode_tmap_bf16_2d(&p.tm_x, X, K, M, tc::BK, pl.bn)) return cudaErrorInvalidValue;
-    p.nseg = nseg;
-    p.M = static_cast<int>(M);
-    p.kb_total = ceil_div(K, tc::BK);
-    p.kb_per_split = pl.kb_per_split;
-    p.n_cols = pl.n_cols;
-    p.partial = partial;
-    p.status = status;
-    dim3 grid(tiles, ceil_div(M, pl.bn), pl.splits);
-    return tc::dispatch<false>(pl.bn, p, grid, st);
-  }
+static cudaError_t launch_gemm_simt(const GemmJob& job, const GemmPlan& pl, float* partial,
+                                    uint32_t* status, cudaStream_t st) {
   simt::Params p{};
-  int tiles = 0;
-  for (int s = 0; s < nseg; ++s) {
-    p.w[s] = segs[s].w;
-    p.seg_tile_begin[s] = tiles;
-    p.seg_rows[s] = segs[s].rows;
-    p.seg_col0[s] = s == 0 ? 0 : p.seg_col0[s - 1] + segs[s - 1].rows;
-    tiles += ceil_div(segs[s].rows, simt::TR);
+  simt::FinishParams f{};
+  int tiles = 0, col = 0, n = 0;
+  for (int s = 0; s < job.nseg; ++s) {
+    const GemmOut& o = job.seg[s];
+    const int mats = o.op == EPI_SWIGLU ? 2 : 1;
+    f.seg[s] = {o.op, o.rows, col, o.rope, o.use_dst, o.op == EPI_SWIGLU ? col + o.rows : 0,
+                o.out_stride, o.out};
+    for (int m = 0; m < mats; ++m) {
+      p.w[n] = m == 0 ? o.w0 : o.w1;
+      p.seg_tile_begin[n] = tiles;
+      p.seg_rows[n] = o.rows;
+      p.seg_col0[n] = col;
+      tiles += ceil_div(o.rows, simt::TR);
+      col += o.rows;
+      ++n;
+    }
   }
-  p.seg_tile_begin[nseg] = tiles;
-  p.nseg = nseg;
-  p.x = X;
-  p.M = static_cast<int>(M);
-  p.K = K;
+  p.seg_tile_begin[n] = tiles;
+  p.nseg = n;
+  p.x = job.x;
+  p.M = static_cast<int>(job.M);
+  p.K = job.K;
   p.k_per_split = pl.kb_per_split * simt::TK;
-  p.n_cols = pl.n_cols;
+  p.n_cols = col;
   p.partial = partial;
   p.status = status;
-  dim3 grid(tiles, ceil_div(M, simt::TT), pl.splits);
-  simt::gemm_kernel<float, false><<<grid, 256, 0, st>>>(p);
-  count_launch();
-  return cudaGetLastError();
+  cudaError_t e = launch_k(simt::gemm_kernel<false>, dim3(tiles, pl.tok_tiles, pl.splits),
+                           dim3(256), 0, st, p);
+  if (e != cudaSuccess) return e;
+  f.nseg = job.nseg;
+  f.out_cols = 0;
+  for (int s = 0; s < job.nseg; ++s) f.out_cols += job.seg[s].rows;
+  f.M = job.M;
+  f.n_cols = col;
+  f.splits = pl.splits;
+  f.partial = partial;
+  f.pos = job.pos;
+  f.dst = job.dst;
+  f.head_dim = job.head_dim;
+  fill_inv_freq(job.theta, std::max(job.head_dim, 2), f.inv_freq);
+  const int64_t total = job.M * f.out_cols;
+  const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, kNumSMs * 16));
+  return launch_k(simt::finish_kernel, dim3(grid), dim3(256), 0, st, f);
+}
+
+cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& pl, float* partial,
+                        uint32_t* counters, uint32_t* status, cudaStream_t st) {
+  if (job.M <= 0) return cudaSuccess;
+  if (job.dtype != DFLASH_BF16) return launch_gemm_simt(job, pl, partial, status, st);
+  tc::Params p{};
+  int tiles = 0, maps = 0;
+  for (int s = 0; s < job.nseg; ++s) {
+    const GemmOut& o = job.seg[s];
+    tc::Seg& S = p.seg[s];
+    S.tile_begin = tiles;
+    S.map = maps;
+    S.rows = o.rows;
+    S.pair = o.op == EPI_SWIGLU;
+    S.op = o.op;
+    S.rope = o.rope;
+    S.use_dst = o.use_dst;
+    S.out_stride = o.out_stride;
+    S.out = o.out;
+    if (S.pair) {
+      if (!encode_tmap_bf16_2d(&p.tm[maps++], o.w0, job.K, o.rows, tc::BK, tc::BM / 2) ||
+          !encode_tmap_bf16_2d(&p.tm[maps++], o.w1, job.K, o.rows, tc::BK, tc::BM / 2))
+        return cudaErrorInvalidValue;
+      tiles += ceil_div(o.rows, tc::BM / 2);
+    } else {
+      if (!encode_tmap_bf16_2d(&p.tm[maps++], o.w0, job.K, o.rows, tc::BK, tc::BM))
+        return cudaErrorInvalidValue;
+      tiles += ceil_div(o.rows, tc::BM);
+    }
+    if (maps > 4) return cudaErrorInvalidValue;
+  }
+  if (!encode_tmap_bf16_2d(&p.tm_x, job.x, job.K, job.M, tc::BK, pl.bn))
+    return cudaErrorInvalidValue;
+  p.nseg = job.nseg;
+  p.M = static_cast<int>(job.M);
+  p.kb_total = ceil_div(job.K, tc::BK);
+  p.kb_per_split = pl.kb_per_split;
+  p.splits = pl.splits;
+  p.row_tiles = tiles;
+  p.partial = partial;
+  p.counters = counters;
+  p.pos = job.pos;
+  p.dst = job.dst;
+  p.head_dim = job.head_dim > 0 ? job.head_dim : 128;
+  fill_inv_freq(job.theta, p.head_dim, p.inv_freq);
+  p.status = status;
+  dim3 grid(tiles, pl.tok_tiles, pl.splits);
+  return tc::dispatch<false>(pl.bn, p, grid, st);
 }
 
 cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X, int64_t M,
                                  int K, unsigned long long* keys, uint32_t* status,
                                  cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(keys, 0, sizeof(unsigned long long) * M, st);
-  if (e != cudaSuccess) return e;
   if (dtype == DFLASH_BF16) {
     tc::Params p{};
-    if (!encode_tmap_bf16_2d(&p.tm_w0, W, K, V, tc::BK, tc::BM)) return cudaErrorInvalidValue;
+    if (!encode_tmap_bf16_2d(&p.tm[0], W, K, V, tc::BK, tc::BM)) return cudaErrorInvalidValue;
     const int bn = tc::pick_bn(M);
     if (!encode_tmap_bf16_2d(&p.tm_x, X, K, M, tc::BK, bn)) return cudaErrorInvalidValue;
-    p.seg_tile_begin[0] = 0;
-    p.seg_tile_begin[1] = ceil_div(V, tc::BM);
-    p.seg_rows[0] = V;
+    p.seg[0].tile_begin = 0;
+    p.seg[0].map = 0;
+    p.seg[0].rows = V;
     p.nseg = 1;
     p.M = static_cast<int>(M);
     p.kb_total = ceil_div(K, tc::BK);
     p.kb_per_split = p.kb_total;
+    p.splits = 1;
+    p.row_tiles = ceil_div(V, tc::BM);
     p.keys = keys;
     p.status = status;
     dim3 grid(ceil_div(V, tc::BM), ceil_div(M, bn), 1);
@@ -503,82 +777,8 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X,
   p.k_per_split = K;
   p.keys = keys;
   p.status = status;
-  dim3 grid(ceil_div(V, simt::TR), ceil_div(M, simt::TT), 1);
-  simt::gemm_kernel<float, true><<<grid, 256, 0, st>>>(p);
-  count_launch();
-  return cudaGetLastError();
-}
-
-// ===========================================================================
-// finish: fixed-order split reduction + epilogue op
-// ===========================================================================
-template <typename T>
-__global__ void __launch_bounds__(256) finish_kernel(const EpiParams p) {
-  // output columns of all active segments, concatenated
-  int out_cols = 0;
-  for (int s = 0; s < p.nseg; ++s)
-    if (p.seg[s].op != EPI_NONE) out_cols += p.seg[s].rows;
-  const int64_t total = p.M * out_cols;
-  const size_t split_stride = static_cast<size_t>(p.M) * p.n_cols;
-  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t m = idx / out_cols;
-    int c = static_cast<int>(idx % out_cols);
-    int s = 0;
-    while (p.seg[s].op == EPI_NONE || c >= p.seg[s].rows) {
-      if (p.seg[s].op != EPI_NONE) c -= p.seg[s].rows;
-      ++s;
-    }
-    const EpiSeg& sg = p.seg[s];
-    const float* src = p.partial + static_cast<size_t>(m) * p.n_cols + sg.col0;
-    float v = 0.f;
-    for (int k = 0; k < p.splits; ++k) v += src[k * split_stride + c];
-    if (sg.op == EPI_RESID) {
-      float* h = static_cast<float*>(sg.out) + m * sg.out_stride + c;
-      *h = *h + v;
-      continue;
-    }
-    if (sg.op == EPI_SWIGLU) {
-      const float* up = p.partial + static_cast<size_t>(m) * p.n_cols + p.seg[s + 1].col0;
-      float u = 0.f;
-      for (int k = 0; k < p.splits; ++k) u += up[k * split_stride + c];
-      const float a = v / (1.f + __expf(-v)) * u;
-      static_cast<T*>(sg.out)[m * sg.out_stride + c] = from_f<T>(a);
-      continue;
-    }
-    // EPI_STORE
-    if (sg.rope) {
-      const int d = p.head_dim, half = d >> 1;
-      const int i = c % d;
-      const int pc = i < half ? c + half : c - half;
-      float pv = 0.f;
-      for (int k = 0; k < p.splits; ++k) pv += src[k * split_stride + pc];
-      const int fi = i < half ? i : i - half;
-      double ang = static_cast<double>(p.pos[m]) * p.inv_freq[fi];
-      ang -= 6.283185307179586 * rint(ang * 0.15915494309189535);
-      float sn, cs;
-      sincosf(static_cast<float>(ang), &sn, &cs);
-      v = i < half ? v * cs - pv * sn : v * cs + pv * sn;
-    }
-    const int64_t orow = sg.use_dst ? p.dst_row[m] : m;
-    static_cast<T*>(sg.out)[orow * sg.out_stride + c] = from_f<T>(v);
-  }
-}
-
-cudaError_t launch_gemm_finish(const EpiParams& p, cudaStream_t st) {
-  int out_cols = 0;
-  for (int s = 0; s < p.nseg; ++s)
-    if (p.seg[s].op != EPI_NONE) out_cols += p.seg[s].rows;
-  const int64_t total = p.M * out_cols;
-  if (total <= 0) return cudaSuccess;
-  const int64_t want = (total + 255) / 256;
-  const int grid = static_cast<int>(std::min<int64_t>(want, kNumSMs * 16));
-  if (p.out_bf16)
-    finish_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(p);
-  else
-    finish_kernel<float><<<grid, 256, 0, st>>>(p);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(simt::gemm_kernel<true>, dim3(ceil_div(V, simt::TR), ceil_div(M, simt::TT), 1),
+                  dim3(256), 0, st, p);
 }
 
 }  // namespace dfl

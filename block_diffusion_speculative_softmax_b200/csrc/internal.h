@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/dflash.h"
 
 namespace dfl {
@@ -19,63 +21,62 @@ constexpr int kMaxBlock = 32;
 void count_launch(int n = 1);
 
 // ---------------------------------------------------------------- GEMM
-// Partial products of a "weight-stationary" GEMM: for every segment s
-// (a weight matrix W_s [rows_s][K]) and every token m of X [M][K]:
-//   partial[split][m][col0_s + r] = sum_{k in split} X[m][k] * W_s[r][k].
-struct GemmSeg {
-  const void* w;
-  int rows;
-};
+// Weight-stationary GEMM with a fused epilogue.  For every output segment s
+// (a weight matrix W_s [rows_s][K], or a gate/up pair for SwiGLU) and every
+// token m of X [M][K]:  y[m][r] = sum_k X[m][k] W_s[r][k], then the
+// segment's epilogue op writes the result.
 constexpr int kMaxSegs = 3;
+enum EpiOp { EPI_NONE = 0, EPI_STORE = 1, EPI_RESID = 2, EPI_SWIGLU = 3 };
+
+struct GemmOut {
+  const void* w0;      // weights [rows][K]; the gate matrix for EPI_SWIGLU
+  const void* w1;      // EPI_SWIGLU: the up matrix [rows][K]
+  int rows;            // output features of the segment
+  int op;              // EPI_STORE: out = y (dtype), optional RoPE and row scatter
+                       // EPI_RESID: fp32 out += y
+                       // EPI_SWIGLU: out = silu(y_gate) * y_up (dtype)
+  int rope;            // EPI_STORE: rotate-half RoPE over heads of head_dim
+  void* out;
+  int64_t out_stride;  // elements between output rows
+  int use_dst;         // EPI_STORE: token m goes to output row dst[m]
+};
+
+struct GemmJob {
+  GemmOut seg[kMaxSegs];
+  int nseg = 0;
+  const void* x = nullptr;   // [M][K] dtype
+  int64_t M = 0;
+  int K = 0;
+  int dtype = 0;
+  const int32_t* pos = nullptr;   // RoPE positions [M]
+  const int64_t* dst = nullptr;   // [M]
+  int head_dim = 0;
+  double theta = 1e6;
+};
 
 struct GemmPlan {
-  int bn;          // token tile (tcgen05 N) or SIMT token tile
-  int splits;      // K splits
-  int kb_per_split;
-  int n_cols;      // sum of segment rows
+  int bn;            // token tile
+  int row_tiles;     // tiles along the output features (all segments)
+  int tok_tiles;
+  int splits;        // K splits
+  int kb_per_split;  // k-blocks per split
+  size_t partial_floats;
+  size_t counters;
 };
 
-// Split plan for M tokens, K reduction length, given segments.  Same plan
-// for workspace sizing and for the launch.
-GemmPlan plan_gemm(int dtype, const int* seg_rows, int nseg, int64_t M, int K);
+GemmPlan plan_gemm(const GemmJob& job);
+// Launch (one kernel for bf16; GEMM + finish for fp32).  `partial` and
+// `counters` are workspace regions of plan.partial_floats floats and
+// plan.counters words; counters must be zero (they are left zero).
+cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& plan, float* partial,
+                        uint32_t* counters, uint32_t* status, cudaStream_t st);
 
-cudaError_t launch_gemm_partial(int dtype, const GemmSeg* segs, int nseg,
-                                const void* X, int64_t M, int K,
-                                const GemmPlan& plan, float* partial,
-                                uint32_t* status, cudaStream_t st);
-
-// LM head: keys[m] = max over v of argmax_key(x[m] . W[v], v).
+// LM head: keys[m] = max over v of argmax_key(x[m] . W[v], v).  keys must be
+// zero on entry (launch_argmax_finish leaves them zero).
 cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V,
                                  const void* X, int64_t M, int K,
                                  unsigned long long* keys, uint32_t* status,
                                  cudaStream_t st);
-
-// ---------------------------------------------------------------- epilogues
-enum EpiOp { EPI_NONE = 0, EPI_STORE = 1, EPI_RESID = 2, EPI_SWIGLU = 3 };
-struct EpiSeg {
-  int op;             // EpiOp.  EPI_SWIGLU: this segment holds the gate, the
-                      // next one the up projection; writes silu(g) * u.
-  int rows;           // outputs of the segment
-  int col0;           // column of the segment in the partial buffer
-  int rope;           // rotate-half RoPE over heads of head_dim
-  void* out;          // STORE/SWIGLU: dtype [*][out_stride]; RESID: fp32
-  int64_t out_stride; // elements between output rows
-  int use_dst;        // STORE: row m goes to dst_row[m]
-};
-struct EpiParams {
-  EpiSeg seg[kMaxSegs];
-  int nseg;
-  int64_t M;
-  int n_cols;
-  int splits;
-  const float* partial;
-  const int32_t* pos;      // RoPE positions [M]
-  const int64_t* dst_row;  // [M] or null
-  int head_dim;
-  int out_bf16;
-  double inv_freq[64];
-};
-cudaError_t launch_gemm_finish(const EpiParams& p, cudaStream_t st);
 
 // ---------------------------------------------------------------- others
 cudaError_t launch_fuse(int dtype, const void* states, int64_t N, int T, int H,
@@ -92,11 +93,35 @@ cudaError_t launch_prep_rows(int R, int nb, int B, const int32_t* block_req,
                              const int64_t* ctx_off, const int64_t* new_off,
                              const int32_t* ctx_cached, int64_t n_new,
                              int32_t* blk_pos, int32_t* new_pos,
-                             int64_t* new_dst, cudaStream_t st);
-cudaError_t launch_argmax_finish(const unsigned long long* keys, int64_t M,
+                             int64_t* new_dst, uint32_t* zero, int64_t n_zero,
+                             cudaStream_t st);
+// tokens (+ max logit) from the argmax keys; resets the keys to zero.
+cudaError_t launch_argmax_finish(unsigned long long* keys, int64_t M,
                                  int B, const int32_t* block_tokens,
                                  const int32_t* known_len, int32_t* tok,
                                  float* max_logit, cudaStream_t st);
+cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t st);
+
+// Kernel launch with programmatic dependent launch enabled: the kernel may
+// start while the previous kernel on the stream finishes; every kernel of
+// this library calls pdl_wait() before touching memory the previous kernel
+// may write.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 struct AttnPlan {
   int splits;
@@ -107,11 +132,13 @@ struct AttnPlan {
 AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d,
                    int64_t max_ctx_len);
 size_t attn_ws_bytes(const AttnPlan& p, int nb, int B, int Hq, int d);
+size_t attn_counters(const AttnPlan& p, int nb, int Hkv);
+// counters: attn_counters() words, zero on entry (left zero).
 cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq,
                         int Hkv, int d, const void* q, const void* kb,
                         const void* vb, const void* kc, const void* vc,
                         const int64_t* ctx_off, const int32_t* block_req,
-                        void* out, float* ws, uint32_t* status,
+                        void* out, float* ws, uint32_t* counters, uint32_t* status,
                         cudaStream_t st);
 
 cudaError_t launch_accept(int R, int K, int B, const int32_t* draft,

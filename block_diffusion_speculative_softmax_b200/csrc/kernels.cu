@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(const T* __rest
   __shared__ float red[32][kMaxLayers];
   __shared__ float scale[kMaxLayers];
   const int tid = threadIdx.x;
+  pdl_wait();
+  if (tid == 0) pdl_launch();
   if (tid < D) {
     float mx = -INFINITY;
     for (int j = 0; j < nT; ++j) mx = fmaxf(mx, w_fuse[tid * nT + j]);
@@ -142,13 +144,14 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(const T* __rest
 }
 
 template <typename T, int MAXT, int VW>
-static void fuse_go(const void* states, int64_t N, int nT, int H, int D, const float* w_fuse,
+static cudaError_t fuse_go(const void* states, int64_t N, int nT, int H, int D, const float* w_fuse,
                     const FuseGains& g, void* fused, float eps, cudaStream_t st) {
   const int nvec = H / VecN<T, VW>::N;
   const int threads = ((nvec + 31) / 32) * 32;
   const int grid = static_cast<int>(std::min<int64_t>(N, 1 << 20));
-  fuse_rows_kernel<T, MAXT, VW><<<grid, threads, 0, st>>>(
-      static_cast<const T*>(states), N, nT, H, D, w_fuse, g, static_cast<T*>(fused), eps);
+  return launch_k(fuse_rows_kernel<T, MAXT, VW>, dim3(grid), dim3(threads), 0, st,
+                  static_cast<const T*>(states), N, nT, H, D, w_fuse, g,
+                  static_cast<T*>(fused), eps);
 }
 
 // Largest hidden size each variant covers with kFuseThreads threads.
@@ -163,13 +166,11 @@ static cudaError_t launch_fuse_t(const void* states, int64_t N, int nT, int H, i
                                  const float* w_fuse, const FuseGains& g, void* fused, float eps,
                                  cudaStream_t st) {
   if (H > fuse_max_hidden<T>(nT)) return cudaErrorInvalidValue;
-  if (nT <= 4) fuse_go<T, 4, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
-  else if (nT <= 5) fuse_go<T, 5, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
-  else if (nT <= 8) fuse_go<T, 8, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
-  else if (nT <= 9) fuse_go<T, 9, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
-  else fuse_go<T, 16, 8>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
-  count_launch();
-  return cudaGetLastError();
+  if (nT <= 4) return fuse_go<T, 4, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+  if (nT <= 5) return fuse_go<T, 5, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+  if (nT <= 8) return fuse_go<T, 8, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+  if (nT <= 9) return fuse_go<T, 9, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+  return fuse_go<T, 16, 8>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
 }
 
 int fuse_hidden_limit(int dtype, int nT) {
@@ -195,6 +196,8 @@ __global__ void embed_kernel(const T* __restrict__ embed, int H, int B,
                              const int32_t* __restrict__ block_tokens,
                              const int32_t* __restrict__ known_len, int mask_id,
                              float* __restrict__ h) {
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
   const int m = blockIdx.x;
   const int b = m / B, s = m % B;
   const int kl = known_len ? known_len[b] : 1;
@@ -209,13 +212,11 @@ cudaError_t launch_embed(int dtype, const void* embed, int H, int nb, int B,
                          float* h, cudaStream_t st) {
   if (nb <= 0) return cudaSuccess;
   if (dtype == DFLASH_BF16)
-    embed_kernel<__nv_bfloat16><<<nb * B, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(embed), H, B, block_tokens, known_len, mask_id, h);
-  else
-    embed_kernel<float><<<nb * B, 256, 0, st>>>(static_cast<const float*>(embed), H, B,
-                                                block_tokens, known_len, mask_id, h);
-  count_launch();
-  return cudaGetLastError();
+    return launch_k(embed_kernel<__nv_bfloat16>, dim3(nb * B), dim3(256), 0, st,
+                    static_cast<const __nv_bfloat16*>(embed), H, B, block_tokens, known_len,
+                    mask_id, h);
+  return launch_k(embed_kernel<float>, dim3(nb * B), dim3(256), 0, st,
+                  static_cast<const float*>(embed), H, B, block_tokens, known_len, mask_id, h);
 }
 
 // ===========================================================================
@@ -226,6 +227,8 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
                                                       const float* __restrict__ g, float eps,
                                                       T* __restrict__ x) {
   __shared__ float red[8];
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
   const int64_t m = blockIdx.x;
   const float* row = h + m * H;
   float ss = 0.f;
@@ -247,13 +250,10 @@ cudaError_t launch_rmsnorm(int dtype, const float* h, int64_t M, int H, const fl
                            void* x, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   if (dtype == DFLASH_BF16)
-    rmsnorm_kernel<__nv_bfloat16><<<static_cast<unsigned>(M), 256, 0, st>>>(
-        h, H, g, eps, static_cast<__nv_bfloat16*>(x));
-  else
-    rmsnorm_kernel<float><<<static_cast<unsigned>(M), 256, 0, st>>>(h, H, g, eps,
-                                                                    static_cast<float*>(x));
-  count_launch();
-  return cudaGetLastError();
+    return launch_k(rmsnorm_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(M)), dim3(256), 0,
+                    st, h, H, g, eps, static_cast<__nv_bfloat16*>(x));
+  return launch_k(rmsnorm_kernel<float>, dim3(static_cast<unsigned>(M)), dim3(256), 0, st, h, H,
+                  g, eps, static_cast<float*>(x));
 }
 
 // ===========================================================================
@@ -265,9 +265,13 @@ __global__ void prep_rows_kernel(int R, int nb, int B, const int32_t* __restrict
                                  const int64_t* __restrict__ new_off,
                                  const int32_t* __restrict__ ctx_cached, int64_t n_new,
                                  int32_t* __restrict__ blk_pos, int32_t* __restrict__ new_pos,
-                                 int64_t* __restrict__ new_dst) {
+                                 int64_t* __restrict__ new_dst, uint32_t* __restrict__ zero,
+                                 int64_t n_zero) {
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
   const int64_t tid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = tid; i < n_zero; i += stride) zero[i] = 0u;
   for (int64_t m = tid; m < static_cast<int64_t>(nb) * B; m += stride) {
     const int r = block_req[m / B];
     blk_pos[m] = static_cast<int32_t>(ctx_off[r + 1] - ctx_off[r] + m % B);
@@ -288,26 +292,44 @@ __global__ void prep_rows_kernel(int R, int nb, int B, const int32_t* __restrict
 cudaError_t launch_prep_rows(int R, int nb, int B, const int32_t* block_req,
                              const int64_t* ctx_off, const int64_t* new_off,
                              const int32_t* ctx_cached, int64_t n_new, int32_t* blk_pos,
-                             int32_t* new_pos, int64_t* new_dst, cudaStream_t st) {
-  const int64_t work = std::max<int64_t>(static_cast<int64_t>(nb) * B, n_new);
+                             int32_t* new_pos, int64_t* new_dst, uint32_t* zero, int64_t n_zero,
+                             cudaStream_t st) {
+  const int64_t work =
+      std::max(std::max<int64_t>(static_cast<int64_t>(nb) * B, n_new), n_zero);
   if (work <= 0) return cudaSuccess;
   const int grid = static_cast<int>(std::min<int64_t>((work + 255) / 256, kNumSMs * 8));
-  prep_rows_kernel<<<grid, 256, 0, st>>>(R, nb, B, block_req, ctx_off, new_off, ctx_cached,
-                                         n_new, blk_pos, new_pos, new_dst);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(prep_rows_kernel, dim3(grid), dim3(256), 0, st, R, nb, B, block_req, ctx_off,
+                  new_off, ctx_cached, n_new, blk_pos, new_pos, new_dst, zero, n_zero);
+}
+
+__global__ void zero_kernel(uint32_t* __restrict__ p, int64_t n) {
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[i] = 0u;
+}
+
+cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(bytes / 4);
+  if (n <= 0) return cudaSuccess;
+  const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, kNumSMs * 8));
+  return launch_k(zero_kernel, dim3(grid), dim3(256), 0, st, static_cast<uint32_t*>(p), n);
 }
 
 // ===========================================================================
 // argmax keys -> tokens (+ max logit); known slots keep their input token
 // ===========================================================================
-__global__ void argmax_finish_kernel(const unsigned long long* __restrict__ keys, int64_t M,
+__global__ void argmax_finish_kernel(unsigned long long* __restrict__ keys, int64_t M,
                                      int B, const int32_t* __restrict__ block_tokens,
                                      const int32_t* __restrict__ known_len,
                                      int32_t* __restrict__ tok, float* __restrict__ max_logit) {
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
   const int64_t m = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (m >= M) return;
   const unsigned long long k = keys[m];
+  keys[m] = 0ull;   // re-armed for the next LM-head launch
   int32_t t = static_cast<int32_t>(key_index(k));
   if (block_tokens) {
     const int64_t b = m / B;
@@ -318,14 +340,12 @@ __global__ void argmax_finish_kernel(const unsigned long long* __restrict__ keys
   if (max_logit) max_logit[m] = key_value(k);
 }
 
-cudaError_t launch_argmax_finish(const unsigned long long* keys, int64_t M, int B,
+cudaError_t launch_argmax_finish(unsigned long long* keys, int64_t M, int B,
                                  const int32_t* block_tokens, const int32_t* known_len,
                                  int32_t* tok, float* max_logit, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  argmax_finish_kernel<<<static_cast<unsigned>((M + 255) / 256), 256, 0, st>>>(
-      keys, M, B, block_tokens, known_len, tok, max_logit);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(argmax_finish_kernel, dim3(static_cast<unsigned>((M + 255) / 256)), dim3(256),
+                  0, st, keys, M, B, block_tokens, known_len, tok, max_logit);
 }
 
 // ===========================================================================
@@ -336,6 +356,8 @@ cudaError_t launch_argmax_finish(const unsigned long long* keys, int64_t M, int 
 __global__ void accept_kernel(int R, int K, int B, const int32_t* __restrict__ draft,
                               const int32_t* __restrict__ target, int32_t* __restrict__ n_acc,
                               int32_t* __restrict__ best_k, int32_t* __restrict__ out_tok) {
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= R) return;
@@ -366,10 +388,8 @@ cudaError_t launch_accept(int R, int K, int B, const int32_t* draft, const int32
                           int32_t* n_acc, int32_t* best_k, int32_t* out_tok, cudaStream_t st) {
   if (R <= 0) return cudaSuccess;
   const int wpb = 4;
-  accept_kernel<<<(R + wpb - 1) / wpb, wpb * 32, 0, st>>>(R, K, B, draft, target, n_acc, best_k,
-                                                          out_tok);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(accept_kernel, dim3((R + wpb - 1) / wpb), dim3(wpb * 32), 0, st, R, K, B, draft,
+                  target, n_acc, best_k, out_tok);
 }
 
 // ===========================================================================
@@ -380,6 +400,8 @@ cudaError_t launch_accept(int R, int K, int B, const int32_t* draft, const int32
 __global__ void d2sd_kernel(int R, int B, int K, int mask_id, const int32_t* __restrict__ base,
                             const float* __restrict__ conf, int32_t* __restrict__ known_len,
                             int32_t* __restrict__ cand, int32_t* __restrict__ block_req) {
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= R) return;
@@ -410,10 +432,8 @@ cudaError_t launch_d2sd(int R, int B, int K, int mask_id, const int32_t* base, c
                         int32_t* known_len, int32_t* cand, int32_t* block_req, cudaStream_t st) {
   if (R <= 0) return cudaSuccess;
   const int wpb = 4;
-  d2sd_kernel<<<(R + wpb - 1) / wpb, wpb * 32, 0, st>>>(R, B, K, mask_id, base, conf, known_len,
-                                                        cand, block_req);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(d2sd_kernel, dim3((R + wpb - 1) / wpb), dim3(wpb * 32), 0, st, R, B, K, mask_id,
+                  base, conf, known_len, cand, block_req);
 }
 
 // ===========================================================================
@@ -421,6 +441,7 @@ cudaError_t launch_d2sd(int R, int B, int K, int mask_id, const int32_t* base, c
 // ===========================================================================
 __global__ void wait_selftest_kernel(uint32_t* status, int64_t limit_ns) {
   __shared__ __align__(8) uint64_t bar;
+  pdl_wait();
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     fence_mbar_init();
@@ -431,9 +452,7 @@ __global__ void wait_selftest_kernel(uint32_t* status, int64_t limit_ns) {
 }
 
 cudaError_t launch_wait_selftest(uint32_t* status, int64_t limit_ns, cudaStream_t st) {
-  wait_selftest_kernel<<<1, 32, 0, st>>>(status, limit_ns);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(wait_selftest_kernel, dim3(1), dim3(32), 0, st, status, limit_ns);
 }
 
 }  // namespace dfl
