@@ -143,7 +143,8 @@ GemmJob job_swiglu(const dflash_config* c, const void* wg, const void* wu, const
 struct Layout {
   size_t h = 0, x = 0, q = 0, kb = 0, vb = 0, attn = 0, act = 0, fused = 0, partial = 0,
          attn_ws = 0, zero = 0, keys = 0, counters = 0, blk_pos = 0, new_pos = 0, new_dst = 0,
-         total = 0;
+         rope = 0, total = 0;
+  int rope_len = 0;
   size_t zero_bytes = 0;   // [keys | counters], zeroed at the start of a step
 };
 
@@ -197,7 +198,7 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
   L.fused = take(static_cast<size_t>(c->n_draft_layers) * n_new * H * e);
   L.partial = take(nd.partial_floats * 4);
   L.attn_ws = take(attn_ws_bytes(ap, nb, c->block, c->n_q_heads, c->head_dim));
-  const size_t ncount = std::max(nd.counters, attn_counters(ap, nb, c->n_kv_heads));
+  const size_t ncount = nd.counters;
   L.zero = off;
   L.keys = take(M * 8);
   L.counters = take(ncount * 4);
@@ -205,6 +206,8 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
   L.blk_pos = take(M * 4);
   L.new_pos = take(n_new * 4);
   L.new_dst = take(n_new * 8);
+  L.rope_len = static_cast<int>(max_ctx + c->block);
+  L.rope = take(static_cast<size_t>(L.rope_len) * (c->head_dim / 2) * 8);
   L.total = off;
   return L;
 }
@@ -289,7 +292,7 @@ dflash_status dflash_fuse_ctx(const dflash_config* cfg, const void* states, int6
   DFL_CHECK(g_fuse != nullptr, DFLASH_EINVAL, "g_fuse is NULL");
   for (int i = 0; i < cfg->n_draft_layers; ++i) DFL_PTR(g_fuse[i], "g_fuse[i]");
   DFL_CUDA(launch_fuse(cfg->dtype, states, n_rows, cfg->n_target_layers, cfg->hidden,
-                       cfg->n_draft_layers, w_fuse, g_fuse, fused, cfg->rms_eps,
+                       cfg->n_draft_layers, w_fuse, g_fuse, fused, cfg->rms_eps, nullptr,
                        static_cast<cudaStream_t>(stream)),
            "fusion kernel");
   return DFLASH_OK;
@@ -343,16 +346,13 @@ dflash_status dflash_block_attn(const dflash_config* cfg, int32_t n_blocks, cons
   }
   AttnPlan ap = plan_attn(cfg->dtype, n_blocks, cfg->block, cfg->n_q_heads, cfg->n_kv_heads,
                           cfg->head_dim, max_ctx_len);
-  const size_t off_cnt = align256(
-      sizeof(DevStatus) + attn_ws_bytes(ap, n_blocks, cfg->block, cfg->n_q_heads, cfg->head_dim));
-  const size_t ncnt = attn_counters(ap, n_blocks, cfg->n_kv_heads);
-  if ((s = check_ws(ws, ws_bytes, off_cnt + ncnt * 4)) != DFLASH_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  DFL_CUDA(launch_zero(at<void>(ws, off_cnt), ncnt * 4, st), "counter reset");
+  const size_t need =
+      sizeof(DevStatus) + attn_ws_bytes(ap, n_blocks, cfg->block, cfg->n_q_heads, cfg->head_dim);
+  if ((s = check_ws(ws, ws_bytes, need)) != DFLASH_OK) return s;
   DFL_CUDA(launch_attn(cfg->dtype, ap, n_blocks, cfg->block, cfg->n_q_heads, cfg->n_kv_heads,
                        cfg->head_dim, q, k_blk, v_blk, k_ctx, v_ctx, ctx_off, block_req, out,
-                       at<float>(ws, sizeof(DevStatus)), at<uint32_t>(ws, off_cnt),
-                       status_word(ws), st),
+                       at<float>(ws, sizeof(DevStatus)), status_word(ws),
+                       static_cast<cudaStream_t>(stream)),
            "attention kernel");
   return DFLASH_OK;
 }
@@ -528,11 +528,13 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
                             a->new_off, a->ctx_cached, a->n_ctx_new, blk_pos, new_pos, new_dst,
                             at<uint32_t>(ws, L.zero), static_cast<int64_t>(L.zero_bytes / 4), st),
            "row bookkeeping");
+  float2* rope_tab = at<float2>(ws, L.rope);
+  DFL_CUDA(launch_rope_table(rope_tab, L.rope_len, c->head_dim, c->rope_theta, st), "RoPE table");
   if (a->n_ctx_new > 0) {
     const float* gf[kMaxLayers];
     for (int i = 0; i < D; ++i) gf[i] = w->layers[i].g_fuse;
     DFL_CUDA(launch_fuse(dt, a->new_states, a->n_ctx_new, c->n_target_layers, H, D, w->w_fuse,
-                         gf, fused, c->rms_eps, st),
+                         gf, fused, c->rms_eps, status, st),
              "fusion kernel");
   }
   DFL_CUDA(launch_embed(dt, w->embed, H, a->n_blocks, c->block, a->block_tokens, a->known_len,
@@ -544,19 +546,23 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
     const dflash_layer_weights& l = w->layers[i];
     // context K/V of the new rows through W^t, into the caches
     if (a->n_ctx_new > 0) {
-      s = run_job(job_kv(c, fused + static_cast<size_t>(i) * a->n_ctx_new * H * e, a->n_ctx_new,
-                         new_pos, new_dst, l.w_kt, l.w_vt, a->k_cache[i], a->v_cache[i]),
-                  partial, counters, status, st, "context K/V GEMM");
+      GemmJob jc = job_kv(c, fused + static_cast<size_t>(i) * a->n_ctx_new * H * e,
+                          a->n_ctx_new, new_pos, new_dst, l.w_kt, l.w_vt, a->k_cache[i],
+                          a->v_cache[i]);
+      jc.rope_tab = rope_tab;
+      jc.rope_len = L.rope_len;
+      s = run_job(jc, partial, counters, status, st, "context K/V GEMM");
       if (s != DFLASH_OK) return s;
     }
     // block: RMSNorm -> Q (RoPE), K^d (RoPE), V^d
     DFL_CUDA(launch_rmsnorm(dt, h, M, H, l.g_attn, c->rms_eps, x, st), "attention rmsnorm");
-    if ((s = run_job(job_qkv(c, l, x, M, blk_pos, q, kb, vb), partial, counters, status, st,
-                     "QKV GEMM")) != DFLASH_OK)
-      return s;
+    GemmJob jq = job_qkv(c, l, x, M, blk_pos, q, kb, vb);
+    jq.rope_tab = rope_tab;
+    jq.rope_len = L.rope_len;
+    if ((s = run_job(jq, partial, counters, status, st, "QKV GEMM")) != DFLASH_OK) return s;
     DFL_CUDA(launch_attn(dt, ap, a->n_blocks, c->block, c->n_q_heads, c->n_kv_heads,
                          c->head_dim, q, kb, vb, a->k_cache[i], a->v_cache[i], a->ctx_off,
-                         a->block_req, attn, at<float>(ws, L.attn_ws), counters, status, st),
+                         a->block_req, attn, at<float>(ws, L.attn_ws), status, st),
              "attention");
     if ((s = run_job(job_resid(c, l.w_o, attn, M, qd, h), partial, counters, status, st,
                      "O GEMM")) != DFLASH_OK)

@@ -28,60 +28,7 @@ struct AttnParams {
   float scale;
   float* part_o;   // [nb*B*Hq][splits][d]
   float* part_ml;  // [nb*B*Hq][splits][2]
-  uint32_t* counters;  // [nb*Hkv*row_chunks], zero on entry, left zero
-  void* out;       // [nb*B][Hq][d]
 };
-
-// Called by every CTA after writing its split's partials: the last CTA of
-// a (block, kv head, row chunk) group merges the splits in fixed order,
-//   out = sum_s o_s e^{m_s - M} / sum_s l_s e^{m_s - M},  M = max_s m_s,
-// and re-arms the group's counter.
-template <typename T, int D>
-__device__ void attn_merge_splits(const AttnParams& p, int b, int g, int row0, int nrows) {
-  __shared__ float wts[64][65];
-  __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  const int grp = (b * p.Hkv + g) * gridDim.z + blockIdx.z;
-  if (threadIdx.x == 0) {
-    const uint32_t prev = atomicAdd(p.counters + grp, 1u);
-    s_last = prev == static_cast<uint32_t>(p.splits - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  auto prow = [&](int r) {
-    const int rr = row0 + r;
-    const int s = rr / p.G, j = rr % p.G;
-    return (static_cast<size_t>(b) * p.B + s) * p.Hq + g * p.G + j;
-  };
-  for (int r = threadIdx.x; r < nrows; r += blockDim.x) {
-    const float* ml = p.part_ml + prow(r) * p.splits * 2;
-    float M = -INFINITY;
-    for (int s = 0; s < p.splits; ++s)
-      if (__ldcg(ml + 2 * s + 1) > 0.f) M = fmaxf(M, __ldcg(ml + 2 * s));
-    float den = 0.f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float ls = __ldcg(ml + 2 * s + 1);
-      const float w = ls > 0.f ? expf(__ldcg(ml + 2 * s) - M) : 0.f;
-      wts[r][s] = w;
-      den = fmaf(ls, w, den);
-    }
-    const float inv = 1.f / den;
-    for (int s = 0; s < p.splits; ++s) wts[r][s] *= inv;
-  }
-  __syncthreads();
-  T* out = static_cast<T*>(p.out);
-  for (int e = threadIdx.x; e < nrows * D; e += blockDim.x) {
-    const int r = e / D, dd = e % D;
-    const size_t pr = prow(r);
-    const float* po = p.part_o + pr * p.splits * D + dd;
-    float acc = 0.f;
-    for (int s = 0; s < p.splits; ++s) acc = fmaf(__ldcg(po + s * D), wts[r][s], acc);
-    out[pr * D + dd] = from_f<T>(acc);
-  }
-  if (threadIdx.x == 0) p.counters[grp] = 0u;
-}
 
 constexpr int kAttnWarps = 4;
 constexpr int kAttnRowsPerWarp = 8;
@@ -189,7 +136,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_simt_kernel(const AttnPa
       p.part_ml[(pr * p.splits + split) * 2 + 1] = l[i];
     }
   }
-  attn_merge_splits<T, D>(p, b, g, row0, nrows);
 }
 
 // ---------------------------------------------------------------------------
@@ -430,8 +376,35 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnParams p) {
       p.part_ml[(pr * p.splits + split) * 2 + 1] = h ? l1 : l0;
     }
   }
-  attn_merge_splits<__nv_bfloat16, D>(p, b, g, blockIdx.z * kMmaRows,
-                                      min(kMmaRows, nrows_all - blockIdx.z * kMmaRows));
+}
+
+// out[pr][dd] = sum_s o_s e^{m_s - M} / sum_s l_s e^{m_s - M}, splits in a
+// fixed order; one thread per output element.
+template <typename T>
+__global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_o,
+                                                           const float* __restrict__ part_ml,
+                                                           int64_t n_rows, int splits, int D,
+                                                           T* __restrict__ out) {
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
+  const int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (idx >= n_rows * D) return;
+  const int64_t pr = idx / D;
+  const int dd = static_cast<int>(idx - pr * D);
+  const float* ml = part_ml + pr * splits * 2;
+  const float* po = part_o + pr * splits * D + dd;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s)
+    if (ml[2 * s + 1] > 0.f) M = fmaxf(M, ml[2 * s]);
+  float num = 0.f, den = 0.f;
+#pragma unroll 8
+  for (int s = 0; s < splits; ++s) {
+    const float ls = ml[2 * s + 1];
+    const float w = ls > 0.f ? __expf(ml[2 * s] - M) : 0.f;
+    den = fmaf(ls, w, den);
+    num = fmaf(po[s * D], w, num);
+  }
+  out[idx] = from_f<T>(num / den);
 }
 
 // Opt every attention kernel into large dynamic shared memory once (on the
@@ -465,7 +438,9 @@ AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d, int64_t max
     p.chunk = 64;
     return p;
   }
-  const int64_t max_splits = std::min<int64_t>(64, (max_ctx_len + 63) / 64);
+  // at least 256 context keys per split: the fp32 partials of a split then
+  // stay well below the K/V bytes it streams
+  const int64_t max_splits = std::min<int64_t>(64, (max_ctx_len + 255) / 256);
   int64_t want = (2 * kNumSMs + base - 1) / base;
   int64_t splits = std::max<int64_t>(1, std::min(want, max_splits));
   int64_t chunk = (max_ctx_len + splits - 1) / splits;
@@ -480,15 +455,10 @@ size_t attn_ws_bytes(const AttnPlan& p, int nb, int B, int Hq, int d) {
   return rows * p.splits * (d + 2) * sizeof(float);
 }
 
-size_t attn_counters(const AttnPlan& p, int nb, int Hkv) {
-  return static_cast<size_t>(nb) * Hkv * p.row_chunks;
-}
-
 cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq, int Hkv, int d,
                         const void* q, const void* kb, const void* vb, const void* kc,
                         const void* vc, const int64_t* ctx_off, const int32_t* block_req,
-                        void* out, float* ws, uint32_t* counters, uint32_t* status,
-                        cudaStream_t st) {
+                        void* out, float* ws, uint32_t* status, cudaStream_t st) {
   (void)status;
   if (nb <= 0) return cudaSuccess;
   AttnParams p{};
@@ -503,20 +473,28 @@ cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq, 
   const int64_t n_rows = static_cast<int64_t>(nb) * B * Hq;
   p.part_o = ws;
   p.part_ml = ws + static_cast<size_t>(n_rows) * plan.splits * d;
-  p.counters = counters;
-  p.out = out;
   dim3 grid(nb * Hkv, plan.splits, plan.row_chunks);
   cudaError_t e = allow_smem();
   if (e != cudaSuccess) return e;
   if (dtype == DFLASH_BF16) {
     const size_t smem = 2 * 2 * static_cast<size_t>(kMmaKeys) * d * sizeof(__nv_bfloat16);
-    if (d == 64) return launch_k(attn_mma_kernel<64>, grid, dim3(128), smem, st, p);
-    return launch_k(attn_mma_kernel<128>, grid, dim3(128), smem, st, p);
+    e = d == 64 ? launch_k(attn_mma_kernel<64>, grid, dim3(128), smem, st, p)
+                : launch_k(attn_mma_kernel<128>, grid, dim3(128), smem, st, p);
+  } else {
+    const size_t smem = (static_cast<size_t>(plan.rows_per_cta) * d +
+                         kAttnKeyTile * (d + 1) + kAttnKeyTile * d) * sizeof(float);
+    e = d == 64 ? launch_k(attn_simt_kernel<float, 64>, grid, dim3(kAttnWarps * 32), smem, st, p)
+                : launch_k(attn_simt_kernel<float, 128>, grid, dim3(kAttnWarps * 32), smem, st,
+                           p);
   }
-  const size_t smem = (static_cast<size_t>(plan.rows_per_cta) * d +
-                       kAttnKeyTile * (d + 1) + kAttnKeyTile * d) * sizeof(float);
-  if (d == 64) return launch_k(attn_simt_kernel<float, 64>, grid, dim3(kAttnWarps * 32), smem, st, p);
-  return launch_k(attn_simt_kernel<float, 128>, grid, dim3(kAttnWarps * 32), smem, st, p);
+  if (e != cudaSuccess) return e;
+  const int64_t total = n_rows * d;
+  const dim3 cgrid(static_cast<unsigned>((total + 255) / 256));
+  if (dtype == DFLASH_BF16)
+    return launch_k(attn_combine_kernel<__nv_bfloat16>, cgrid, dim3(256), 0, st, p.part_o,
+                    p.part_ml, n_rows, plan.splits, d, static_cast<__nv_bfloat16*>(out));
+  return launch_k(attn_combine_kernel<float>, cgrid, dim3(256), 0, st, p.part_o, p.part_ml,
+                  n_rows, plan.splits, d, static_cast<float*>(out));
 }
 
 }  // namespace dfl

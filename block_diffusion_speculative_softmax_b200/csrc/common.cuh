@@ -184,6 +184,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map,
         "r"(c0), "r"(c1)
       : "memory");
 }
+// Contiguous global -> shared bulk copy (size and both addresses multiples
+// of 16 bytes), completing on an mbarrier transaction count.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

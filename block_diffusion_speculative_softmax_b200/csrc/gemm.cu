@@ -84,10 +84,24 @@ struct Params {
   const int32_t* pos;
   const int64_t* dst;
   int head_dim;
+  const float2* rope_tab;           // (cos, sin) [rope_len][head_dim / 2] or null
+  int rope_len;
   double inv_freq[64];
   unsigned long long* keys;         // argmax mode: [M]
   uint32_t* status;
 };
+
+// cos / sin of pos * inv_freq[fi]: from the step's table when the position
+// is inside it, else computed (angle reduced mod 2 pi in double first).
+__device__ __forceinline__ float2 rope_cs(const Params& p, int pos, int fi) {
+  if (p.rope_tab != nullptr && pos < p.rope_len)
+    return __ldg(p.rope_tab + static_cast<size_t>(pos) * (p.head_dim >> 1) + fi);
+  double ang = static_cast<double>(pos) * p.inv_freq[fi];
+  ang -= 6.283185307179586 * rint(ang * 0.15915494309189535);
+  float sn, cs;
+  sincosf(static_cast<float>(ang), &sn, &cs);
+  return make_float2(cs, sn);
+}
 
 template <int BN, int STAGES, bool ARGMAX>
 __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Params p) {
@@ -283,57 +297,90 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
       do_op = s_last != 0;
       if (do_op) {
         __threadfence();
-        const float* base = p.partial + static_cast<size_t>(tile_lin) * p.splits * BN * BM;
+        // fixed split order; 16 independent loads in flight per thread
+        const float* base = p.partial + static_cast<size_t>(tile_lin) * p.splits * BN * BM + tid;
+        constexpr int JC = BN < 16 ? BN : 16;
 #pragma unroll 1
-        for (int j = 0; j < BN; ++j) {
-          float acc = 0.f;
-          for (int s = 0; s < p.splits; ++s) acc += __ldcg(base + (s * BN + j) * BM + tid);
-          st[j * SROW + tid] = acc;
+        for (int j0 = 0; j0 < BN; j0 += JC) {
+          float acc[JC];
+#pragma unroll
+          for (int q = 0; q < JC; ++q) acc[q] = 0.f;
+#pragma unroll 1
+          for (int s = 0; s < p.splits; ++s) {
+            float v[JC];
+#pragma unroll
+            for (int q = 0; q < JC; ++q) v[q] = __ldcg(base + (s * BN + j0 + q) * BM);
+#pragma unroll
+            for (int q = 0; q < JC; ++q) acc[q] += v[q];
+          }
+#pragma unroll
+          for (int q = 0; q < JC; ++q) st[(j0 + q) * SROW + tid] = acc[q];
         }
         if (tid == 0) p.counters[tile_lin] = 0u;
       }
     }
     __syncthreads();
     if (do_op) {
+      constexpr int JU = BN < 8 ? BN : 8;   // tokens per unrolled group
       if (S.op == EPI_SWIGLU) {
         const int r = tid & 63;
         const int f = row0 + r;
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out);
+#pragma unroll 4
         for (int j = tid >> 6; j < BN; j += 2) {
           const int t = tok0 + j;
           if (f < S.rows && t < p.M) {
             const float g = st[j * SROW + r], u = st[j * SROW + r + 64];
-            const float a = g / (1.f + __expf(-g)) * u;
-            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out);
-            o[static_cast<int64_t>(t) * S.out_stride + f] = __float2bfloat16_rn(a);
+            o[static_cast<int64_t>(t) * S.out_stride + f] =
+                __float2bfloat16_rn(g / (1.f + __expf(-g)) * u);
+          }
+        }
+      } else if (S.op == EPI_RESID) {
+        const int f = row0 + tid;
+        float* h = static_cast<float*>(S.out) + f;
+#pragma unroll 1
+        for (int j0 = 0; j0 < BN; j0 += JU) {
+          float hv[JU];
+#pragma unroll
+          for (int q = 0; q < JU; ++q) {
+            const int t = tok0 + j0 + q;
+            hv[q] = (f < S.rows && t < p.M) ? h[static_cast<int64_t>(t) * S.out_stride] : 0.f;
+          }
+#pragma unroll
+          for (int q = 0; q < JU; ++q) {
+            const int t = tok0 + j0 + q;
+            if (f < S.rows && t < p.M)
+              h[static_cast<int64_t>(t) * S.out_stride] = hv[q] + st[(j0 + q) * SROW + tid];
           }
         }
       } else {
         const int f = row0 + tid;
-        const int d = p.head_dim, half = d >> 1;
-        const int i = tid % d;
+        const int half = p.head_dim >> 1;
+        const int i = tid % p.head_dim;
         const int prt = i < half ? tid + half : tid - half;
         const int fi = i < half ? i : i - half;
-        const double invf = S.rope ? p.inv_freq[fi] : 0.0;
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out);
 #pragma unroll 1
-        for (int j = 0; j < BN; ++j) {
-          const int t = tok0 + j;
-          if (f >= S.rows || t >= p.M) continue;
-          float v = st[j * SROW + tid];
-          if (S.op == EPI_RESID) {
-            float* h = static_cast<float*>(S.out) + static_cast<int64_t>(t) * S.out_stride + f;
-            *h += v;
-            continue;
+        for (int j0 = 0; j0 < BN; j0 += JU) {
+          float2 cs[JU];
+          int64_t orow[JU];
+#pragma unroll
+          for (int q = 0; q < JU; ++q) {
+            const int t = min(tok0 + j0 + q, p.M - 1);
+            cs[q] = S.rope ? rope_cs(p, p.pos[t], fi) : make_float2(1.f, 0.f);
+            orow[q] = S.use_dst ? p.dst[t] : t;
           }
-          if (S.rope) {
-            const float pv = st[j * SROW + prt];
-            double ang = static_cast<double>(p.pos[t]) * invf;
-            ang -= 6.283185307179586 * rint(ang * 0.15915494309189535);
-            float sn, cs;
-            sincosf(static_cast<float>(ang), &sn, &cs);
-            v = i < half ? v * cs - pv * sn : v * cs + pv * sn;
+#pragma unroll
+          for (int q = 0; q < JU; ++q) {
+            const int t = tok0 + j0 + q;
+            if (f >= S.rows || t >= p.M) continue;
+            float v = st[(j0 + q) * SROW + tid];
+            if (S.rope) {
+              const float pv = st[(j0 + q) * SROW + prt];
+              v = i < half ? v * cs[q].x - pv * cs[q].y : v * cs[q].x + pv * cs[q].y;
+            }
+            o[orow[q] * S.out_stride + f] = __float2bfloat16_rn(v);
           }
-          const int64_t orow = S.use_dst ? p.dst[t] : t;
-          static_cast<__nv_bfloat16*>(S.out)[orow * S.out_stride + f] = __float2bfloat16_rn(v);
         }
       }
     }
@@ -736,6 +783,8 @@ cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& pl, float* partial,
   p.pos = job.pos;
   p.dst = job.dst;
   p.head_dim = job.head_dim > 0 ? job.head_dim : 128;
+  p.rope_tab = job.rope_tab;
+  p.rope_len = job.rope_len;
   fill_inv_freq(job.theta, p.head_dim, p.inv_freq);
   p.status = status;
   dim3 grid(tiles, pl.tok_tiles, pl.splits);

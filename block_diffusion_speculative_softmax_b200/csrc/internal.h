@@ -52,6 +52,8 @@ struct GemmJob {
   const int64_t* dst = nullptr;   // [M]
   int head_dim = 0;
   double theta = 1e6;
+  const float2* rope_tab = nullptr;   // (cos, sin) [rope_len][head_dim / 2]
+  int rope_len = 0;
 };
 
 struct GemmPlan {
@@ -81,7 +83,7 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V,
 // ---------------------------------------------------------------- others
 cudaError_t launch_fuse(int dtype, const void* states, int64_t N, int T, int H,
                         int D, const float* w_fuse, const float* const* g_fuse,
-                        void* fused, float eps, cudaStream_t st);
+                        void* fused, float eps, uint32_t* status, cudaStream_t st);
 // Largest hidden size the fusion kernel covers for T target layers.
 int fuse_hidden_limit(int dtype, int nT);
 cudaError_t launch_embed(int dtype, const void* embed, int H, int nb, int B,
@@ -101,6 +103,9 @@ cudaError_t launch_argmax_finish(unsigned long long* keys, int64_t M,
                                  const int32_t* known_len, int32_t* tok,
                                  float* max_logit, cudaStream_t st);
 cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t st);
+// RoPE table: tab[p][i] = (cos, sin)(p * theta^(-2i/d)), p < len, i < d/2.
+cudaError_t launch_rope_table(float2* tab, int len, int head_dim, double theta,
+                              cudaStream_t st);
 
 // Kernel launch with programmatic dependent launch enabled: the kernel may
 // start while the previous kernel on the stream finishes; every kernel of
@@ -132,14 +137,11 @@ struct AttnPlan {
 AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d,
                    int64_t max_ctx_len);
 size_t attn_ws_bytes(const AttnPlan& p, int nb, int B, int Hq, int d);
-size_t attn_counters(const AttnPlan& p, int nb, int Hkv);
-// counters: attn_counters() words, zero on entry (left zero).
 cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq,
                         int Hkv, int d, const void* q, const void* kb,
                         const void* vb, const void* kc, const void* vc,
                         const int64_t* ctx_off, const int32_t* block_req,
-                        void* out, float* ws, uint32_t* counters, uint32_t* status,
-                        cudaStream_t st);
+                        void* out, float* ws, uint32_t* status, cudaStream_t st);
 
 cudaError_t launch_accept(int R, int K, int B, const int32_t* draft,
                           const int32_t* target, int32_t* n_acc,

@@ -1,5 +1,7 @@
 // Bandwidth- and latency-bound kernels of the draft step.
 #include <algorithm>
+#include <cmath>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -9,168 +11,204 @@ namespace dfl {
 // ===========================================================================
 // Adaptive layer fusion + RMSNorm (DFLARE summary, section 2.1)
 //
-// One CTA per context row.  Thread t owns one 16-byte vector of columns and
-// keeps that vector of all T target layers in registers, so the T states
-// are read from HBM exactly once; all D draft layers' fused rows are
-// produced from them:  u_i = sum_j alpha_ij h_j,  f_i = u_i * rsqrt(mean
-// (u_i^2) + eps) * g_i  with alpha_i = softmax(W_fuse[i]).
+// Persistent CTAs walk the context rows.  A row's T target states are
+// contiguous ([T][H]), so thread 0 streams whole rows into a shared-memory
+// ring with cp.async.bulk (one copy per row, completion on an mbarrier).
+// Thread t owns one 16-byte vector of columns: it reads that vector of the
+// T states once and accumulates, in registers, the fused vectors of all D
+// draft layers  u_i = sum_j alpha_ij h_j  (alpha_i = softmax(W_fuse[i])) and
+// their sums of squares; one block barrier per row combines the sums, and
+// f_i = u_i * rsqrt(mean(u_i^2) + eps) * g_i is stored straight from the
+// registers.  The states are read from HBM exactly once.
 // ===========================================================================
 struct FuseGains {
   const float* g[kMaxLayers];
 };
 
-// VW = 16: one 128-bit load per target layer; VW = 8 halves the registers
-// for large T.
-template <typename T, int VW> struct VecN;
-template <typename T> struct VecN<T, 16> : Vec16<T> {};
-template <> struct VecN<__nv_bfloat16, 8> {
-  static constexpr int N = 4;
-  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* out) {
-    uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-    float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-    out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
-  }
-  __device__ __forceinline__ static void store(__nv_bfloat16* p, const float* in) {
-    uint2 u;
-    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
-    h[0] = __floats2bfloat162_rn(in[0], in[1]);
-    h[1] = __floats2bfloat162_rn(in[2], in[3]);
-    *reinterpret_cast<uint2*>(p) = u;
-  }
-};
-template <> struct VecN<float, 8> {
-  static constexpr int N = 2;
-  __device__ __forceinline__ static void load(const float* p, float* out) {
-    float2 u = __ldg(reinterpret_cast<const float2*>(p));
-    out[0] = u.x; out[1] = u.y;
-  }
-  __device__ __forceinline__ static void store(float* p, const float* in) {
-    *reinterpret_cast<float2*>(p) = make_float2(in[0], in[1]);
-  }
-};
-
 constexpr int kFuseThreads = 512;
+constexpr int kFuseSmemBudget = 200 * 1024;
 
-template <typename T, int MAXT, int VW>
-__global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(const T* __restrict__ states,
-                                                                 int64_t N, int nT, int H, int D,
-                                                                 const float* __restrict__ w_fuse,
-                                                                 const FuseGains gains,
-                                                                 T* __restrict__ fused, float eps) {
-  using V = VecN<T, VW>;
+template <typename T, int MAXD>
+__global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
+    const T* __restrict__ states, int64_t N, int nT, int H, int D,
+    const float* __restrict__ w_fuse, const FuseGains gains, T* __restrict__ fused, float eps,
+    int slots, uint32_t* status) {
+  using V = Vec16<T>;
   constexpr int VE = V::N;
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ __align__(8) uint64_t full[8];
   __shared__ float alpha[kMaxLayers][kMaxTargetLayers];
-  __shared__ float red[32][kMaxLayers];
-  __shared__ float scale[kMaxLayers];
-  const int tid = threadIdx.x;
+  __shared__ float red[2][32][MAXD];
+  __shared__ volatile int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nwarps = (blockDim.x + 31) >> 5;
+  const uint32_t row_bytes = static_cast<uint32_t>(nT) * H * sizeof(T);
   pdl_wait();
   if (tid == 0) pdl_launch();
+  if (tid == 0) {
+    for (int s = 0; s < slots; ++s) mbar_init(&full[s], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
   if (tid < D) {
     float mx = -INFINITY;
     for (int j = 0; j < nT; ++j) mx = fmaxf(mx, w_fuse[tid * nT + j]);
-    float s = 0.f;
+    float sum = 0.f;
     for (int j = 0; j < nT; ++j) {
       const float e = expf(w_fuse[tid * nT + j] - mx);
       alpha[tid][j] = e;
-      s += e;
+      sum += e;
     }
-    for (int j = 0; j < nT; ++j) alpha[tid][j] /= s;
+    for (int j = 0; j < nT; ++j) alpha[tid][j] /= sum;
   }
   __syncthreads();
+  // rows of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int64_t my_rows = N > blockIdx.x ? (N - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (tid == 0) {
+    for (int k = 0; k < slots && k < my_rows; ++k) {
+      const int64_t n = blockIdx.x + k * static_cast<int64_t>(gridDim.x);
+      mbar_arrive_expect_tx(&full[k], row_bytes);
+      bulk_load(ring + static_cast<size_t>(k) * row_bytes, states + n * nT * H, row_bytes,
+                &full[k]);
+    }
+  }
   const int nvec = H / VE;
   const bool active = tid < nvec;
   const int col = tid * VE;
-  for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
-    float h[MAXT][VE];
-    if (active) {
-      const T* src = states + (static_cast<size_t>(n) * nT) * H + col;
-#pragma unroll
-      for (int j = 0; j < MAXT; ++j)
-        if (j < nT) V::load(src + static_cast<size_t>(j) * H, h[j]);
+  int64_t k = 0;
+  for (; k < my_rows; ++k) {
+    const int slot = static_cast<int>(k % slots);
+    const int64_t n = blockIdx.x + k * static_cast<int64_t>(gridDim.x);
+    if (!mbar_wait(&full[slot], static_cast<uint32_t>((k / slots) & 1), status, 21)) {
+      abort_flag = 1;
     }
-    float ss[kMaxLayers];
+    float u[MAXD][VE];
+    float ss[MAXD];
 #pragma unroll
-    for (int i = 0; i < kMaxLayers; ++i) ss[i] = 0.f;
-    if (active) {
+    for (int i = 0; i < MAXD; ++i) {
+      ss[i] = 0.f;
 #pragma unroll
-      for (int i = 0; i < kMaxLayers; ++i) {
-        if (i >= D) break;
-        float acc = 0.f;
+      for (int e = 0; e < VE; ++e) u[i][e] = 0.f;
+    }
+    if (active && !abort_flag) {
+      const T* row = reinterpret_cast<const T*>(ring + static_cast<size_t>(slot) * row_bytes);
+      for (int j = 0; j < nT; ++j) {
+        float h[VE];
+        const uint4 raw = *reinterpret_cast<const uint4*>(row + static_cast<size_t>(j) * H + col);
+        if constexpr (VE == 8) {
+          const __nv_bfloat162* hp = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-        for (int e = 0; e < VE; ++e) {
-          float u = 0.f;
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(hp[q]);
+            h[2 * q] = f.x;
+            h[2 * q + 1] = f.y;
+          }
+        } else {
+          const float* fp = reinterpret_cast<const float*>(&raw);
 #pragma unroll
-          for (int j = 0; j < MAXT; ++j)
-            if (j < nT) u = fmaf(alpha[i][j], h[j][e], u);
-          acc = fmaf(u, u, acc);
+          for (int q = 0; q < VE; ++q) h[q] = fp[q];
         }
-        ss[i] = acc;
+#pragma unroll
+        for (int i = 0; i < MAXD; ++i) {
+          if (i < D) {
+            const float a = alpha[i][j];
+#pragma unroll
+            for (int e = 0; e < VE; ++e) u[i][e] = fmaf(a, h[e], u[i][e]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < MAXD; ++i)
+#pragma unroll
+        for (int e = 0; e < VE; ++e) ss[i] = fmaf(u[i][e], u[i][e], ss[i]);
+    }
+    const int par = static_cast<int>(k & 1);
+#pragma unroll
+    for (int i = 0; i < MAXD; ++i) {
+      if (i < D) {
+        const float v = warp_sum(ss[i]);
+        if (lane == 0) red[par][warp][i] = v;
       }
     }
-    // block reduction of the D sums of squares
-    const int warp = tid >> 5, lane = tid & 31, nwarps = (blockDim.x + 31) >> 5;
-#pragma unroll
-    for (int i = 0; i < kMaxLayers; ++i) {
-      if (i >= D) break;
-      const float v = warp_sum(ss[i]);
-      if (lane == 0) red[warp][i] = v;
+    __syncthreads();   // the slot is consumed and the per-warp sums are visible
+    if (tid == 0 && !abort_flag && k + slots < my_rows) {
+      const int64_t n2 = blockIdx.x + (k + slots) * static_cast<int64_t>(gridDim.x);
+      mbar_arrive_expect_tx(&full[slot], row_bytes);
+      bulk_load(ring + static_cast<size_t>(slot) * row_bytes, states + n2 * nT * H, row_bytes,
+                &full[slot]);
     }
-    __syncthreads();
-    if (tid < D) {
-      float s = 0.f;
-      for (int w = 0; w < nwarps; ++w) s += red[w][tid];
-      scale[tid] = rsqrtf(s / static_cast<float>(H) + eps);
-    }
-    __syncthreads();
+    if (abort_flag) break;
     if (active) {
-      for (int i = 0; i < D; ++i) {
-        const float sc = scale[i];
-        const float* g = gains.g[i] + col;
-        float o[VE];
 #pragma unroll
-        for (int e = 0; e < VE; ++e) {
-          float u = 0.f;
+      for (int i = 0; i < MAXD; ++i) {
+        if (i < D) {
+          float tot = 0.f;
+          for (int w = 0; w < nwarps; ++w) tot += red[par][w][i];
+          const float sc = rsqrtf(tot / static_cast<float>(H) + eps);
+          const float* g = gains.g[i] + col;
+          float o[VE];
 #pragma unroll
-          for (int j = 0; j < MAXT; ++j)
-            if (j < nT) u = fmaf(alpha[i][j], h[j][e], u);
-          o[e] = u * sc * __ldg(g + e);
+          for (int e = 0; e < VE; ++e) o[e] = u[i][e] * sc * __ldg(g + e);
+          V::store(fused + (static_cast<size_t>(i) * N + n) * H + col, o);
         }
-        V::store(fused + (static_cast<size_t>(i) * N + n) * H + col, o);
       }
     }
-    __syncthreads();
+  }
+  if (abort_flag && tid == 0) {
+    // let copies still in flight land before the CTA's shared memory goes away
+    for (int64_t q = k; q < my_rows && q < k + slots; ++q)
+      mbar_wait(&full[q % slots], static_cast<uint32_t>((q / slots) & 1), status, 22);
   }
 }
 
-template <typename T, int MAXT, int VW>
-static cudaError_t fuse_go(const void* states, int64_t N, int nT, int H, int D, const float* w_fuse,
-                    const FuseGains& g, void* fused, float eps, cudaStream_t st) {
-  const int nvec = H / VecN<T, VW>::N;
-  const int threads = ((nvec + 31) / 32) * 32;
-  const int grid = static_cast<int>(std::min<int64_t>(N, 1 << 20));
-  return launch_k(fuse_rows_kernel<T, MAXT, VW>, dim3(grid), dim3(threads), 0, st,
-                  static_cast<const T*>(states), N, nT, H, D, w_fuse, g,
-                  static_cast<T*>(fused), eps);
+// Ring depth: rows of up to ~96 KB in flight per CTA (two CTAs per SM fit
+// when the ring is small), never fewer than two rows.
+template <typename T>
+static int fuse_slots(int nT, int H) {
+  const int rb = nT * H * static_cast<int>(sizeof(T));
+  return std::max(2, std::min(8, (96 * 1024) / rb));
 }
 
-// Largest hidden size each variant covers with kFuseThreads threads.
+template <typename T, int MAXD>
+static cudaError_t fuse_go(const void* states, int64_t N, int nT, int H, int D,
+                           const float* w_fuse, const FuseGains& g, void* fused, float eps,
+                           uint32_t* status, cudaStream_t st) {
+  const int nvec = H / Vec16<T>::N;
+  const int threads = ((nvec + 31) / 32) * 32;
+  const int slots = fuse_slots<T>(nT, H);
+  const size_t smem = static_cast<size_t>(slots) * nT * H * sizeof(T);
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(fuse_rows_kernel<T, MAXD>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kFuseSmemBudget);
+  });
+  if (attr != cudaSuccess) return attr;
+  // two CTAs per SM when the ring is small enough
+  const int per_sm = smem <= 100 * 1024 && threads <= 512 ? 2 : 1;
+  const int grid = static_cast<int>(std::min<int64_t>(N, kNumSMs * per_sm));
+  return launch_k(fuse_rows_kernel<T, MAXD>, dim3(grid), dim3(threads), smem, st,
+                  static_cast<const T*>(states), N, nT, H, D, w_fuse, g,
+                  static_cast<T*>(fused), eps, slots, status);
+}
+
+// Largest hidden size the fusion kernel covers (one 16-byte vector per
+// thread, at most kFuseThreads threads, at least one row in the ring).
 template <typename T>
 static int fuse_max_hidden(int nT) {
-  const int ve16 = 16 / static_cast<int>(sizeof(T));
-  return kFuseThreads * (nT <= 9 ? ve16 : ve16 / 2);
+  const int by_threads = kFuseThreads * (16 / static_cast<int>(sizeof(T)));
+  const int by_smem = kFuseSmemBudget / 2 / (nT * static_cast<int>(sizeof(T)));
+  return std::min(by_threads, by_smem / 16 * 16);
 }
 
 template <typename T>
 static cudaError_t launch_fuse_t(const void* states, int64_t N, int nT, int H, int D,
                                  const float* w_fuse, const FuseGains& g, void* fused, float eps,
-                                 cudaStream_t st) {
+                                 uint32_t* status, cudaStream_t st) {
   if (H > fuse_max_hidden<T>(nT)) return cudaErrorInvalidValue;
-  if (nT <= 4) return fuse_go<T, 4, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
-  if (nT <= 5) return fuse_go<T, 5, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
-  if (nT <= 8) return fuse_go<T, 8, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
-  if (nT <= 9) return fuse_go<T, 9, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
-  return fuse_go<T, 16, 8>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+  if (D <= 4) return fuse_go<T, 4>(states, N, nT, H, D, w_fuse, g, fused, eps, status, st);
+  if (D <= 8) return fuse_go<T, 8>(states, N, nT, H, D, w_fuse, g, fused, eps, status, st);
+  return fuse_go<T, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, status, st);
 }
 
 int fuse_hidden_limit(int dtype, int nT) {
@@ -179,13 +217,13 @@ int fuse_hidden_limit(int dtype, int nT) {
 
 cudaError_t launch_fuse(int dtype, const void* states, int64_t N, int nT, int H, int D,
                         const float* w_fuse, const float* const* g_fuse, void* fused, float eps,
-                        cudaStream_t st) {
+                        uint32_t* status, cudaStream_t st) {
   if (N <= 0) return cudaSuccess;
   FuseGains g{};
   for (int i = 0; i < D; ++i) g.g[i] = g_fuse[i];
   if (dtype == DFLASH_BF16)
-    return launch_fuse_t<__nv_bfloat16>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
-  return launch_fuse_t<float>(states, N, nT, H, D, w_fuse, g, fused, eps, st);
+    return launch_fuse_t<__nv_bfloat16>(states, N, nT, H, D, w_fuse, g, fused, eps, status, st);
+  return launch_fuse_t<float>(states, N, nT, H, D, w_fuse, g, fused, eps, status, st);
 }
 
 // ===========================================================================
@@ -300,6 +338,36 @@ cudaError_t launch_prep_rows(int R, int nb, int B, const int32_t* block_req,
   const int grid = static_cast<int>(std::min<int64_t>((work + 255) / 256, kNumSMs * 8));
   return launch_k(prep_rows_kernel, dim3(grid), dim3(256), 0, st, R, nb, B, block_req, ctx_off,
                   new_off, ctx_cached, n_new, blk_pos, new_pos, new_dst, zero, n_zero);
+}
+
+struct InvFreq {
+  double v[64];
+};
+
+__global__ void rope_table_kernel(float2* __restrict__ tab, int len, int half, const InvFreq f) {
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
+  const int64_t n = static_cast<int64_t>(len) * half;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int pos = static_cast<int>(e / half), i = static_cast<int>(e % half);
+    double ang = static_cast<double>(pos) * f.v[i];
+    ang -= 6.283185307179586 * rint(ang * 0.15915494309189535);
+    float sn, cs;
+    sincosf(static_cast<float>(ang), &sn, &cs);
+    tab[e] = make_float2(cs, sn);
+  }
+}
+
+cudaError_t launch_rope_table(float2* tab, int len, int head_dim, double theta,
+                              cudaStream_t st) {
+  const int half = head_dim / 2;
+  const int64_t n = static_cast<int64_t>(len) * half;
+  if (n <= 0) return cudaSuccess;
+  InvFreq f{};
+  for (int i = 0; i < half && i < 64; ++i) f.v[i] = std::pow(theta, -2.0 * i / head_dim);
+  const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, kNumSMs * 8));
+  return launch_k(rope_table_kernel, dim3(grid), dim3(256), 0, st, tab, len, half, f);
 }
 
 __global__ void zero_kernel(uint32_t* __restrict__ p, int64_t n) {
