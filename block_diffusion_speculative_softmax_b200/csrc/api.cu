@@ -1,6 +1,7 @@
 // C ABI of libdflash.so: argument validation, workspace layout and the
 // kernel sequence of one draft step.  No entry point allocates memory.
 #include <atomic>
+#include <mutex>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -590,3 +591,71 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// LM-head argmax for callers that cannot allocate device memory
+// ===========================================================================
+// Some callers cannot call cudaMalloc or hand us a workspace: a plugin loaded
+// into a serving process whose device memory is owned by that process's
+// caching allocator, or a latency-critical loop that is not allowed to
+// allocate after start-up.  This variant keeps its only scratch -- one
+// 64-bit argmax key per token -- in a fixed array that lives in the module's
+// global memory for as long as the library is loaded, on every GPU that
+// loads it.
+namespace dfl {
+namespace {
+
+constexpr int64_t kNoAllocMaxTokens = 4096;       // 32 KiB of keys per device
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned long long g_noalloc_keys[kNoAllocMaxTokens];
+
+std::mutex g_noalloc_mu;
+unsigned long long* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_keys on the current device.  In host code the
+// array's name is only a stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+dflash_status noalloc_scratch(unsigned long long** out) {
+  int dev = 0;
+  DFL_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  DFL_CHECK(dev >= 0 && dev < kNoAllocMaxDevices, DFLASH_EUNSUPPORTED,
+            "device ordinal %d beyond %d", dev, kNoAllocMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    DFL_CUDA(cudaGetSymbolAddress(&p, g_noalloc_keys), "cudaGetSymbolAddress");
+    g_noalloc_ptr[dev] = static_cast<unsigned long long*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return DFLASH_OK;
+}
+
+}  // namespace
+}  // namespace dfl
+
+extern "C" dflash_status dflash_lmhead_argmax_noalloc(const dflash_config* cfg, int64_t M,
+                                                      const void* x, const void* w_lm,
+                                                      int32_t* tok, float* max_logit,
+                                                      void* stream) {
+  dflash_status s = check_config(cfg);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(M >= 0 && M <= kNoAllocMaxTokens, DFLASH_EINVAL,
+            "M = %lld exceeds the %lld tokens this allocation-free variant can hold",
+            static_cast<long long>(M), static_cast<long long>(kNoAllocMaxTokens));
+  if (M == 0) return DFLASH_OK;
+  DFL_PTR(x, "x");
+  DFL_PTR(w_lm, "w_lm");
+  DFL_CHECK(tok != nullptr, DFLASH_EINVAL, "tok is NULL");
+  unsigned long long* keys = nullptr;
+  if ((s = noalloc_scratch(&keys)) != DFLASH_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the array keeps the previous call's contents: the keys must start at zero
+  DFL_CUDA(launch_zero(keys, static_cast<size_t>(M) * 8, st), "argmax key reset");
+  DFL_CUDA(launch_lmhead_argmax(cfg->dtype, w_lm, cfg->vocab, x, M, cfg->hidden, keys, nullptr,
+                                st),
+           "LM head argmax");
+  DFL_CUDA(launch_argmax_finish(keys, M, cfg->block, nullptr, nullptr, tok, max_logit, st),
+           "argmax finish");
+  return DFLASH_OK;
+}

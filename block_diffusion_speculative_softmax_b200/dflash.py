@@ -83,6 +83,7 @@ SIGNATURES = {
     "dflash_draft_step": (C.c_int, [_CFG, C.POINTER(Weights), C.POINTER(StepArgs), _VP, _SZ,
                                     _VP]),
     "dflash_selftest_wait_timeout": (C.c_int, [_VP, _SZ, _I64, _VP]),
+    "dflash_lmhead_argmax_noalloc": (C.c_int, [_CFG, _I64, _VP, _VP, _VP, _VP, _VP]),
 }
 
 _lib = None
@@ -206,6 +207,14 @@ def dflash_mlp(cfg: Config, h, g_mlp, w_gate, w_up, w_down, ws, stream=None):
 def dflash_lmhead_argmax(cfg: Config, x, w_lm, tok, max_logit, ws, stream=None):
     _check(load().dflash_lmhead_argmax(C.byref(cfg), x.shape[0], _p(x), _p(w_lm), _p(tok),
                                        _p(max_logit), _p(ws), ws.numel(), _stream(stream)))
+
+
+def dflash_lmhead_argmax_noalloc(cfg: Config, x, w_lm, tok, max_logit=None, stream=None):
+    """LM-head argmax without a workspace, for callers that cannot allocate
+    device memory (scratch lives in the library's device globals; at most
+    4096 tokens per call; concurrent calls on one device race)."""
+    _check(load().dflash_lmhead_argmax_noalloc(C.byref(cfg), x.shape[0], _p(x), _p(w_lm),
+                                               _p(tok), _p(max_logit), _stream(stream)))
 
 
 def dflash_accept(draft: torch.Tensor, target: torch.Tensor, n_acc, best_k, out_tok,

@@ -217,6 +217,25 @@ dflash_status dflash_d2sd_candidates(int32_t R, int32_t B, int32_t K,
                                      int32_t* cand_tokens, int32_t* block_req,
                                      void* stream);
 
+/* LM-head argmax that allocates nothing and takes no workspace.  The pages
+ * have no counterpart to this entry point; it exists for callers that cannot
+ * call cudaMalloc or hand over a workspace -- e.g. a plugin inside a serving
+ * process whose device memory belongs to that process's caching allocator,
+ * or a real-time loop that must not allocate after start-up.
+ * Computes exactly what dflash_lmhead_argmax computes.  Its scratch (one
+ * 8-byte key per token) is a fixed array in the library's device globals,
+ * present on every GPU that loads the library until the process exits, so:
+ *   - M may be at most 4096 tokens; larger M returns DFLASH_EINVAL;
+ *   - the first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture;
+ *   - all calls share the array: calls that overlap on the GPU (different
+ *     streams, or different host threads on one device) race;
+ *   - non-finite logits are not reported (there is no workspace header). */
+dflash_status dflash_lmhead_argmax_noalloc(const dflash_config* cfg, int64_t M,
+                                           const void* x, const void* w_lm,
+                                           int32_t* tok, float* max_logit,
+                                           void* stream);
+
 /* ------------------------------------------------------------------------
  * The whole draft step (+ optional verification)
  * ----------------------------------------------------------------------*/
