@@ -393,6 +393,299 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
   }
 }
 
+// ---------------------------------------------------------------------------
+// Token-major variant for M >= 128 tokens (the context K/V projection over
+// L rows, and every GEMM when many blocks are drafted together): the TOKENS
+// sit on UMMA M (128 per tile) and the weight rows on N (BW = 128 or 256
+// features per tile), so each epilogue thread owns one token row of the
+// accumulator.  RoPE pairs (i, i + d/2), the gate and up halves of a SwiGLU
+// tile, a residual row and an argmax over the tile's vocabulary rows are
+// all formed in that thread's registers, straight out of TMEM.
+// ---------------------------------------------------------------------------
+template <int BW, int STAGES, bool ARGMAX>
+__global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant__ Params p) {
+  constexpr int X_BYTES = BM * BK * 2;        // 128 tokens x 64 k
+  constexpr int W_BYTES = BW * BK * 2;
+  constexpr int STAGE = X_BYTES + W_BYTES;
+  constexpr uint32_t TMEM_COLS = BW;
+  constexpr uint32_t IDESC = idesc_bf16(BM, BW);
+  static_assert(STAGE % 1024 == 0, "stages must stay 1024-byte aligned");
+
+  extern __shared__ uint8_t dsmem[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t acc_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;
+  __shared__ int s_last;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
+
+  const int tile = blockIdx.x;                // feature tile
+  int sg = 0;
+  while (sg + 1 < p.nseg && tile >= p.seg[sg + 1].tile_begin) ++sg;
+  const Seg& S = p.seg[sg];
+  const int pair = S.pair;
+  const int f0 = (tile - S.tile_begin) * (pair ? BW / 2 : BW);   // first output feature
+  const int tok0 = blockIdx.y * BM;
+  const int kb0 = blockIdx.z * p.kb_per_split;
+  const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
+  const int nkb = kb1 - kb0;
+  const CUtensorMap* tma = &p.tm[S.map];
+  const CUtensorMap* tmb = pair ? &p.tm[S.map + 1] : nullptr;
+
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&acc_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(tma);
+    if (tmb) tma_prefetch_desc(tmb);
+    tma_prefetch_desc(&p.tm_x);
+  }
+  if (warp == 2) tmem_alloc(&tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  if (tid == 0) pdl_launch();
+
+  // stage layout: [X tile 16 KB][W tile BW x 128 B]
+  auto load_w = [&](int i, uint8_t* sw) {
+    const int kc = (kb0 + i) * BK;
+    if (pair) {
+      tma_load_2d(sw, tma, &full_bar[i % STAGES], kc, f0);
+      tma_load_2d(sw + W_BYTES / 2, tmb, &full_bar[i % STAGES], kc, f0);
+    } else {
+      tma_load_2d(sw, tma, &full_bar[i % STAGES], kc, f0);
+    }
+  };
+
+  if (warp == 0 && lane == 0) {
+    const int npre = min(STAGES, nkb);
+    for (int i = 0; i < npre; ++i) {
+      mbar_arrive_expect_tx(&full_bar[i], STAGE);
+      load_w(i, smem + i * STAGE + X_BYTES);
+    }
+    pdl_wait();
+    for (int i = 0; i < npre; ++i)
+      tma_load_2d(smem + i * STAGE, &p.tm_x, &full_bar[i], (kb0 + i) * BK, tok0);
+    int issued = npre;
+    for (int i = npre; i < nkb; ++i) {
+      const int s = i % STAGES;
+      if (!mbar_wait(&empty_bar[s], ((i / STAGES) & 1) ^ 1, p.status, 31)) {
+        abort_flag = 1;
+        break;
+      }
+      if (abort_flag) break;
+      uint8_t* sa = smem + s * STAGE;
+      mbar_arrive_expect_tx(&full_bar[s], STAGE);
+      load_w(i, sa + X_BYTES);
+      tma_load_2d(sa, &p.tm_x, &full_bar[s], (kb0 + i) * BK, tok0);
+      ++issued;
+    }
+    if (abort_flag) {
+      for (int i = max(0, issued - STAGES); i < issued; ++i)
+        mbar_wait(&full_bar[i % STAGES], (i / STAGES) & 1, p.status, 32);
+    }
+  } else if (warp == 1 && lane == 0) {
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % STAGES;
+      if (!mbar_wait(&full_bar[s], (i / STAGES) & 1, p.status, 33)) {
+        abort_flag = 1;
+        break;
+      }
+      if (abort_flag) break;
+      tc_fence_after();
+      const uint8_t* sa = smem + s * STAGE;
+      const uint64_t da = smem_desc_sw128(sa);
+      const uint64_t db = smem_desc_sw128(sa + X_BYTES);
+#pragma unroll
+      for (int k = 0; k < BK / UK; ++k)
+        tc_mma_bf16(tmem, da + 2 * k, db + 2 * k, IDESC, (i > 0 || k > 0) ? 1u : 0u);
+      tc_commit(&empty_bar[s]);
+    }
+    tc_commit(&acc_bar);
+  }
+  __syncwarp();
+
+  // ---------------- epilogue: thread = token row tok0 + tid
+  const bool ok = mbar_wait(&acc_bar, 0, p.status, 34);
+  tc_fence_after();
+  pdl_wait();
+  const bool live = ok && !abort_flag;
+  const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const int t = tok0 + tid;
+  const bool tv = t < p.M;
+  const int tile_lin = blockIdx.y * p.row_tiles + blockIdx.x;
+
+  // split-K: every split parks its fp32 tile, the last one sums them
+  bool do_op = live;
+  float* mine = nullptr;
+  if (p.splits > 1) {
+    mine = p.partial + (static_cast<size_t>(tile_lin) * p.splits + blockIdx.z) * BM * BW +
+           static_cast<size_t>(tid) * BW;
+    if (live) {
+#pragma unroll 1
+      for (int c = 0; c < BW; c += 16) {
+        float v[16];
+        tmem_ld16(lane_addr + c, v);
+#pragma unroll
+        for (int q = 0; q < 16; q += 4)
+          __stcg(reinterpret_cast<float4*>(mine + c + q), make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]));
+      }
+      __threadfence();
+    }
+    __syncthreads();
+    if (tid == 0) {
+      const uint32_t prev = live ? atomicAdd(p.counters + tile_lin, 1u) : 0u;
+      s_last = live && prev == static_cast<uint32_t>(p.splits - 1);
+    }
+    __syncthreads();
+    do_op = s_last != 0;
+    if (do_op) __threadfence();
+  }
+  const float* rowbase = p.partial + static_cast<size_t>(tile_lin) * p.splits * BM * BW +
+                         static_cast<size_t>(tid) * BW;
+  // 16 accumulator columns [c, c + 16) of this thread's token row
+  auto cols = [&](int c, float* v) {
+    if (p.splits == 1) {
+      tmem_ld16(lane_addr + c, v);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 16; ++q) v[q] = 0.f;
+      for (int s = 0; s < p.splits; ++s) {
+        const float4* src = reinterpret_cast<const float4*>(rowbase + static_cast<size_t>(s) * BM * BW + c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 a = __ldcg(src + q);
+          v[4 * q] += a.x; v[4 * q + 1] += a.y; v[4 * q + 2] += a.z; v[4 * q + 3] += a.w;
+        }
+      }
+    }
+  };
+
+  if (do_op) {
+    if constexpr (ARGMAX) {
+      unsigned long long best = 0ull;
+#pragma unroll 1
+      for (int c = 0; c < BW; c += 16) {
+        float v[16];
+        cols(c, v);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const int f = f0 + c + q;
+          if (f < S.rows) {
+            if (!isfinite(v[q]) && tv) report(p.status, DFLASH_ENUMERIC, 35);
+            const unsigned long long k = argmax_key(v[q], static_cast<uint32_t>(f));
+            best = k > best ? k : best;
+          }
+        }
+      }
+      if (tv && best) atomicMax(p.keys + t, best);
+    } else if (S.op == EPI_SWIGLU) {
+      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out) + static_cast<int64_t>(t) * S.out_stride;
+#pragma unroll 1
+      for (int c = 0; c < BW / 2; c += 16) {
+        float g[16], u[16];
+        cols(c, g);
+        cols(BW / 2 + c, u);
+        if (tv) {
+          alignas(16) __nv_bfloat16 r[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) r[q] = __float2bfloat16_rn(g[q] / (1.f + __expf(-g[q])) * u[q]);
+          const int f = f0 + c;
+          if (f + 16 <= S.rows) {
+            reinterpret_cast<uint4*>(o + f)[0] = reinterpret_cast<const uint4*>(r)[0];
+            reinterpret_cast<uint4*>(o + f)[1] = reinterpret_cast<const uint4*>(r)[1];
+          } else {
+            for (int q = 0; q < 16 && f + q < S.rows; ++q) o[f + q] = r[q];
+          }
+        }
+      }
+    } else if (S.op == EPI_RESID) {
+      float* h = static_cast<float*>(S.out) + static_cast<int64_t>(t) * S.out_stride;
+#pragma unroll 1
+      for (int c = 0; c < BW; c += 16) {
+        float v[16];
+        cols(c, v);
+        const int f = f0 + c;
+        if (tv) {
+          if (f + 16 <= S.rows) {
+#pragma unroll
+            for (int q = 0; q < 16; q += 4) {
+              float4 a = *reinterpret_cast<float4*>(h + f + q);
+              a.x += v[q]; a.y += v[q + 1]; a.z += v[q + 2]; a.w += v[q + 3];
+              *reinterpret_cast<float4*>(h + f + q) = a;
+            }
+          } else {
+            for (int q = 0; q < 16 && f + q < S.rows; ++q) h[f + q] += v[q];
+          }
+        }
+      }
+    } else {   // EPI_STORE, optional RoPE over heads of head_dim
+      const int64_t orow = tv ? (S.use_dst ? p.dst[t] : t) : 0;
+      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out) + orow * S.out_stride;
+      const int d = p.head_dim, half = d >> 1;
+      const int pos = (tv && S.rope) ? p.pos[t] : 0;
+      auto put16 = [&](int f, const float* v) {
+        alignas(16) __nv_bfloat16 r[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) r[q] = __float2bfloat16_rn(v[q]);
+        if (f + 16 <= S.rows) {
+          reinterpret_cast<uint4*>(o + f)[0] = reinterpret_cast<const uint4*>(r)[0];
+          reinterpret_cast<uint4*>(o + f)[1] = reinterpret_cast<const uint4*>(r)[1];
+        } else {
+          for (int q = 0; q < 16 && f + q < S.rows; ++q) o[f + q] = r[q];
+        }
+      };
+      if (S.rope) {
+        // chunk c of the first half of a head pairs with chunk c + d/2
+#pragma unroll 1
+        for (int c = 0; c < BW; c += 16) {
+          const int i = c % d;
+          if (i >= half) continue;
+          float a[16], b[16];
+          cols(c, a);
+          cols(c + half, b);
+          if (tv) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const float2 cs = rope_cs(p, pos, i + q);
+              const float x1 = a[q], x2 = b[q];
+              a[q] = x1 * cs.x - x2 * cs.y;
+              b[q] = x2 * cs.x + x1 * cs.y;
+            }
+            put16(f0 + c, a);
+            put16(f0 + c + half, b);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BW; c += 16) {
+          float v[16];
+          cols(c, v);
+          if (tv) put16(f0 + c, v);
+        }
+      }
+    }
+    if (p.splits > 1 && tid == 0) p.counters[tile_lin] = 0u;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 template <int BN, int STAGES, bool ARGMAX>
 cudaError_t launch(const Params& p, dim3 grid, cudaStream_t st) {
   constexpr int SMEM = STAGES * (A_BYTES + BN * BK * 2) + 1024;
@@ -418,6 +711,31 @@ cudaError_t dispatch(int bn, const Params& p, dim3 grid, cudaStream_t st) {
     default: return cudaErrorInvalidValue;
   }
 }
+
+template <int BW, int STAGES, bool ARGMAX>
+cudaError_t launch_tok(const Params& p, dim3 grid, cudaStream_t st) {
+  constexpr int SMEM = STAGES * (BM * BK * 2 + BW * BK * 2) + 1024;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_tok_kernel<BW, STAGES, ARGMAX>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  return launch_k(gemm_tok_kernel<BW, STAGES, ARGMAX>, grid, dim3(128), SMEM, st, p);
+}
+
+template <bool ARGMAX>
+cudaError_t dispatch_tok(int bw, const Params& p, dim3 grid, cudaStream_t st) {
+  switch (bw) {
+    case 128: return launch_tok<128, 6, ARGMAX>(p, grid, st);   // 192 KB ring
+    case 256: return launch_tok<256, 4, ARGMAX>(p, grid, st);   // 192 KB ring
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Tokens at or above which the token-major kernel is used.
+constexpr int64_t kTokMajorMin = 128;
 
 inline int pick_bn(int64_t M) {
   if (M <= 16) return 16;
@@ -649,27 +967,43 @@ GemmPlan plan_gemm(const GemmJob& job) {
   const int64_t M = job.M;
   int n_cols = 0;
   if (job.dtype == DFLASH_BF16) {
-    for (int s = 0; s < job.nseg; ++s)
-      pl.row_tiles += job.seg[s].op == EPI_SWIGLU ? ceil_div(job.seg[s].rows, tc::BM / 2)
-                                                  : ceil_div(job.seg[s].rows, tc::BM);
-    pl.bn = tc::pick_bn(M);
-    pl.tok_tiles = ceil_div(M, pl.bn);
     const int kb_total = ceil_div(job.K, tc::BK);
-    const int tiles = pl.row_tiles * pl.tok_tiles;
+    auto feature_tiles = [&](int per_tile) {
+      int n = 0;
+      for (int s = 0; s < job.nseg; ++s)
+        n += job.seg[s].op == EPI_SWIGLU ? ceil_div(job.seg[s].rows, per_tile / 2)
+                                         : ceil_div(job.seg[s].rows, per_tile);
+      return n;
+    };
     int splits = 1;
-    if (pl.bn <= 64) {
-      // weight streaming: about two CTAs per SM in flight
-      const int target = kNumSMs * tc::ctas_per_sm(pl.bn);
-      if (tiles < target) splits = std::min(kb_total, ceil_div(target, tiles));
-    } else if (tiles * 2 < kNumSMs) {
-      // tensor-bound: split only when fewer than half the SMs have a tile
-      splits = std::min(kb_total, ceil_div(kNumSMs, tiles));
+    if (M >= tc::kTokMajorMin) {
+      // token-major: 128 tokens x BW features per tile, tensor-bound
+      pl.tok_major = 1;
+      pl.tok_tiles = ceil_div(M, tc::BM);
+      pl.bn = 256;
+      pl.row_tiles = feature_tiles(256);
+      if (pl.row_tiles * pl.tok_tiles * 2 < kNumSMs) {   // under half the SMs busy
+        pl.bn = 128;
+        pl.row_tiles = feature_tiles(128);
+      }
+      const int tiles = pl.row_tiles * pl.tok_tiles;
+      if (tiles * 2 < kNumSMs) splits = std::min(kb_total, kNumSMs / tiles);
+    } else {
+      // weight-major (swap-AB): 128 weight rows x BN tokens, weight streaming;
+      // split K so about two CTAs per SM stream at once, never more than fit
+      pl.bn = tc::pick_bn(M);
+      pl.tok_tiles = ceil_div(M, pl.bn);
+      pl.row_tiles = feature_tiles(tc::BM);
+      const int tiles = pl.row_tiles * pl.tok_tiles;
+      const int slots = kNumSMs * tc::ctas_per_sm(pl.bn);
+      if (tiles < slots) splits = std::max(1, std::min(kb_total, slots / tiles));
     }
     splits = std::max(1, std::min(splits, 32));
     pl.kb_per_split = ceil_div(kb_total, splits);
     pl.splits = ceil_div(kb_total, pl.kb_per_split);
-    pl.partial_floats = pl.splits > 1 ? static_cast<size_t>(tiles) * pl.splits * pl.bn * tc::BM
-                                      : 0;
+    const int tiles = pl.row_tiles * pl.tok_tiles;
+    pl.partial_floats =
+        pl.splits > 1 ? static_cast<size_t>(tiles) * pl.splits * pl.bn * tc::BM : 0;
     pl.counters = pl.splits > 1 ? tiles : 0;
     return pl;
   }
@@ -758,19 +1092,23 @@ cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& pl, float* partial,
     S.use_dst = o.use_dst;
     S.out_stride = o.out_stride;
     S.out = o.out;
+    // rows of one weight box: the tile's feature count (half of it per
+    // matrix for a SwiGLU pair)
+    const int per_tile = pl.tok_major ? pl.bn : tc::BM;
     if (S.pair) {
-      if (!encode_tmap_bf16_2d(&p.tm[maps++], o.w0, job.K, o.rows, tc::BK, tc::BM / 2) ||
-          !encode_tmap_bf16_2d(&p.tm[maps++], o.w1, job.K, o.rows, tc::BK, tc::BM / 2))
+      if (!encode_tmap_bf16_2d(&p.tm[maps++], o.w0, job.K, o.rows, tc::BK, per_tile / 2) ||
+          !encode_tmap_bf16_2d(&p.tm[maps++], o.w1, job.K, o.rows, tc::BK, per_tile / 2))
         return cudaErrorInvalidValue;
-      tiles += ceil_div(o.rows, tc::BM / 2);
+      tiles += ceil_div(o.rows, per_tile / 2);
     } else {
-      if (!encode_tmap_bf16_2d(&p.tm[maps++], o.w0, job.K, o.rows, tc::BK, tc::BM))
+      if (!encode_tmap_bf16_2d(&p.tm[maps++], o.w0, job.K, o.rows, tc::BK, per_tile))
         return cudaErrorInvalidValue;
-      tiles += ceil_div(o.rows, tc::BM);
+      tiles += ceil_div(o.rows, per_tile);
     }
     if (maps > 4) return cudaErrorInvalidValue;
   }
-  if (!encode_tmap_bf16_2d(&p.tm_x, job.x, job.K, job.M, tc::BK, pl.bn))
+  if (!encode_tmap_bf16_2d(&p.tm_x, job.x, job.K, job.M, tc::BK,
+                           pl.tok_major ? tc::BM : pl.bn))
     return cudaErrorInvalidValue;
   p.nseg = job.nseg;
   p.M = static_cast<int>(job.M);
@@ -788,6 +1126,7 @@ cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& pl, float* partial,
   fill_inv_freq(job.theta, p.head_dim, p.inv_freq);
   p.status = status;
   dim3 grid(tiles, pl.tok_tiles, pl.splits);
+  if (pl.tok_major) return tc::dispatch_tok<false>(pl.bn, p, grid, st);
   return tc::dispatch<false>(pl.bn, p, grid, st);
 }
 
@@ -795,6 +1134,23 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X,
                                  int K, unsigned long long* keys, uint32_t* status,
                                  cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
+  if (dtype == DFLASH_BF16 && M >= tc::kTokMajorMin) {
+    tc::Params p{};
+    constexpr int BW = 256;
+    if (!encode_tmap_bf16_2d(&p.tm[0], W, K, V, tc::BK, BW)) return cudaErrorInvalidValue;
+    if (!encode_tmap_bf16_2d(&p.tm_x, X, K, M, tc::BK, tc::BM)) return cudaErrorInvalidValue;
+    p.seg[0].rows = V;
+    p.nseg = 1;
+    p.M = static_cast<int>(M);
+    p.kb_total = ceil_div(K, tc::BK);
+    p.kb_per_split = p.kb_total;
+    p.splits = 1;
+    p.row_tiles = ceil_div(V, BW);
+    p.keys = keys;
+    p.status = status;
+    dim3 grid(ceil_div(V, BW), ceil_div(M, tc::BM), 1);
+    return tc::dispatch_tok<true>(BW, p, grid, st);
+  }
   if (dtype == DFLASH_BF16) {
     tc::Params p{};
     if (!encode_tmap_bf16_2d(&p.tm[0], W, K, V, tc::BK, tc::BM)) return cudaErrorInvalidValue;

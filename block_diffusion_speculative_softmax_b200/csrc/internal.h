@@ -57,7 +57,8 @@ struct GemmJob {
 };
 
 struct GemmPlan {
-  int bn;            // token tile
+  int tok_major;     // 1: tokens on the MMA's M (large M), features per tile = bn
+  int bn;            // token tile (weight-major) or feature tile (token-major)
   int row_tiles;     // tiles along the output features (all segments)
   int tok_tiles;
   int splits;        // K splits

@@ -258,19 +258,26 @@ cudaError_t launch_embed(int dtype, const void* embed, int H, int nb, int B,
 }
 
 // ===========================================================================
-// RMSNorm of the fp32 residual stream into the GEMM input dtype
+// RMSNorm of the fp32 residual stream into the GEMM input dtype.  One CTA
+// per row; every thread holds up to two float4 of the row in registers, so
+// the row is read once with all loads in flight.
 // ===========================================================================
 template <typename T>
-__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ h, int H,
-                                                      const float* __restrict__ g, float eps,
-                                                      T* __restrict__ x) {
-  __shared__ float red[8];
+__global__ void __launch_bounds__(1024) rmsnorm_kernel(const float* __restrict__ h, int H,
+                                                       const float* __restrict__ g, float eps,
+                                                       T* __restrict__ x) {
+  __shared__ float red[32];
   pdl_wait();
   if (threadIdx.x == 0) pdl_launch();
   const int64_t m = blockIdx.x;
-  const float* row = h + m * H;
-  float ss = 0.f;
-  for (int c = threadIdx.x; c < H; c += blockDim.x) ss = fmaf(row[c], row[c], ss);
+  const int nv = H >> 2;
+  const int i0 = threadIdx.x, i1 = threadIdx.x + blockDim.x;
+  const float4* row = reinterpret_cast<const float4*>(h + m * H);
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4 a = i0 < nv ? row[i0] : z;
+  const float4 b = i1 < nv ? row[i1] : z;
+  float ss = a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w + b.x * b.x + b.y * b.y + b.z * b.z +
+             b.w * b.w;
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
@@ -281,17 +288,33 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
   }
   __syncthreads();
   const float sc = red[0];
-  for (int c = threadIdx.x; c < H; c += blockDim.x) x[m * H + c] = from_f<T>(row[c] * sc * g[c]);
+  const float4* gv = reinterpret_cast<const float4*>(g);
+  T* out = x + m * H;
+  if (i0 < nv) {
+    const float4 q = __ldg(gv + i0);
+    const float o[4] = {a.x * sc * q.x, a.y * sc * q.y, a.z * sc * q.z, a.w * sc * q.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) out[4 * i0 + e] = from_f<T>(o[e]);
+  }
+  if (i1 < nv) {
+    const float4 q = __ldg(gv + i1);
+    const float o[4] = {b.x * sc * q.x, b.y * sc * q.y, b.z * sc * q.z, b.w * sc * q.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) out[4 * i1 + e] = from_f<T>(o[e]);
+  }
 }
 
 cudaError_t launch_rmsnorm(int dtype, const float* h, int64_t M, int H, const float* g, float eps,
                            void* x, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
+  const int nv = H / 4;
+  const int threads = std::min(1024, ((nv + 1) / 2 + 31) / 32 * 32);
+  if (2 * threads < nv || H % 4) return cudaErrorInvalidValue;
   if (dtype == DFLASH_BF16)
-    return launch_k(rmsnorm_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(M)), dim3(256), 0,
-                    st, h, H, g, eps, static_cast<__nv_bfloat16*>(x));
-  return launch_k(rmsnorm_kernel<float>, dim3(static_cast<unsigned>(M)), dim3(256), 0, st, h, H,
-                  g, eps, static_cast<float*>(x));
+    return launch_k(rmsnorm_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(M)), dim3(threads),
+                    0, st, h, H, g, eps, static_cast<__nv_bfloat16*>(x));
+  return launch_k(rmsnorm_kernel<float>, dim3(static_cast<unsigned>(M)), dim3(threads), 0, st, h,
+                  H, g, eps, static_cast<float*>(x));
 }
 
 // ===========================================================================
