@@ -168,6 +168,7 @@ Needs step_needs(const dflash_config* c, int64_t M, int64_t n_new) {
     n.take(plan_gemm(job_resid(c, nullptr, nullptr, M, c->n_q_heads * c->head_dim, 0)));
     n.take(plan_gemm(job_swiglu(c, nullptr, nullptr, nullptr, M, 0)));
     n.take(plan_gemm(job_resid(c, nullptr, nullptr, M, c->ffn, 0)));
+    n.take(plan_lmhead(c->dtype, c->vocab, M, c->hidden));
   }
   return n;
 }
@@ -403,12 +404,19 @@ dflash_status dflash_lmhead_argmax(const dflash_config* cfg, int64_t M, const vo
   DFL_PTR(x, "x");
   DFL_PTR(w_lm, "w_lm");
   DFL_CHECK(tok != nullptr, DFLASH_EINVAL, "tok is NULL");
-  if ((s = check_ws(ws, ws_bytes, sizeof(DevStatus) + M * 8)) != DFLASH_OK) return s;
+  const GemmPlan pl = plan_lmhead(cfg->dtype, cfg->vocab, M, cfg->hidden);
+  const size_t off_keys = sizeof(DevStatus);
+  const size_t off_cnt = align256(off_keys + M * 8);
+  const size_t off_part = align256(off_cnt + pl.counters * 4);
+  if ((s = check_ws(ws, ws_bytes, off_part + pl.partial_floats * 4)) != DFLASH_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  auto* keys = at<unsigned long long>(ws, sizeof(DevStatus));
-  DFL_CUDA(launch_zero(keys, M * 8, st), "argmax key reset");
+  auto* keys = at<unsigned long long>(ws, off_keys);
+  // keys and tile counters start at zero
+  DFL_CUDA(launch_zero(keys, off_part - off_keys, st), "argmax key reset");
   DFL_CUDA(launch_lmhead_argmax(cfg->dtype, w_lm, cfg->vocab, x, M, cfg->hidden, keys,
-                                status_word(ws), st),
+                                status_word(ws), st,
+                                pl.stream_k ? at<float>(ws, off_part) : nullptr,
+                                pl.stream_k ? at<uint32_t>(ws, off_cnt) : nullptr),
            "LM head argmax");
   DFL_CUDA(launch_argmax_finish(keys, M, cfg->block, nullptr, nullptr, tok, max_logit, st),
            "argmax finish");
@@ -577,7 +585,8 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
       return s;
   }
   DFL_CUDA(launch_rmsnorm(dt, h, M, H, w->g_final, c->rms_eps, x, st), "final rmsnorm");
-  DFL_CUDA(launch_lmhead_argmax(dt, w->lm_head, c->vocab, x, M, H, keys, status, st),
+  DFL_CUDA(launch_lmhead_argmax(dt, w->lm_head, c->vocab, x, M, H, keys, status, st, partial,
+                                counters),
            "LM head argmax");
   DFL_CUDA(launch_argmax_finish(keys, M, c->block, a->block_tokens, a->known_len,
                                 a->draft_tokens, a->max_logit, st),

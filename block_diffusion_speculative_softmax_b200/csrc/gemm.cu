@@ -686,6 +686,371 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
   }
 }
 
+// ---------------------------------------------------------------------------
+// Stream-K weight-major variant for M <= 64 tokens (weight streaming at small
+// batch).  A persistent grid of one CTA per SM; the (tile, k-block) work
+// units of the whole GEMM are cut into G equal contiguous ranges, one per
+// CTA, so every SM streams the same number of weight bytes whatever the
+// tile count.  Warp 0 issues TMA, warp 1 issues tcgen05.mma, warps 2..5
+// drain TMEM; the accumulator is double-buffered in TMEM so a finished
+// tile is drained while the next one accumulates.  A tile whose k range is
+// shared by several CTAs is reduced by the last contributor, slots summed
+// in CTA order (deterministic).
+// ---------------------------------------------------------------------------
+struct SkGeom {
+  int64_t units;     // tiles * kb_total
+  int grid;          // G
+  int max_slots;     // partial slots reserved per tile
+};
+
+__device__ __forceinline__ int64_t sk_u0(int64_t units, int grid, int c) {
+  return (static_cast<int64_t>(c) * units) / grid;
+}
+// CTA owning unit u: the largest c with u0(c) <= u.
+__device__ __forceinline__ int sk_cta_of(int64_t units, int grid, int64_t u) {
+  return static_cast<int>(((u + 1) * grid - 1) / units);
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <int BN, int STAGES, bool ARGMAX>
+__global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__ Params p,
+                                                         const SkGeom geo) {
+  constexpr int B_BYTES = BN * BK * 2;
+  constexpr int STAGE = A_BYTES + B_BYTES;
+  constexpr uint32_t ACC_COLS = BN < 32 ? 32 : BN;
+  constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+  constexpr uint32_t IDESC = idesc_bf16(BM, BN);
+  constexpr int EPI = 128;                     // epilogue threads (warps 2..5)
+  static_assert(STAGE % 1024 == 0, "stages must stay 1024-byte aligned");
+
+  extern __shared__ uint8_t dsmem[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  float* st = reinterpret_cast<float*>(smem + STAGES * STAGE);   // staging [BN][SROW]
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t accf_bar[2];
+  __shared__ __align__(8) uint64_t acce_bar[2];
+  __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;
+  __shared__ int s_last;
+  __shared__ unsigned long long red[ARGMAX ? 4 : 1][ARGMAX ? BN : 1];
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int kbt = p.kb_total;
+  const int64_t u0 = sk_u0(geo.units, geo.grid, blockIdx.x);
+  const int64_t u1 = sk_u0(geo.units, geo.grid, blockIdx.x + 1);
+  const int n_units = static_cast<int>(u1 - u0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf_bar[b], 1);
+      mbar_init(&acce_bar[b], EPI);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+    for (int g = 0; g < p.nseg; ++g) {
+      tma_prefetch_desc(&p.tm[p.seg[g].map]);
+      if (p.seg[g].pair) tma_prefetch_desc(&p.tm[p.seg[g].map + 1]);
+    }
+    tma_prefetch_desc(&p.tm_x);
+  }
+  if (warp == 2) tmem_alloc(&tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  if (threadIdx.x == 0) pdl_launch();
+
+  // tile -> (segment, first weight row, first token)
+  auto tile_info = [&](int tile, int& sg, int& row0, int& tok0) {
+    const int rt = tile % p.row_tiles, tt = tile / p.row_tiles;
+    sg = 0;
+    while (sg + 1 < p.nseg && rt >= p.seg[sg + 1].tile_begin) ++sg;
+    row0 = (rt - p.seg[sg].tile_begin) * (p.seg[sg].pair ? BM / 2 : BM);
+    tok0 = tt * BN;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer over this CTA's units
+      auto load_w = [&](int i, uint8_t* sa) {
+        const int64_t u = u0 + i;
+        int sg, row0, tok0;
+        tile_info(static_cast<int>(u / kbt), sg, row0, tok0);
+        const int kc = static_cast<int>(u % kbt) * BK;
+        const Seg& S = p.seg[sg];
+        if (S.pair) {
+          tma_load_2d(sa, &p.tm[S.map], &full_bar[i % STAGES], kc, row0);
+          tma_load_2d(sa + A_BYTES / 2, &p.tm[S.map + 1], &full_bar[i % STAGES], kc, row0);
+        } else {
+          tma_load_2d(sa, &p.tm[S.map], &full_bar[i % STAGES], kc, row0);
+        }
+      };
+      auto load_x = [&](int i, uint8_t* sa) {
+        const int64_t u = u0 + i;
+        int sg, row0, tok0;
+        tile_info(static_cast<int>(u / kbt), sg, row0, tok0);
+        tma_load_2d(sa + A_BYTES, &p.tm_x, &full_bar[i % STAGES], static_cast<int>(u % kbt) * BK,
+                    tok0);
+      };
+      const int npre = min(STAGES, n_units);
+      for (int i = 0; i < npre; ++i) {
+        mbar_arrive_expect_tx(&full_bar[i], STAGE);
+        load_w(i, smem + i * STAGE);
+      }
+      pdl_wait();
+      for (int i = 0; i < npre; ++i) load_x(i, smem + i * STAGE);
+      int issued = npre;
+      for (int i = npre; i < n_units; ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&empty_bar[s], ((i / STAGES) & 1) ^ 1, p.status, 41)) {
+          abort_flag = 1;
+          break;
+        }
+        if (abort_flag) break;
+        uint8_t* sa = smem + s * STAGE;
+        mbar_arrive_expect_tx(&full_bar[s], STAGE);
+        load_w(i, sa);
+        load_x(i, sa);
+        ++issued;
+      }
+      if (abort_flag) {
+        for (int i = max(0, issued - STAGES); i < issued; ++i)
+          mbar_wait(&full_bar[i % STAGES], (i / STAGES) & 1, p.status, 42);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer; one accumulator buffer per tile segment
+      int seg_i = 0;
+      for (int i = 0; i < n_units; ++i) {
+        const int64_t u = u0 + i;
+        const int k = static_cast<int>(u % kbt);
+        const bool first = (i == 0) || (k == 0);
+        const bool last = (i == n_units - 1) || (k == kbt - 1);
+        const int b = seg_i & 1;
+        if (first && seg_i >= 2) {
+          if (!mbar_wait(&acce_bar[b], ((seg_i >> 1) - 1) & 1, p.status, 43)) {
+            abort_flag = 1;
+          }
+        }
+        const int s = i % STAGES;
+        if (!abort_flag && !mbar_wait(&full_bar[s], (i / STAGES) & 1, p.status, 44)) abort_flag = 1;
+        if (!abort_flag) {
+          tc_fence_after();
+          const uint8_t* sa = smem + s * STAGE;
+          const uint64_t da = smem_desc_sw128(sa);
+          const uint64_t db = smem_desc_sw128(sa + A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk)
+            tc_mma_bf16(tmem + b * ACC_COLS, da + 2 * kk, db + 2 * kk, IDESC,
+                        (first && kk == 0) ? 0u : 1u);
+          tc_commit(&empty_bar[s]);
+        }
+        if (last) {
+          tc_commit(&accf_bar[b]);   // arrives even after an abort, so nobody hangs
+          ++seg_i;
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5: tile row = TMEM lane
+    const int et = threadIdx.x - 64;                  // 0..127
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                // tile row
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    int seg_i = 0;
+    int64_t u = u0;
+    pdl_wait();
+    while (u < u1) {
+      const int tile = static_cast<int>(u / kbt);
+      const int kb_begin = static_cast<int>(u % kbt);
+      const int64_t left = u1 - u;
+      const int seg_len = static_cast<int>(left < kbt - kb_begin ? left : kbt - kb_begin);
+      u += seg_len;
+      const int b = seg_i & 1;
+      const bool ok = mbar_wait(&accf_bar[b], (seg_i >> 1) & 1, p.status, 45);
+      tc_fence_after();
+      float v[BN];
+#pragma unroll
+      for (int c = 0; c < BN; c += 16) tmem_ld16(lane_addr + b * ACC_COLS + c, v + c);
+      tc_fence_before();
+      mbar_arrive(&acce_bar[b]);
+      ++seg_i;
+      const bool live = ok && !abort_flag;
+      int sg, row0, tok0;
+      tile_info(tile, sg, row0, tok0);
+      const Seg& S = p.seg[sg];
+      // contributors to this tile
+      const int c_lo = sk_cta_of(geo.units, geo.grid, static_cast<int64_t>(tile) * kbt);
+      const int c_hi = sk_cta_of(geo.units, geo.grid, static_cast<int64_t>(tile + 1) * kbt - 1);
+      bool do_op = live;
+      if (c_hi > c_lo) {
+        float* slots = p.partial + static_cast<size_t>(tile) * geo.max_slots * BN * BM;
+        float* mine = slots + static_cast<size_t>(blockIdx.x - c_lo) * BN * BM;
+        if (live) {
+#pragma unroll
+          for (int j = 0; j < BN; ++j) __stcg(mine + j * BM + r, v[j]);
+          __threadfence();
+        }
+        named_sync(1, EPI);
+        if (et == 0) {
+          const uint32_t prev = live ? atomicAdd(p.counters + tile, 1u) : 0u;
+          s_last = live && prev == static_cast<uint32_t>(c_hi - c_lo);
+        }
+        named_sync(1, EPI);
+        do_op = s_last != 0;
+        if (do_op) {
+          __threadfence();
+          // the tile's BN x 128 floats as float4 items (token j, rows 4q..4q+3),
+          // each summed over the slots in CTA order, straight into the staging
+          const int nsl = c_hi - c_lo + 1;
+          constexpr int ITEMS = BN * (BM / 4);
+#pragma unroll 1
+          for (int it0 = 0; it0 < ITEMS; it0 += 4 * EPI) {
+            float4 acc[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+            for (int sl = 0; sl < nsl; ++sl) {
+              const float4* src = reinterpret_cast<const float4*>(
+                  slots + static_cast<size_t>(sl) * BN * BM);
+              float4 a[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int it = it0 + q * EPI + et;
+                a[q] = it < ITEMS ? __ldcg(src + it) : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                acc[q].x += a[q].x; acc[q].y += a[q].y; acc[q].z += a[q].z; acc[q].w += a[q].w;
+              }
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int it = it0 + q * EPI + et;
+              if (it < ITEMS) {
+                const int j = it / (BM / 4), rq = (it % (BM / 4)) * 4;
+                *reinterpret_cast<float4*>(st + j * SROW + rq) = acc[q];
+              }
+            }
+          }
+          if (et == 0) p.counters[tile] = 0u;
+        }
+      } else if (do_op) {
+        // stage [BN][SROW] so RoPE partners and SwiGLU halves meet
+#pragma unroll
+        for (int j = 0; j < BN; ++j) st[j * SROW + r] = v[j];
+      }
+      named_sync(1, EPI);
+      if constexpr (ARGMAX) {
+        if (do_op && c_hi > c_lo) {
+#pragma unroll
+          for (int j = 0; j < BN; ++j) v[j] = st[j * SROW + r];
+        }
+      }
+      if (do_op) {
+        if constexpr (ARGMAX) {
+          const int row = row0 + r;
+#pragma unroll
+          for (int j = 0; j < BN; ++j) {
+            unsigned long long key = 0ull;
+            if (row < S.rows && tok0 + j < p.M) {
+              if (!isfinite(v[j])) report(p.status, DFLASH_ENUMERIC, 46);
+              key = argmax_key(v[j], static_cast<uint32_t>(row));
+            }
+            key = warp_max_u64(key);
+            if (lane == 0) red[quarter][j] = key;
+          }
+          named_sync(1, EPI);
+          for (int j = et; j < BN; j += EPI) {
+            unsigned long long k = red[0][j];
+#pragma unroll
+            for (int w = 1; w < 4; ++w) k = red[w][j] > k ? red[w][j] : k;
+            if (tok0 + j < p.M && k != 0ull) atomicMax(p.keys + tok0 + j, k);
+          }
+        } else if (S.op == EPI_SWIGLU) {
+          const int rr = et & 63;
+          const int f = row0 + rr;
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out);
+#pragma unroll 4
+          for (int j = et >> 6; j < BN; j += 2) {
+            const int t = tok0 + j;
+            if (f < S.rows && t < p.M) {
+              const float g = st[j * SROW + rr], uu = st[j * SROW + rr + 64];
+              o[static_cast<int64_t>(t) * S.out_stride + f] =
+                  __float2bfloat16_rn(g / (1.f + __expf(-g)) * uu);
+            }
+          }
+        } else if (S.op == EPI_RESID) {
+          const int f = row0 + et;
+          float* h = static_cast<float*>(S.out) + f;
+          float hv[BN];
+#pragma unroll
+          for (int j = 0; j < BN; ++j) {
+            const int t = tok0 + j;
+            hv[j] = (f < S.rows && t < p.M) ? h[static_cast<int64_t>(t) * S.out_stride] : 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < BN; ++j) {
+            const int t = tok0 + j;
+            if (f < S.rows && t < p.M)
+              h[static_cast<int64_t>(t) * S.out_stride] = hv[j] + st[j * SROW + et];
+          }
+        } else {
+          const int f = row0 + et;
+          const int half = p.head_dim >> 1;
+          const int i = et % p.head_dim;
+          const int prt = i < half ? et + half : et - half;
+          const int fi = i < half ? i : i - half;
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out);
+#pragma unroll 1
+          for (int j0 = 0; j0 < BN; j0 += 8) {
+            float2 cs[8];
+            int64_t orow[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int t = min(tok0 + j0 + q, p.M - 1);
+              cs[q] = S.rope ? rope_cs(p, p.pos[t], fi) : make_float2(1.f, 0.f);
+              orow[q] = S.use_dst ? p.dst[t] : t;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int t = tok0 + j0 + q;
+              if (j0 + q >= BN || f >= S.rows || t >= p.M) continue;
+              float x = st[(j0 + q) * SROW + et];
+              if (S.rope) {
+                const float pv = st[(j0 + q) * SROW + prt];
+                x = i < half ? x * cs[q].x - pv * cs[q].y : x * cs[q].x + pv * cs[q].y;
+              }
+              o[orow[q] * S.out_stride + f] = __float2bfloat16_rn(x);
+            }
+          }
+        }
+      }
+      named_sync(1, EPI);   // staging buffer free for the next tile
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 template <int BN, int STAGES, bool ARGMAX>
 cudaError_t launch(const Params& p, dim3 grid, cudaStream_t st) {
   constexpr int SMEM = STAGES * (A_BYTES + BN * BK * 2) + 1024;
@@ -710,6 +1075,49 @@ cudaError_t dispatch(int bn, const Params& p, dim3 grid, cudaStream_t st) {
     case 256: return launch<256, 4, ARGMAX>(p, grid, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+template <int BN, int STAGES, bool ARGMAX>
+cudaError_t launch_sk(const Params& p, const SkGeom& geo, cudaStream_t st) {
+  constexpr int SMEM = STAGES * (A_BYTES + BN * BK * 2) + BN * SROW * 4 + 1024;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_sk_kernel<BN, STAGES, ARGMAX>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  return launch_k(gemm_sk_kernel<BN, STAGES, ARGMAX>, dim3(geo.grid), dim3(192), SMEM, st, p,
+                  geo);
+}
+
+// One CTA per SM with a ring of ~180 KB.
+template <bool ARGMAX>
+cudaError_t dispatch_sk(int bn, const Params& p, const SkGeom& geo, cudaStream_t st) {
+  switch (bn) {
+    case 16: return launch_sk<16, 10, ARGMAX>(p, geo, st);
+    case 32: return launch_sk<32, 9, ARGMAX>(p, geo, st);
+    case 64: return launch_sk<64, 7, ARGMAX>(p, geo, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Stream-K partition of `tiles` x `kbt` units over at most one CTA per SM:
+// the grid and the largest number of CTAs sharing one tile.
+inline SkGeom sk_geometry(int tiles, int kbt) {
+  SkGeom g{};
+  g.units = static_cast<int64_t>(tiles) * kbt;
+  g.grid = static_cast<int>(std::min<int64_t>(g.units, kNumSMs));
+  g.max_slots = 1;
+  auto u0 = [&](int64_t c) { return (c * g.units) / g.grid; };
+  auto cta_of = [&](int64_t u) { return static_cast<int>(((u + 1) * g.grid - 1) / g.units); };
+  for (int t = 0; t < tiles; ++t) {
+    const int n = cta_of(static_cast<int64_t>(t + 1) * kbt - 1) -
+                  cta_of(static_cast<int64_t>(t) * kbt) + 1;
+    g.max_slots = std::max(g.max_slots, n);
+  }
+  (void)u0;
+  return g;
 }
 
 template <int BW, int STAGES, bool ARGMAX>
@@ -989,14 +1397,22 @@ GemmPlan plan_gemm(const GemmJob& job) {
       const int tiles = pl.row_tiles * pl.tok_tiles;
       if (tiles * 2 < kNumSMs) splits = std::min(kb_total, kNumSMs / tiles);
     } else {
-      // weight-major (swap-AB): 128 weight rows x BN tokens, weight streaming;
-      // split K so about two CTAs per SM stream at once, never more than fit
+      // weight-major (swap-AB), stream-K: 128 weight rows x BN tokens per
+      // tile, the (tile, k-block) units split evenly over one CTA per SM
       pl.bn = tc::pick_bn(M);
       pl.tok_tiles = ceil_div(M, pl.bn);
       pl.row_tiles = feature_tiles(tc::BM);
       const int tiles = pl.row_tiles * pl.tok_tiles;
-      const int slots = kNumSMs * tc::ctas_per_sm(pl.bn);
-      if (tiles < slots) splits = std::max(1, std::min(kb_total, slots / tiles));
+      const tc::SkGeom g = tc::sk_geometry(tiles, kb_total);
+      pl.stream_k = 1;
+      pl.sk_grid = g.grid;
+      pl.sk_slots = g.max_slots;
+      pl.splits = 1;
+      pl.kb_per_split = kb_total;
+      pl.partial_floats =
+          g.max_slots > 1 ? static_cast<size_t>(tiles) * g.max_slots * pl.bn * tc::BM : 0;
+      pl.counters = g.max_slots > 1 ? tiles : 0;
+      return pl;
     }
     splits = std::max(1, std::min(splits, 32));
     pl.kb_per_split = ceil_div(kb_total, splits);
@@ -1125,14 +1541,39 @@ cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& pl, float* partial,
   p.rope_len = job.rope_len;
   fill_inv_freq(job.theta, p.head_dim, p.inv_freq);
   p.status = status;
+  if (pl.stream_k) {
+    tc::SkGeom geo{};
+    geo.units = static_cast<int64_t>(tiles) * pl.tok_tiles * p.kb_total;
+    geo.grid = pl.sk_grid;
+    geo.max_slots = pl.sk_slots;
+    return tc::dispatch_sk<false>(pl.bn, p, geo, st);
+  }
   dim3 grid(tiles, pl.tok_tiles, pl.splits);
   if (pl.tok_major) return tc::dispatch_tok<false>(pl.bn, p, grid, st);
   return tc::dispatch<false>(pl.bn, p, grid, st);
 }
 
+GemmPlan plan_lmhead(int dtype, int V, int64_t M, int K) {
+  GemmPlan pl{};
+  if (dtype != DFLASH_BF16 || M >= tc::kTokMajorMin) return pl;
+  pl.bn = tc::pick_bn(M);
+  pl.tok_tiles = ceil_div(M, pl.bn);
+  pl.row_tiles = ceil_div(V, tc::BM);
+  const int tiles = pl.row_tiles * pl.tok_tiles;
+  const tc::SkGeom g = tc::sk_geometry(tiles, ceil_div(K, tc::BK));
+  pl.stream_k = 1;
+  pl.sk_grid = g.grid;
+  pl.sk_slots = g.max_slots;
+  pl.splits = 1;
+  pl.partial_floats = g.max_slots > 1 ? static_cast<size_t>(tiles) * g.max_slots * pl.bn * tc::BM
+                                      : 0;
+  pl.counters = g.max_slots > 1 ? tiles : 0;
+  return pl;
+}
+
 cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X, int64_t M,
                                  int K, unsigned long long* keys, uint32_t* status,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, float* partial, uint32_t* counters) {
   if (M <= 0) return cudaSuccess;
   if (dtype == DFLASH_BF16 && M >= tc::kTokMajorMin) {
     tc::Params p{};
@@ -1150,6 +1591,25 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X,
     p.status = status;
     dim3 grid(ceil_div(V, BW), ceil_div(M, tc::BM), 1);
     return tc::dispatch_tok<true>(BW, p, grid, st);
+  }
+  if (dtype == DFLASH_BF16 && partial != nullptr) {
+    tc::Params p{};
+    if (!encode_tmap_bf16_2d(&p.tm[0], W, K, V, tc::BK, tc::BM)) return cudaErrorInvalidValue;
+    const int bn = tc::pick_bn(M);
+    if (!encode_tmap_bf16_2d(&p.tm_x, X, K, M, tc::BK, bn)) return cudaErrorInvalidValue;
+    p.seg[0].rows = V;
+    p.nseg = 1;
+    p.M = static_cast<int>(M);
+    p.kb_total = ceil_div(K, tc::BK);
+    p.kb_per_split = p.kb_total;
+    p.splits = 1;
+    p.row_tiles = ceil_div(V, tc::BM);
+    p.partial = partial;
+    p.counters = counters;
+    p.keys = keys;
+    p.status = status;
+    const tc::SkGeom geo = tc::sk_geometry(p.row_tiles * ceil_div(M, bn), p.kb_total);
+    return tc::dispatch_sk<true>(bn, p, geo, st);
   }
   if (dtype == DFLASH_BF16) {
     tc::Params p{};

@@ -58,6 +58,9 @@ struct GemmJob {
 
 struct GemmPlan {
   int tok_major;     // 1: tokens on the MMA's M (large M), features per tile = bn
+  int stream_k;      // 1: persistent stream-K weight-major kernel (small M)
+  int sk_grid;       // its CTAs
+  int sk_slots;      // partial slots reserved per tile
   int bn;            // token tile (weight-major) or feature tile (token-major)
   int row_tiles;     // tiles along the output features (all segments)
   int tok_tiles;
@@ -75,11 +78,15 @@ cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& plan, float* partial
                         uint32_t* counters, uint32_t* status, cudaStream_t st);
 
 // LM head: keys[m] = max over v of argmax_key(x[m] . W[v], v).  keys must be
-// zero on entry (launch_argmax_finish leaves them zero).
+// zero on entry (launch_argmax_finish leaves them zero).  With `partial`
+// (plan_lmhead().partial_floats floats) and `counters` (zero, left zero) the
+// small-M path runs the stream-K kernel; without them, one CTA per tile.
+GemmPlan plan_lmhead(int dtype, int V, int64_t M, int K);
 cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V,
                                  const void* X, int64_t M, int K,
                                  unsigned long long* keys, uint32_t* status,
-                                 cudaStream_t st);
+                                 cudaStream_t st, float* partial = nullptr,
+                                 uint32_t* counters = nullptr);
 
 // ---------------------------------------------------------------- others
 cudaError_t launch_fuse(int dtype, const void* states, int64_t N, int T, int H,
