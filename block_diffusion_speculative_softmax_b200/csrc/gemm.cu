@@ -785,46 +785,60 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer over this CTA's units
-      auto load_w = [&](int i, uint8_t* sa) {
-        const int64_t u = u0 + i;
-        int sg, row0, tok0;
-        tile_info(static_cast<int>(u / kbt), sg, row0, tok0);
-        const int kc = static_cast<int>(u % kbt) * BK;
-        const Seg& S = p.seg[sg];
-        if (S.pair) {
-          tma_load_2d(sa, &p.tm[S.map], &full_bar[i % STAGES], kc, row0);
-          tma_load_2d(sa + A_BYTES / 2, &p.tm[S.map + 1], &full_bar[i % STAGES], kc, row0);
-        } else {
-          tma_load_2d(sa, &p.tm[S.map], &full_bar[i % STAGES], kc, row0);
+      // walk the units with running (tile, k) counters: no divisions per unit
+      struct Cursor {
+        int tile, k, sg, row0, tok0;
+      };
+      auto at_tile = [&](Cursor& c) { tile_info(c.tile, c.sg, c.row0, c.tok0); };
+      auto step = [&](Cursor& c) {
+        if (++c.k == kbt) {
+          c.k = 0;
+          ++c.tile;
+          at_tile(c);
         }
       };
-      auto load_x = [&](int i, uint8_t* sa) {
-        const int64_t u = u0 + i;
-        int sg, row0, tok0;
-        tile_info(static_cast<int>(u / kbt), sg, row0, tok0);
-        tma_load_2d(sa + A_BYTES, &p.tm_x, &full_bar[i % STAGES], static_cast<int>(u % kbt) * BK,
-                    tok0);
+      auto load_w = [&](const Cursor& c, int s, uint8_t* sa) {
+        const Seg& S = p.seg[c.sg];
+        const int kc = c.k * BK;
+        tma_load_2d(sa, &p.tm[S.map], &full_bar[s], kc, c.row0);
+        if (S.pair) tma_load_2d(sa + A_BYTES / 2, &p.tm[S.map + 1], &full_bar[s], kc, c.row0);
       };
+      auto load_x = [&](const Cursor& c, int s, uint8_t* sa) {
+        tma_load_2d(sa + A_BYTES, &p.tm_x, &full_bar[s], c.k * BK, c.tok0);
+      };
+      Cursor cw{static_cast<int>(u0 / kbt), static_cast<int>(u0 % kbt), 0, 0, 0};
+      at_tile(cw);
+      Cursor cx = cw;
       const int npre = min(STAGES, n_units);
       for (int i = 0; i < npre; ++i) {
         mbar_arrive_expect_tx(&full_bar[i], STAGE);
-        load_w(i, smem + i * STAGE);
+        load_w(cw, i, smem + i * STAGE);
+        step(cw);
       }
       pdl_wait();
-      for (int i = 0; i < npre; ++i) load_x(i, smem + i * STAGE);
+      for (int i = 0; i < npre; ++i) {
+        load_x(cx, i, smem + i * STAGE);
+        step(cx);
+      }
       int issued = npre;
+      int s = npre % STAGES;
+      uint32_t ph = (npre / STAGES) & 1;
       for (int i = npre; i < n_units; ++i) {
-        const int s = i % STAGES;
-        if (!mbar_wait(&empty_bar[s], ((i / STAGES) & 1) ^ 1, p.status, 41)) {
+        if (!mbar_wait(&empty_bar[s], ph ^ 1, p.status, 41)) {
           abort_flag = 1;
           break;
         }
         if (abort_flag) break;
         uint8_t* sa = smem + s * STAGE;
         mbar_arrive_expect_tx(&full_bar[s], STAGE);
-        load_w(i, sa);
-        load_x(i, sa);
+        load_w(cw, s, sa);
+        load_x(cw, s, sa);
+        step(cw);
         ++issued;
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1;
+        }
       }
       if (abort_flag) {
         for (int i = max(0, issued - STAGES); i < issued; ++i)
@@ -835,9 +849,11 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
     if (lane == 0) {
       // ---------------- MMA issuer; one accumulator buffer per tile segment
       int seg_i = 0;
-      for (int i = 0; i < n_units; ++i) {
-        const int64_t u = u0 + i;
-        const int k = static_cast<int>(u % kbt);
+      int k = static_cast<int>(u0 % kbt);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < n_units; ++i, ++k) {
+        if (k == kbt) k = 0;
         const bool first = (i == 0) || (k == 0);
         const bool last = (i == n_units - 1) || (k == kbt - 1);
         const int b = seg_i & 1;
@@ -846,8 +862,7 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
             abort_flag = 1;
           }
         }
-        const int s = i % STAGES;
-        if (!abort_flag && !mbar_wait(&full_bar[s], (i / STAGES) & 1, p.status, 44)) abort_flag = 1;
+        if (!abort_flag && !mbar_wait(&full_bar[s], ph, p.status, 44)) abort_flag = 1;
         if (!abort_flag) {
           tc_fence_after();
           const uint8_t* sa = smem + s * STAGE;
@@ -858,6 +873,10 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
             tc_mma_bf16(tmem + b * ACC_COLS, da + 2 * kk, db + 2 * kk, IDESC,
                         (first && kk == 0) ? 0u : 1u);
           tc_commit(&empty_bar[s]);
+        }
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1;
         }
         if (last) {
           tc_commit(&accf_bar[b]);   // arrives even after an abort, so nobody hangs
@@ -1142,8 +1161,9 @@ cudaError_t dispatch_tok(int bw, const Params& p, dim3 grid, cudaStream_t st) {
   }
 }
 
-// Tokens at or above which the token-major kernel is used.
-constexpr int64_t kTokMajorMin = 128;
+// Tokens at or above which the token-major kernel is used (the stream-K
+// weight-major kernel covers up to 64).
+constexpr int64_t kTokMajorMin = 65;
 
 inline int pick_bn(int64_t M) {
   if (M <= 16) return 16;
