@@ -144,7 +144,7 @@ GemmJob job_swiglu(const dflash_config* c, const void* wg, const void* wu, const
 struct Layout {
   size_t h = 0, x = 0, q = 0, kb = 0, vb = 0, attn = 0, act = 0, fused = 0, partial = 0,
          attn_ws = 0, zero = 0, keys = 0, counters = 0, blk_pos = 0, new_pos = 0, new_dst = 0,
-         rope = 0, total = 0;
+         rope = 0, partial_side = 0, counters_side = 0, total = 0;
   int rope_len = 0;
   size_t zero_bytes = 0;   // [keys | counters], zeroed at the start of a step
 };
@@ -201,9 +201,14 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
   L.partial = take(nd.partial_floats * 4);
   L.attn_ws = take(attn_ws_bytes(ap, nb, c->block, c->n_q_heads, c->head_dim));
   const size_t ncount = nd.counters;
+  // the context branch runs on a second stream: its own split-K scratch
+  Needs side;
+  if (n_new > 0) side.take(plan_gemm(job_kv(c, nullptr, n_new, nullptr, nullptr, 0, 0, 0, 0)));
+  L.partial_side = take(side.partial_floats * 4);
   L.zero = off;
   L.keys = take(M * 8);
   L.counters = take(ncount * 4);
+  L.counters_side = take(side.counters * 4);
   L.zero_bytes = off - L.zero;
   L.blk_pos = take(M * 4);
   L.new_pos = take(n_new * 4);
@@ -226,6 +231,35 @@ dflash_status check_ws(void* ws, size_t ws_bytes, size_t need) {
             "workspace must be 256-byte aligned");
   DFL_CHECK(ws_bytes >= need, DFLASH_EINVAL, "workspace too small: %zu bytes, need %zu",
             ws_bytes, need);
+  return DFLASH_OK;
+}
+
+// A second stream (per host thread and device) for the context branch of a
+// draft step: fusion and the context K/V projections of every layer depend
+// only on the new context rows, not on the block path, so they run beside
+// the weight-streaming block GEMMs; layer i's attention waits for its
+// context K/V through an event.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t done[kMaxLayers] = {};
+};
+constexpr int kSideDevices = 16;
+thread_local SideStream t_side[kSideDevices];
+
+dflash_status side_stream(SideStream** out) {
+  *out = nullptr;
+  int dev = 0;
+  DFL_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kSideDevices) return DFLASH_OK;   // run the branch in order instead
+  SideStream& r = t_side[dev];
+  if (r.stream == nullptr) {
+    DFL_CUDA(cudaStreamCreateWithFlags(&r.stream, cudaStreamNonBlocking), "side stream");
+    DFL_CUDA(cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming), "side event");
+    for (int i = 0; i < kMaxLayers; ++i)
+      DFL_CUDA(cudaEventCreateWithFlags(&r.done[i], cudaEventDisableTiming), "side event");
+  }
+  *out = &r;
   return DFLASH_OK;
 }
 
@@ -539,12 +573,34 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
            "row bookkeeping");
   float2* rope_tab = at<float2>(ws, L.rope);
   DFL_CUDA(launch_rope_table(rope_tab, L.rope_len, c->head_dim, c->rope_theta, st), "RoPE table");
+  // context branch: fusion + every layer's context K/V projection
+  SideStream* side = nullptr;
   if (a->n_ctx_new > 0) {
+    if ((s = side_stream(&side)) != DFLASH_OK) return s;
+    cudaStream_t cs = st;
+    if (side) {
+      DFL_CUDA(cudaEventRecord(side->fork, st), "fork");
+      DFL_CUDA(cudaStreamWaitEvent(side->stream, side->fork, 0), "fork");
+      cs = side->stream;
+    }
     const float* gf[kMaxLayers];
     for (int i = 0; i < D; ++i) gf[i] = w->layers[i].g_fuse;
     DFL_CUDA(launch_fuse(dt, a->new_states, a->n_ctx_new, c->n_target_layers, H, D, w->w_fuse,
-                         gf, fused, c->rms_eps, status, st),
+                         gf, fused, c->rms_eps, status, cs),
              "fusion kernel");
+    for (int i = 0; i < D; ++i) {
+      const dflash_layer_weights& l = w->layers[i];
+      GemmJob jc = job_kv(c, fused + static_cast<size_t>(i) * a->n_ctx_new * H * e,
+                          a->n_ctx_new, new_pos, new_dst, l.w_kt, l.w_vt, a->k_cache[i],
+                          a->v_cache[i]);
+      jc.rope_tab = rope_tab;
+      jc.rope_len = L.rope_len;
+      s = run_job(jc, side ? at<float>(ws, L.partial_side) : partial,
+                  side ? at<uint32_t>(ws, L.counters_side) : counters, status, cs,
+                  "context K/V GEMM");
+      if (s != DFLASH_OK) return s;
+      if (side) DFL_CUDA(cudaEventRecord(side->done[i], side->stream), "context done");
+    }
   }
   DFL_CUDA(launch_embed(dt, w->embed, H, a->n_blocks, c->block, a->block_tokens, a->known_len,
                         c->mask_token_id, h, st),
@@ -553,22 +609,13 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
                                 c->head_dim, a->max_ctx_len);
   for (int i = 0; i < D; ++i) {
     const dflash_layer_weights& l = w->layers[i];
-    // context K/V of the new rows through W^t, into the caches
-    if (a->n_ctx_new > 0) {
-      GemmJob jc = job_kv(c, fused + static_cast<size_t>(i) * a->n_ctx_new * H * e,
-                          a->n_ctx_new, new_pos, new_dst, l.w_kt, l.w_vt, a->k_cache[i],
-                          a->v_cache[i]);
-      jc.rope_tab = rope_tab;
-      jc.rope_len = L.rope_len;
-      s = run_job(jc, partial, counters, status, st, "context K/V GEMM");
-      if (s != DFLASH_OK) return s;
-    }
     // block: RMSNorm -> Q (RoPE), K^d (RoPE), V^d
     DFL_CUDA(launch_rmsnorm(dt, h, M, H, l.g_attn, c->rms_eps, x, st), "attention rmsnorm");
     GemmJob jq = job_qkv(c, l, x, M, blk_pos, q, kb, vb);
     jq.rope_tab = rope_tab;
     jq.rope_len = L.rope_len;
     if ((s = run_job(jq, partial, counters, status, st, "QKV GEMM")) != DFLASH_OK) return s;
+    if (side) DFL_CUDA(cudaStreamWaitEvent(st, side->done[i], 0), "join context");
     DFL_CUDA(launch_attn(dt, ap, a->n_blocks, c->block, c->n_q_heads, c->n_kv_heads,
                          c->head_dim, q, kb, vb, a->k_cache[i], a->v_cache[i], a->ctx_off,
                          a->block_req, attn, at<float>(ws, L.attn_ws), status, st),

@@ -34,6 +34,7 @@
 // models run on a SIMT FFMA kernel (partials + finish kernel): tensor-core
 // tf32 would miss a 1e-4 tolerance.
 #include <algorithm>
+#include <cstdlib>
 #include <cmath>
 #include <mutex>
 
@@ -297,24 +298,40 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
       do_op = s_last != 0;
       if (do_op) {
         __threadfence();
-        // fixed split order; 16 independent loads in flight per thread
-        const float* base = p.partial + static_cast<size_t>(tile_lin) * p.splits * BN * BM + tid;
-        constexpr int JC = BN < 16 ? BN : 16;
+        // the tile's BN x 128 floats as float4 items (token j, rows 4q..4q+3),
+        // each summed over the splits in fixed order, straight into staging;
+        // every thread keeps 4 items x 2 splits of loads in flight
+        const float4* base = reinterpret_cast<const float4*>(
+            p.partial + static_cast<size_t>(tile_lin) * p.splits * BN * BM);
+        constexpr int ITEMS = BN * (BM / 4);
+        constexpr int NT = 128;
 #pragma unroll 1
-        for (int j0 = 0; j0 < BN; j0 += JC) {
-          float acc[JC];
+        for (int it0 = 0; it0 < ITEMS; it0 += 4 * NT) {
+          float4 acc[4];
 #pragma unroll
-          for (int q = 0; q < JC; ++q) acc[q] = 0.f;
-#pragma unroll 1
-          for (int s = 0; s < p.splits; ++s) {
-            float v[JC];
+          for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+          for (int sp = 0; sp < p.splits; ++sp) {
+            float4 a[4];
 #pragma unroll
-            for (int q = 0; q < JC; ++q) v[q] = __ldcg(base + (s * BN + j0 + q) * BM);
+            for (int q = 0; q < 4; ++q) {
+              const int it = it0 + q * NT + tid;
+              a[q] = it < ITEMS ? __ldcg(base + static_cast<size_t>(sp) * ITEMS + it)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
-            for (int q = 0; q < JC; ++q) acc[q] += v[q];
+            for (int q = 0; q < 4; ++q) {
+              acc[q].x += a[q].x; acc[q].y += a[q].y; acc[q].z += a[q].z; acc[q].w += a[q].w;
+            }
           }
 #pragma unroll
-          for (int q = 0; q < JC; ++q) st[(j0 + q) * SROW + tid] = acc[q];
+          for (int q = 0; q < 4; ++q) {
+            const int it = it0 + q * NT + tid;
+            if (it < ITEMS) {
+              const int j = it / (BM / 4), rq = (it % (BM / 4)) * 4;
+              *reinterpret_cast<float4*>(st + j * SROW + rq) = acc[q];
+            }
+          }
         }
         if (tid == 0) p.counters[tile_lin] = 0u;
       }
@@ -1110,23 +1127,24 @@ cudaError_t launch_sk(const Params& p, const SkGeom& geo, cudaStream_t st) {
                   geo);
 }
 
-// One CTA per SM with a ring of ~180 KB.
+// Two CTAs per SM, each with a ~90 KB ring: two independent TMA streams per
+// SM measured faster than one persistent CTA with twice the ring.
 template <bool ARGMAX>
 cudaError_t dispatch_sk(int bn, const Params& p, const SkGeom& geo, cudaStream_t st) {
   switch (bn) {
-    case 16: return launch_sk<16, 10, ARGMAX>(p, geo, st);
-    case 32: return launch_sk<32, 9, ARGMAX>(p, geo, st);
-    case 64: return launch_sk<64, 7, ARGMAX>(p, geo, st);
+    case 16: return launch_sk<16, 5, ARGMAX>(p, geo, st);
+    case 32: return launch_sk<32, 4, ARGMAX>(p, geo, st);
+    case 64: return launch_sk<64, 3, ARGMAX>(p, geo, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-// Stream-K partition of `tiles` x `kbt` units over at most one CTA per SM:
+// Stream-K partition of `tiles` x `kbt` units over at most two CTAs per SM:
 // the grid and the largest number of CTAs sharing one tile.
 inline SkGeom sk_geometry(int tiles, int kbt) {
   SkGeom g{};
   g.units = static_cast<int64_t>(tiles) * kbt;
-  g.grid = static_cast<int>(std::min<int64_t>(g.units, kNumSMs));
+  g.grid = static_cast<int>(std::min<int64_t>(g.units, kNumSMs * 2));
   g.max_slots = 1;
   auto u0 = [&](int64_t c) { return (c * g.units) / g.grid; };
   auto cta_of = [&](int64_t u) { return static_cast<int>(((u + 1) * g.grid - 1) / g.units); };
@@ -1417,22 +1435,16 @@ GemmPlan plan_gemm(const GemmJob& job) {
       const int tiles = pl.row_tiles * pl.tok_tiles;
       if (tiles * 2 < kNumSMs) splits = std::min(kb_total, kNumSMs / tiles);
     } else {
-      // weight-major (swap-AB), stream-K: 128 weight rows x BN tokens per
-      // tile, the (tile, k-block) units split evenly over one CTA per SM
+      // weight-major (swap-AB): 128 weight rows x BN tokens per tile, split K
+      // so about two CTAs per SM stream at once and all fit in one wave
       pl.bn = tc::pick_bn(M);
       pl.tok_tiles = ceil_div(M, pl.bn);
       pl.row_tiles = feature_tiles(tc::BM);
+      // (the stream-K kernel measured slower here than whole-tile CTAs: its
+      // extra shared-tile reductions cost more than the wave balance gains)
       const int tiles = pl.row_tiles * pl.tok_tiles;
-      const tc::SkGeom g = tc::sk_geometry(tiles, kb_total);
-      pl.stream_k = 1;
-      pl.sk_grid = g.grid;
-      pl.sk_slots = g.max_slots;
-      pl.splits = 1;
-      pl.kb_per_split = kb_total;
-      pl.partial_floats =
-          g.max_slots > 1 ? static_cast<size_t>(tiles) * g.max_slots * pl.bn * tc::BM : 0;
-      pl.counters = g.max_slots > 1 ? tiles : 0;
-      return pl;
+      const int slots = kNumSMs * tc::ctas_per_sm(pl.bn);
+      if (tiles < slots) splits = std::max(1, std::min(kb_total, slots / tiles));
     }
     splits = std::max(1, std::min(splits, 32));
     pl.kb_per_split = ceil_div(kb_total, splits);
