@@ -438,9 +438,10 @@ AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d, int64_t max
     p.chunk = 64;
     return p;
   }
-  // at least 256 context keys per split: the fp32 partials of a split then
-  // stay well below the K/V bytes it streams
-  const int64_t max_splits = std::min<int64_t>(64, (max_ctx_len + 255) / 256);
+  // at least 256 context keys per split: the fp32 partials of a split
+  // then stay below the K/V bytes it streams
+  const int64_t min_chunk = 256;
+  const int64_t max_splits = std::min<int64_t>(64, (max_ctx_len + min_chunk - 1) / min_chunk);
   int64_t want = (2 * kNumSMs + base - 1) / base;
   int64_t splits = std::max<int64_t>(1, std::min(want, max_splits));
   int64_t chunk = (max_ctx_len + splits - 1) / splits;

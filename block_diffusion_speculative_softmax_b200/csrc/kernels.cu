@@ -142,9 +142,15 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
 #pragma unroll
       for (int i = 0; i < MAXD; ++i) {
         if (i < D) {
-          float tot = 0.f;
-          for (int w = 0; w < nwarps; ++w) tot += red[par][w][i];
-          const float sc = rsqrtf(tot / static_cast<float>(H) + eps);
+          // all per-warp partials loaded first, then a short add tree
+          float part[32];
+#pragma unroll
+          for (int w = 0; w < 32; ++w) part[w] = w < nwarps ? red[par][w][i] : 0.f;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int w = 0; w < o; ++w) part[w] += part[w + o];
+          const float sc = rsqrtf(part[0] / static_cast<float>(H) + eps);
           const float* g = gains.g[i] + col;
           float o[VE];
 #pragma unroll
