@@ -42,7 +42,7 @@ import numpy as np
 __all__ = [
     "bf16", "softmax", "rmsnorm", "fuse_ctx", "rope", "kv_project",
     "block_attn", "swiglu_mlp", "lmhead_logits", "lmhead_argmax", "accept",
-    "d2sd_candidates", "draft_request", "draft_step", "Block",
+    "d2sd_candidates", "draft_request", "draft_step", "Block", "draft_confidence",
 ]
 
 
@@ -195,6 +195,19 @@ def lmhead_argmax(x: np.ndarray, w_lm: np.ndarray
     z = lmhead_logits(x, w_lm)
     tok = np.argmax(z, axis=1).astype(np.int32)   # first occurrence = lowest id
     return tok, z.max(axis=1), z
+
+
+def draft_confidence(z: np.ndarray) -> np.ndarray:
+    """Per-slot confidence of the draft's own prediction: the softmax
+    probability of its argmax token, 1 / sum_v exp(z_v - max z).
+
+    D2SD summary, methodology step 1: the first drafter reports, for every
+    position, a confidence that its token will be accepted.  The pages do not
+    say how it is computed; the draft's top-1 probability is the plainest
+    reading (it needs no extra head)."""
+    z = _f64(z)
+    m = z.max(axis=-1, keepdims=True)
+    return 1.0 / np.exp(z - m).sum(axis=-1)
 
 
 # ---------------------------------------------------------------------------

@@ -458,3 +458,19 @@ def test_speculative_loop_with_oracle_draft_is_lossless():
     got, steps = speculative_decode(tw, cfg, dw, prompt, n_new, draft_fn, accept_fn, rng)
     np.testing.assert_array_equal(got, greedy)
     assert steps < n_new          # some steps accepted more than one token
+
+
+# ---------------------------------------------------------------- draft confidence
+
+def test_draft_confidence_is_top1_softmax_probability():
+    rng = np.random.default_rng(15)
+    z = rng.standard_normal((6, 40)) * 3
+    want = scipy.special.softmax(z, axis=1).max(axis=1)
+    np.testing.assert_allclose(O.draft_confidence(z), want, rtol=1e-13)
+    # closed forms: a uniform row gives 1/V, a dominant logit gives ~1
+    assert abs(O.draft_confidence(np.zeros((1, 40)))[0] - 1 / 40) < 1e-15
+    big = np.zeros((1, 40))
+    big[0, 7] = 800.0
+    assert abs(O.draft_confidence(big)[0] - 1.0) < 1e-15
+    # invariant to a constant shift of all logits
+    np.testing.assert_allclose(O.draft_confidence(z + 123.0), O.draft_confidence(z), rtol=1e-12)
