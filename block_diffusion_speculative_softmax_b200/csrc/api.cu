@@ -1,6 +1,7 @@
 // C ABI of libdflash.so: argument validation, workspace layout and the
 // kernel sequence of one draft step.  No entry point allocates memory.
 #include <atomic>
+#include <cstdlib>
 #include <mutex>
 #include <cmath>
 #include <cstdarg>
@@ -144,7 +145,7 @@ GemmJob job_swiglu(const dflash_config* c, const void* wg, const void* wu, const
 struct Layout {
   size_t h = 0, x = 0, q = 0, kb = 0, vb = 0, attn = 0, act = 0, fused = 0, partial = 0,
          attn_ws = 0, zero = 0, keys = 0, counters = 0, blk_pos = 0, new_pos = 0, new_dst = 0,
-         rope = 0, partial_side = 0, counters_side = 0, total = 0;
+         rope = 0, partial_side = 0, counters_side = 0, lse = 0, total = 0;
   int rope_len = 0;
   size_t zero_bytes = 0;   // [keys | counters], zeroed at the start of a step
 };
@@ -213,6 +214,7 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
   L.blk_pos = take(M * 4);
   L.new_pos = take(n_new * 4);
   L.new_dst = take(n_new * 8);
+  L.lse = take(static_cast<size_t>(lmhead_tiles(c->dtype, c->vocab, M)) * M * 8);
   L.rope_len = static_cast<int>(max_ctx + c->block);
   L.rope = take(static_cast<size_t>(L.rope_len) * (c->head_dim / 2) * 8);
   L.total = off;
@@ -429,8 +431,8 @@ dflash_status dflash_mlp(const dflash_config* cfg, int64_t M, float* h, const fl
 }
 
 dflash_status dflash_lmhead_argmax(const dflash_config* cfg, int64_t M, const void* x,
-                                   const void* w_lm, int32_t* tok, float* max_logit, void* ws,
-                                   size_t ws_bytes, void* stream) {
+                                   const void* w_lm, int32_t* tok, float* max_logit, float* conf,
+                                   void* ws, size_t ws_bytes, void* stream) {
   dflash_status s = check_config(cfg);
   if (s != DFLASH_OK) return s;
   DFL_CHECK(M >= 0 && M < (int64_t(1) << 31), DFLASH_EINVAL, "M out of range");
@@ -442,7 +444,11 @@ dflash_status dflash_lmhead_argmax(const dflash_config* cfg, int64_t M, const vo
   const size_t off_keys = sizeof(DevStatus);
   const size_t off_cnt = align256(off_keys + M * 8);
   const size_t off_part = align256(off_cnt + pl.counters * 4);
-  if ((s = check_ws(ws, ws_bytes, off_part + pl.partial_floats * 4)) != DFLASH_OK) return s;
+  const int lt = lmhead_tiles(cfg->dtype, cfg->vocab, M);
+  const size_t off_lse = align256(off_part + pl.partial_floats * 4);
+  const size_t need = off_lse + (conf ? static_cast<size_t>(lt) * M * 8 : 0);
+  if ((s = check_ws(ws, ws_bytes, need)) != DFLASH_OK) return s;
+  float2* lse = conf ? at<float2>(ws, off_lse) : nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto* keys = at<unsigned long long>(ws, off_keys);
   // keys and tile counters start at zero
@@ -450,9 +456,10 @@ dflash_status dflash_lmhead_argmax(const dflash_config* cfg, int64_t M, const vo
   DFL_CUDA(launch_lmhead_argmax(cfg->dtype, w_lm, cfg->vocab, x, M, cfg->hidden, keys,
                                 status_word(ws), st,
                                 pl.stream_k ? at<float>(ws, off_part) : nullptr,
-                                pl.stream_k ? at<uint32_t>(ws, off_cnt) : nullptr),
+                                pl.stream_k ? at<uint32_t>(ws, off_cnt) : nullptr, lse),
            "LM head argmax");
-  DFL_CUDA(launch_argmax_finish(keys, M, cfg->block, nullptr, nullptr, tok, max_logit, st),
+  DFL_CUDA(launch_argmax_finish(keys, M, cfg->block, nullptr, nullptr, tok, max_logit, st, lse,
+                                lt, conf),
            "argmax finish");
   return DFLASH_OK;
 }
@@ -632,11 +639,13 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
       return s;
   }
   DFL_CUDA(launch_rmsnorm(dt, h, M, H, w->g_final, c->rms_eps, x, st), "final rmsnorm");
+  float2* lse = a->confidence ? at<float2>(ws, L.lse) : nullptr;
   DFL_CUDA(launch_lmhead_argmax(dt, w->lm_head, c->vocab, x, M, H, keys, status, st, partial,
-                                counters),
+                                counters, lse),
            "LM head argmax");
   DFL_CUDA(launch_argmax_finish(keys, M, c->block, a->block_tokens, a->known_len,
-                                a->draft_tokens, a->max_logit, st),
+                                a->draft_tokens, a->max_logit, st, lse,
+                                lmhead_tiles(dt, c->vocab, M), a->confidence),
            "argmax finish");
   if (a->target_tokens) {
     DFL_CUDA(launch_accept(a->n_req, a->n_cand, c->block, a->draft_tokens, a->target_tokens,

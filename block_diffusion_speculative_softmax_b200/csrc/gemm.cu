@@ -89,6 +89,7 @@ struct Params {
   int rope_len;
   double inv_freq[64];
   unsigned long long* keys;         // argmax mode: [M]
+  float2* lse;                      // argmax mode: per (vocab tile, token) (max, sum exp)
   uint32_t* status;
 };
 
@@ -123,6 +124,7 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
   __shared__ volatile int abort_flag;
   __shared__ int s_last;
   __shared__ unsigned long long red[ARGMAX ? 4 : 1][ARGMAX ? BN : 1];
+  __shared__ float2 red2[ARGMAX ? 4 : 1][ARGMAX ? BN : 1];
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -249,6 +251,13 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
           }
           key = warp_max_u64(key);
           if (lane == 0) red[warp][c + j] = key;
+          if (p.lse != nullptr) {
+            // this tile's share of the log-sum-exp of token c + j
+            const bool in = row < S.rows;
+            const float mx = warp_max(in ? v[j] : -INFINITY);
+            const float se = warp_sum(in ? __expf(v[j] - mx) : 0.f);
+            if (lane == 0) red2[warp][c + j] = make_float2(mx, se);
+          }
         }
       }
     }
@@ -260,6 +269,16 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
         for (int w = 1; w < 4; ++w) k = red[w][j] > k ? red[w][j] : k;
         const int t = tok0 + j;
         if (t < p.M && k != 0ull) atomicMax(p.keys + t, k);
+        if (t < p.M && p.lse != nullptr) {
+          float mx = red2[0][j].x;
+#pragma unroll
+          for (int w = 1; w < 4; ++w) mx = fmaxf(mx, red2[w][j].x);
+          float se = 0.f;
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            se += red2[w][j].y > 0.f ? red2[w][j].y * __expf(red2[w][j].x - mx) : 0.f;
+          p.lse[static_cast<size_t>(blockIdx.x) * p.M + t] = make_float2(mx, se);
+        }
       }
     }
   } else {
@@ -592,6 +611,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
   if (do_op) {
     if constexpr (ARGMAX) {
       unsigned long long best = 0ull;
+      float mx = -INFINITY, se = 0.f;   // running log-sum-exp share of this tile
 #pragma unroll 1
       for (int c = 0; c < BW; c += 16) {
         float v[16];
@@ -603,10 +623,17 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
             if (!isfinite(v[q]) && tv) report(p.status, DFLASH_ENUMERIC, 35);
             const unsigned long long k = argmax_key(v[q], static_cast<uint32_t>(f));
             best = k > best ? k : best;
+            if (v[q] > mx) {
+              se = se * __expf(mx - v[q]) + 1.f;
+              mx = v[q];
+            } else {
+              se += __expf(v[q] - mx);
+            }
           }
         }
       }
       if (tv && best) atomicMax(p.keys + t, best);
+      if (tv && p.lse != nullptr) p.lse[static_cast<size_t>(blockIdx.x) * p.M + t] = make_float2(mx, se);
     } else if (S.op == EPI_SWIGLU) {
       __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out) + static_cast<int64_t>(t) * S.out_stride;
 #pragma unroll 1
@@ -758,6 +785,7 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
   __shared__ volatile int abort_flag;
   __shared__ int s_last;
   __shared__ unsigned long long red[ARGMAX ? 4 : 1][ARGMAX ? BN : 1];
+  __shared__ float2 red2[ARGMAX ? 4 : 1][ARGMAX ? BN : 1];
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -1009,6 +1037,13 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
             }
             key = warp_max_u64(key);
             if (lane == 0) red[quarter][j] = key;
+            if (p.lse != nullptr) {
+              // this tile's share of the log-sum-exp of token j
+              const bool in = row < S.rows;
+              const float mx = warp_max(in ? v[j] : -INFINITY);
+              const float se = warp_sum(in ? __expf(v[j] - mx) : 0.f);
+              if (lane == 0) red2[quarter][j] = make_float2(mx, se);
+            }
           }
           named_sync(1, EPI);
           for (int j = et; j < BN; j += EPI) {
@@ -1016,6 +1051,17 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
 #pragma unroll
             for (int w = 1; w < 4; ++w) k = red[w][j] > k ? red[w][j] : k;
             if (tok0 + j < p.M && k != 0ull) atomicMax(p.keys + tok0 + j, k);
+            if (p.lse != nullptr && tok0 + j < p.M) {
+              float mx = red2[0][j].x;
+#pragma unroll
+              for (int w = 1; w < 4; ++w) mx = fmaxf(mx, red2[w][j].x);
+              float se = 0.f;
+#pragma unroll
+              for (int w = 0; w < 4; ++w)
+                se += red2[w][j].y > 0.f ? red2[w][j].y * __expf(red2[w][j].x - mx) : 0.f;
+              const int rt = tile % p.row_tiles;
+              p.lse[static_cast<size_t>(rt) * p.M + tok0 + j] = make_float2(mx, se);
+            }
           }
         } else if (S.op == EPI_SWIGLU) {
           const int rr = et & 63;
@@ -1214,6 +1260,7 @@ struct Params {
   int n_cols;
   float* partial;
   unsigned long long* keys;
+  float2* lse;
   uint32_t* status;
 };
 
@@ -1222,6 +1269,7 @@ __global__ void __launch_bounds__(256) gemm_kernel(const __grid_constant__ Param
   __shared__ float ws[TK][TR + 1];
   __shared__ float xs[TK][TT + 1];
   __shared__ unsigned long long red[16][TT];
+  __shared__ float2 red2[16][TT];
   const int tile = blockIdx.x;
   int seg = 0;
   while (seg + 1 < p.nseg && tile >= p.seg_tile_begin[seg + 1]) ++seg;
@@ -1277,6 +1325,7 @@ __global__ void __launch_bounds__(256) gemm_kernel(const __grid_constant__ Param
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       unsigned long long best = 0ull;
+      float mx = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = row0 + ty + 16 * i, t = tok0 + tx + 16 * j;
@@ -1284,15 +1333,32 @@ __global__ void __launch_bounds__(256) gemm_kernel(const __grid_constant__ Param
           if (!isfinite(acc[i][j])) report(p.status, DFLASH_ENUMERIC, 16);
           const unsigned long long k = argmax_key(acc[i][j], static_cast<uint32_t>(r));
           best = k > best ? k : best;
+          mx = fmaxf(mx, acc[i][j]);
         }
       }
+      float se = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = row0 + ty + 16 * i, t = tok0 + tx + 16 * j;
+        if (r < rows && t < p.M) se += expf(acc[i][j] - mx);
+      }
       red[ty][tx + 16 * j] = best;
+      red2[ty][tx + 16 * j] = make_float2(mx, se);
     }
     __syncthreads();
     if (tid < TT) {
       unsigned long long best = 0ull;
-      for (int y = 0; y < 16; ++y) best = red[y][tid] > best ? red[y][tid] : best;
+      float mx = -INFINITY;
+      for (int y = 0; y < 16; ++y) {
+        best = red[y][tid] > best ? red[y][tid] : best;
+        mx = fmaxf(mx, red2[y][tid].x);
+      }
+      float se = 0.f;
+      for (int y = 0; y < 16; ++y)
+        if (red2[y][tid].y > 0.f) se += red2[y][tid].y * expf(red2[y][tid].x - mx);
       if (tok0 + tid < p.M && best) atomicMax(p.keys + tok0 + tid, best);
+      if (tok0 + tid < p.M && p.lse != nullptr)
+        p.lse[static_cast<size_t>(blockIdx.x) * p.M + tok0 + tid] = make_float2(mx, se);
     }
   }
 }
@@ -1603,9 +1669,16 @@ GemmPlan plan_lmhead(int dtype, int V, int64_t M, int K) {
   return pl;
 }
 
+int lmhead_tiles(int dtype, int V, int64_t M) {
+  if (dtype == DFLASH_BF16 && M >= tc::kTokMajorMin) return ceil_div(V, 256);
+  if (dtype == DFLASH_BF16) return ceil_div(V, tc::BM);
+  return ceil_div(V, simt::TR);
+}
+
 cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X, int64_t M,
                                  int K, unsigned long long* keys, uint32_t* status,
-                                 cudaStream_t st, float* partial, uint32_t* counters) {
+                                 cudaStream_t st, float* partial, uint32_t* counters,
+                                 float2* lse) {
   if (M <= 0) return cudaSuccess;
   if (dtype == DFLASH_BF16 && M >= tc::kTokMajorMin) {
     tc::Params p{};
@@ -1620,6 +1693,7 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X,
     p.splits = 1;
     p.row_tiles = ceil_div(V, BW);
     p.keys = keys;
+    p.lse = lse;
     p.status = status;
     dim3 grid(ceil_div(V, BW), ceil_div(M, tc::BM), 1);
     return tc::dispatch_tok<true>(BW, p, grid, st);
@@ -1639,6 +1713,7 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X,
     p.partial = partial;
     p.counters = counters;
     p.keys = keys;
+    p.lse = lse;
     p.status = status;
     const tc::SkGeom geo = tc::sk_geometry(p.row_tiles * ceil_div(M, bn), p.kb_total);
     return tc::dispatch_sk<true>(bn, p, geo, st);
@@ -1658,6 +1733,7 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X,
     p.splits = 1;
     p.row_tiles = ceil_div(V, tc::BM);
     p.keys = keys;
+    p.lse = lse;
     p.status = status;
     dim3 grid(ceil_div(V, tc::BM), ceil_div(M, bn), 1);
     return tc::dispatch<true>(bn, p, grid, st);
@@ -1673,6 +1749,7 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X,
   p.K = K;
   p.k_per_split = K;
   p.keys = keys;
+  p.lse = lse;
   p.status = status;
   return launch_k(simt::gemm_kernel<true>, dim3(ceil_div(V, simt::TR), ceil_div(M, simt::TT), 1),
                   dim3(256), 0, st, p);

@@ -81,12 +81,15 @@ cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& plan, float* partial
 // zero on entry (launch_argmax_finish leaves them zero).  With `partial`
 // (plan_lmhead().partial_floats floats) and `counters` (zero, left zero) the
 // small-M path runs the stream-K kernel; without them, one CTA per tile.
+// With `lse` ([lmhead_tiles()][M]) every vocabulary tile also leaves its
+// (max, sum exp) share of each token's log-sum-exp for the confidence.
 GemmPlan plan_lmhead(int dtype, int V, int64_t M, int K);
+int lmhead_tiles(int dtype, int V, int64_t M);
 cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V,
                                  const void* X, int64_t M, int K,
                                  unsigned long long* keys, uint32_t* status,
                                  cudaStream_t st, float* partial = nullptr,
-                                 uint32_t* counters = nullptr);
+                                 uint32_t* counters = nullptr, float2* lse = nullptr);
 
 // ---------------------------------------------------------------- others
 cudaError_t launch_fuse(int dtype, const void* states, int64_t N, int T, int H,
@@ -109,7 +112,9 @@ cudaError_t launch_prep_rows(int R, int nb, int B, const int32_t* block_req,
 cudaError_t launch_argmax_finish(unsigned long long* keys, int64_t M,
                                  int B, const int32_t* block_tokens,
                                  const int32_t* known_len, int32_t* tok,
-                                 float* max_logit, cudaStream_t st);
+                                 float* max_logit, cudaStream_t st,
+                                 const float2* lse = nullptr, int lse_tiles = 0,
+                                 float* conf = nullptr);
 cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t st);
 // RoPE table: tab[p][i] = (cos, sin)(p * theta^(-2i/d)), p < len, i < d/2.
 cudaError_t launch_rope_table(float2* tab, int len, int head_dim, double theta,

@@ -1,5 +1,6 @@
 // Bandwidth- and latency-bound kernels of the draft step.
 #include <algorithm>
+#include <cstdlib>
 #include <cmath>
 #include <mutex>
 
@@ -417,6 +418,28 @@ cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t st) {
 // ===========================================================================
 // argmax keys -> tokens (+ max logit); known slots keep their input token
 // ===========================================================================
+// Confidence of the draft's argmax token: p = exp(max - lse) = 1 / S with
+// S = sum over vocabulary tiles of sumexp_t * exp(max_t - max), one warp per
+// token (lanes take tiles in a fixed stride, then a fixed-order tree).
+__global__ void confidence_kernel(const float2* __restrict__ lse, int tiles, int64_t M,
+                                  float* __restrict__ conf) {
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
+  const int64_t m = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (m >= M) return;
+  float mx = -INFINITY;
+  for (int t = lane; t < tiles; t += 32) mx = fmaxf(mx, lse[static_cast<size_t>(t) * M + m].x);
+  mx = warp_max(mx);
+  float s = 0.f;
+  for (int t = lane; t < tiles; t += 32) {
+    const float2 v = lse[static_cast<size_t>(t) * M + m];
+    if (v.y > 0.f) s += v.y * __expf(v.x - mx);
+  }
+  s = warp_sum(s);
+  if (lane == 0) conf[m] = 1.f / s;
+}
+
 __global__ void argmax_finish_kernel(unsigned long long* __restrict__ keys, int64_t M,
                                      int B, const int32_t* __restrict__ block_tokens,
                                      const int32_t* __restrict__ known_len,
@@ -439,10 +462,14 @@ __global__ void argmax_finish_kernel(unsigned long long* __restrict__ keys, int6
 
 cudaError_t launch_argmax_finish(unsigned long long* keys, int64_t M, int B,
                                  const int32_t* block_tokens, const int32_t* known_len,
-                                 int32_t* tok, float* max_logit, cudaStream_t st) {
+                                 int32_t* tok, float* max_logit, cudaStream_t st,
+                                 const float2* lse, int lse_tiles, float* conf) {
   if (M <= 0) return cudaSuccess;
-  return launch_k(argmax_finish_kernel, dim3(static_cast<unsigned>((M + 255) / 256)), dim3(256),
-                  0, st, keys, M, B, block_tokens, known_len, tok, max_logit);
+  cudaError_t e = launch_k(argmax_finish_kernel, dim3(static_cast<unsigned>((M + 255) / 256)),
+                           dim3(256), 0, st, keys, M, B, block_tokens, known_len, tok, max_logit);
+  if (e != cudaSuccess || conf == nullptr || lse == nullptr) return e;
+  return launch_k(confidence_kernel, dim3(static_cast<unsigned>((M * 32 + 255) / 256)), dim3(256),
+                  0, st, lse, lse_tiles, M, conf);
 }
 
 // ===========================================================================

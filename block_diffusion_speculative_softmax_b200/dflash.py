@@ -54,7 +54,8 @@ class StepArgs(C.Structure):
                 ("new_states", C.c_void_p), ("ctx_off", C.c_void_p), ("new_off", C.c_void_p),
                 ("ctx_cached", C.c_void_p), ("k_cache", C.POINTER(C.c_void_p)),
                 ("v_cache", C.POINTER(C.c_void_p)), ("draft_tokens", C.c_void_p),
-                ("max_logit", C.c_void_p), ("target_tokens", C.c_void_p),
+                ("max_logit", C.c_void_p), ("confidence", C.c_void_p),
+                ("target_tokens", C.c_void_p),
                 ("n_cand", C.c_int32), ("n_acc", C.c_void_p), ("best_k", C.c_void_p),
                 ("out_tok", C.c_void_p)]
 
@@ -76,7 +77,7 @@ SIGNATURES = {
     "dflash_block_attn": (C.c_int, [_CFG, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _VP,
                                     _VP, _SZ, _VP]),
     "dflash_mlp": (C.c_int, [_CFG, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
-    "dflash_lmhead_argmax": (C.c_int, [_CFG, _I64, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "dflash_lmhead_argmax": (C.c_int, [_CFG, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "dflash_accept": (C.c_int, [_I32, _I32, _I32, _VP, _VP, _VP, _VP, _VP, _VP]),
     "dflash_d2sd_candidates": (C.c_int, [_I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP, _VP,
                                          _VP]),
@@ -204,9 +205,10 @@ def dflash_mlp(cfg: Config, h, g_mlp, w_gate, w_up, w_down, ws, stream=None):
                              _p(w_down), _p(ws), ws.numel(), _stream(stream)))
 
 
-def dflash_lmhead_argmax(cfg: Config, x, w_lm, tok, max_logit, ws, stream=None):
+def dflash_lmhead_argmax(cfg: Config, x, w_lm, tok, max_logit, ws, stream=None, conf=None):
     _check(load().dflash_lmhead_argmax(C.byref(cfg), x.shape[0], _p(x), _p(w_lm), _p(tok),
-                                       _p(max_logit), _p(ws), ws.numel(), _stream(stream)))
+                                       _p(max_logit), _p(conf), _p(ws), ws.numel(),
+                                       _stream(stream)))
 
 
 def dflash_lmhead_argmax_noalloc(cfg: Config, x, w_lm, tok, max_logit=None, stream=None):
@@ -310,6 +312,7 @@ class StepBuffers:
         self.known_len = torch.ones(n_blocks, dtype=torch.int32, device=device)
         self.draft_tokens = torch.zeros(n_blocks, B, dtype=torch.int32, device=device)
         self.max_logit = torch.zeros(n_blocks, B, dtype=torch.float32, device=device)
+        self.confidence = torch.zeros(n_blocks, B, dtype=torch.float32, device=device)
         self.target_tokens = torch.zeros(n_blocks, B, dtype=torch.int32, device=device)
         self.n_acc = torch.zeros(self.R, dtype=torch.int32, device=device)
         self.best_k = torch.zeros(self.R, dtype=torch.int32, device=device)
@@ -320,7 +323,7 @@ def dflash_draft_step(cfg: Config, w: DeviceWeights, buf: StepBuffers,
                       new_states: Optional[torch.Tensor], ws: torch.Tensor,
                       new_off: Optional[torch.Tensor] = None,
                       ctx_cached: Optional[torch.Tensor] = None, verify: bool = False,
-                      stream=None):
+                      stream=None, confidence: bool = False):
     """One draft step over ``buf``'s blocks.  ``new_states`` [n_new][T][H]
     holds the target states of the context rows to (re)compute: all rows
     (``ctx_cached`` None) or rows [cached_r, L_r) of every request."""
@@ -341,6 +344,7 @@ def dflash_draft_step(cfg: Config, w: DeviceWeights, buf: StepBuffers,
     a.v_cache = buf._vc
     a.draft_tokens = buf.draft_tokens.data_ptr()
     a.max_logit = buf.max_logit.data_ptr()
+    a.confidence = buf.confidence.data_ptr() if confidence else None
     a.target_tokens = buf.target_tokens.data_ptr() if verify else None
     a.n_cand = buf.n_cand
     a.n_acc = buf.n_acc.data_ptr()

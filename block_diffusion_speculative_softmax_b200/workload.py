@@ -30,7 +30,8 @@ class Workload:
 
     def __init__(self, cfg: synth.DraftConfig, seed: int = 0, device: str = "cuda",
                  mode: str = "full", steady_new_rows: int = 6, host_weights: Optional[dict] = None,
-                 keep_host: bool = False, ctx_lens: Optional[List[int]] = None):
+                 keep_host: bool = False, ctx_lens: Optional[List[int]] = None,
+                 conf_source: str = "synthetic"):
         self.cfg = cfg
         self.seed = seed
         self.device = device
@@ -84,8 +85,15 @@ class Workload:
         if K > 1:
             self.buf2 = DF.StepBuffers(self.ccfg, self.ctx_lens, R * K, K, device,
                                        share_caches=self.buf)
-            self.conf = torch.from_numpy(synth.make_confidence(cfg, seed)).to(device)
+            # per-slot confidence for the D2SD cuts: a seeded U(0,1) field
+            # ("synthetic", the workload's stated input), or the first pass's
+            # own softmax probability of each drafted token ("draft")
+            if conf_source == "draft":
+                self.conf = self.buf.confidence
+            else:
+                self.conf = torch.from_numpy(synth.make_confidence(cfg, seed)).to(device)
             self.cached_all = torch.tensor(self.ctx_lens, dtype=torch.int32, device=device)
+        self.conf_source = conf_source if K > 1 else None
         nb_max = R * K
         self.ws_bytes = DF.dflash_workspace_size(self.ccfg, R, nb_max, n_new, max(self.ctx_lens))
         self.ws = DF.alloc_workspace(self.ws_bytes, device)
@@ -96,7 +104,8 @@ class Workload:
         """Pass 1: one block per request (the DFlash / DFLARE step)."""
         DF.dflash_draft_step(self.ccfg, self.w, self.buf, self.new_states, self.ws,
                              new_off=self.new_off, ctx_cached=self.ctx_cached,
-                             verify=verify, stream=stream)
+                             verify=verify, stream=stream,
+                             confidence=self.conf_source == "draft")
 
     def candidates(self, stream=None):
         """D2SD cuts from pass-1 tokens into the pass-2 block buffers."""

@@ -185,11 +185,14 @@ dflash_status dflash_mlp(const dflash_config* cfg, int64_t M, float* h,
 
 /* LM head with the argmax fused in (logits never reach memory):
  *   tok[m] = the lowest v with x[m] . w_lm[v] maximal;  max_logit[m] = that
- *   maximum (nullable).  x [M][H] (already normed); w_lm [V][H]. */
+ *   maximum (nullable);  conf[m] (nullable) = softmax probability of tok[m]
+ *   = 1 / sum_v exp(z_v - max z), the per-position confidence the D2SD
+ *   summary (methodology step 1) asks the first drafter for.  x [M][H]
+ *   (already normed); w_lm [V][H]. */
 dflash_status dflash_lmhead_argmax(const dflash_config* cfg, int64_t M,
                                    const void* x, const void* w_lm,
-                                   int32_t* tok, float* max_logit, void* ws,
-                                   size_t ws_bytes, void* stream);
+                                   int32_t* tok, float* max_logit, float* conf,
+                                   void* ws, size_t ws_bytes, void* stream);
 
 /* Greedy verification, DFlash summary methodology step 3 and D2SD summary
  * methodology step 4.  draft, target: [R][K][B] int32; slot 0 of a block is
@@ -256,6 +259,8 @@ typedef struct {
   void* const* v_cache;        /* host [D] */
   int32_t* draft_tokens;       /* out [nb][B]: slots < known_len copy the input */
   float* max_logit;            /* out [nb][B] (nullable) */
+  float* confidence;           /* out [nb][B] (nullable): softmax probability of each
+                                  drafted token (D2SD per-position confidence) */
   const int32_t* target_tokens;/* [nb][B] target argmax per slot (NULL = no verify) */
   int32_t n_cand;              /* K candidates per request in verification (nb = R*K) */
   int32_t* n_acc;              /* out [R] */

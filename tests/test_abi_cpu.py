@@ -78,14 +78,14 @@ def test_bad_pointers_and_sizes_rejected(lib):
     cfg = _cfg()
     # null / misaligned pointers
     st = lib.dflash_lmhead_argmax(C.byref(cfg), 4, None, C.c_void_p(16), C.c_void_p(16), None,
-                                  C.c_void_p(256), 1 << 20, None)
+                                  None, C.c_void_p(256), 1 << 20, None)
     assert st == DF.EINVAL and b"x is NULL" in lib.dflash_last_error()
     st = lib.dflash_lmhead_argmax(C.byref(cfg), 4, C.c_void_p(24), C.c_void_p(16),
-                                  C.c_void_p(16), None, C.c_void_p(256), 1 << 20, None)
+                                  C.c_void_p(16), None, None, C.c_void_p(256), 1 << 20, None)
     assert st == DF.EINVAL and b"aligned" in lib.dflash_last_error()
     # workspace too small
     st = lib.dflash_lmhead_argmax(C.byref(cfg), 4, C.c_void_p(16), C.c_void_p(16),
-                                  C.c_void_p(16), None, C.c_void_p(256), 64, None)
+                                  C.c_void_p(16), None, None, C.c_void_p(256), 64, None)
     assert st == DF.EINVAL and b"workspace too small" in lib.dflash_last_error()
     # accept: K and B out of range
     assert lib.dflash_accept(1, 0, 8, *([C.c_void_p(16)] * 5), None) == DF.EINVAL

@@ -91,3 +91,18 @@ def test_reference_arm_other_ranks_exit_quietly():
                           "--config", "tiny"], capture_output=True, text=True, timeout=120,
                          env=env)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_every_python_module_compiles():
+    """Modules that only GPU runs import (workload, bench's GPU arm) still
+    have to parse on a machine without a GPU."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    files = []
+    for d in ("", "block_diffusion_speculative_softmax_b200", "oracle", "tests",
+              os.path.join("tests", "golden")):
+        base = os.path.join(root, d)
+        files += [os.path.join(base, f) for f in os.listdir(base) if f.endswith(".py")]
+    assert len(files) > 10
+    for f in files:
+        with open(f) as fh:
+            compile(fh.read(), f, "exec")

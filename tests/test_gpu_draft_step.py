@@ -12,7 +12,7 @@ import torch
 
 from oracle import dflash_oracle as O
 from block_diffusion_speculative_softmax_b200 import synth
-from tests.gpu_common import check_draft, need_gpu, oracle_for_workload
+from tests.gpu_common import TOL, check_draft, need_gpu, oracle_for_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -103,15 +103,16 @@ def test_small_steady_state_matches_full(W):
     _run_pass1(W, cfg, mode="steady", steady_new_rows=7)
 
 
-def test_small_d2sd(W):
+@pytest.mark.parametrize("conf_source", ["draft", "synthetic"])
+def test_small_d2sd(W, conf_source):
     cfg = synth.small_config("d2sd_gptoss", hidden=640, n_q_heads=16, n_kv_heads=2, head_dim=64,
                              ffn=704, n_draft_layers=2, n_target_layers=5, ctx_len=150,
                              block=16, vocab=3001, n_req=3, n_cand=4)
-    _d2sd(W, cfg, reqs=None, ctx_lens=[150, 77, 260])
+    _d2sd(W, cfg, reqs=None, ctx_lens=[150, 77, 260], conf_source=conf_source)
 
 
-def _d2sd(W, cfg, reqs=None, ctx_lens=None):
-    wl = W.Workload(cfg, seed=0, keep_host=True, ctx_lens=ctx_lens)
+def _d2sd(W, cfg, reqs=None, ctx_lens=None, conf_source="synthetic"):
+    wl = W.Workload(cfg, seed=0, keep_host=True, ctx_lens=ctx_lens, conf_source=conf_source)
     reqs = list(range(cfg.n_req)) if reqs is None else reqs
     wl.draft()
     wl.check()
@@ -119,6 +120,15 @@ def _d2sd(W, cfg, reqs=None, ctx_lens=None):
     ot1, om1, keep1 = oracle_for_workload(wl, reqs, blocks1)
     check_draft(wl, wl.buf.draft_tokens.cpu().numpy()[reqs],
                 wl.buf.max_logit.cpu().numpy()[reqs], ot1, om1, keep1, blocks1, "d2sd pass 1")
+    if conf_source == "draft":
+        # the first pass's confidence against the oracle's softmax of its logits
+        # (conf = exp(z_max - lse): logits within d of the oracle's move it
+        # by a factor within exp(+-2d), d taken from the logit tolerance)
+        z = np.stack([keep1["logits"][i] for i in range(len(blocks1))])
+        oc = np.stack([O.draft_confidence(zi) for zi in z])[:, 1:]
+        gc = wl.buf.confidence.cpu().numpy()[reqs][:, 1:].astype(np.float64)
+        d = TOL[cfg.dtype] * max(1.0, float(np.abs(z).max()))
+        assert np.all(np.abs(np.log(gc / oc)) <= 2 * d), np.abs(np.log(gc / oc)).max()
     # cuts on the GPU from the GPU's base tokens must equal the oracle's cuts
     # on the same base tokens
     wl.candidates()

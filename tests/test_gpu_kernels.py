@@ -180,8 +180,9 @@ def test_lmhead_argmax(DF, dtype, M, H, V):
     dt = _tdt(cfg)
     tok = torch.full((M,), -7, dtype=torch.int32, device="cuda")
     mx = torch.zeros(M, dtype=torch.float32, device="cuda")
+    conf = torch.full((M,), -1.0, dtype=torch.float32, device="cuda")
     ws = DF.alloc_workspace(DF.dflash_workspace_size(ccfg, 1, (M + 15) // 16, 0, 0))
-    DF.dflash_lmhead_argmax(ccfg, to_dev(x, dt), to_dev(w, dt), tok, mx, ws)
+    DF.dflash_lmhead_argmax(ccfg, to_dev(x, dt), to_dev(w, dt), tok, mx, ws, conf=conf)
     DF.dflash_check(ws)
     otok, omax, z = O.lmhead_argmax(x, w)
     gt = tok.cpu().numpy()
@@ -191,6 +192,11 @@ def test_lmhead_argmax(DF, dtype, M, H, V):
     assert not bad, bad[:5]
     assert gt[0] == min(dup + [win])          # lowest index among exact ties
     assert rel_err(mx.cpu().numpy(), omax) <= (1e-5 if dtype == "fp32" else 1e-3)
+    # confidence = softmax probability of the argmax (one log-sum-exp share
+    # per vocabulary tile, merged in a second pass)
+    oc = O.draft_confidence(z)
+    gc = conf.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(gc - oc) <= (1e-4 if dtype == "fp32" else 1e-3) * oc + 1e-7)
 
 
 def test_lmhead_nonfinite_reports_enumeric(DF):
