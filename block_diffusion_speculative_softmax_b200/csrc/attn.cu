@@ -5,8 +5,13 @@
 // Split-KV (flash-decoding): the grid is (block x kv head, split, query-row
 // chunk).  A split streams its slice of the request's packed context K/V
 // (split 0 also takes the B block keys) and keeps an fp32 online softmax
-// (running max m, sum l, unnormalised output o) per query row; a combine
-// kernel merges the splits in a fixed order.
+// (running max m, sum l, unnormalised output o) per query row.  In the bf16
+// path the splits of one (block, kv head, row chunk) form a thread-block
+// cluster: each split leaves its partials in its own shared memory and, after
+// a cluster barrier, every CTA merges a slice of the rows by reading all the
+// splits' partials over distributed shared memory, so partials never reach
+// global memory and no second kernel runs.  The fp32 path writes partials
+// and a combine kernel merges them.  Both merge the splits in a fixed order.
 #include <algorithm>
 #include <mutex>
 
@@ -28,6 +33,7 @@ struct AttnParams {
   float scale;
   float* part_o;   // [nb*B*Hq][splits][d]
   float* part_ml;  // [nb*B*Hq][splits][2]
+  void* out;       // [nb*B*Hq][d] (bf16 cluster / single-split paths)
 };
 
 constexpr int kAttnWarps = 4;
@@ -183,7 +189,37 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int D>
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory variable in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float dsmem_ld(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 dsmem_ld4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
+// CS = 0: partials to global memory for the combine kernel.  CS = 1: one
+// split, normalised in registers.  CS >= 2: the grid's y extent is CS and
+// each cluster of CS CTAs (one per split) merges through shared memory.
+template <int D, int CS>
 __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnParams p) {
   constexpr int CH = D / 8;                 // 16-byte chunks per key row
   constexpr int NT = kMmaKeys / 8;          // n-tiles of S per key tile
@@ -360,21 +396,117 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnParams p) {
     l1 += __shfl_xor_sync(0xffffffffu, l1, off);
   }
   constexpr float kLn2 = 0.6931471805599453f;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int rr = rbase + gq + 8 * h;
-    if (rr >= nrows_all) continue;
+  auto out_row = [&](int rr) -> size_t {   // output row of query row rr
     const int s = rr / p.G, j = rr % p.G;
-    const size_t pr = (static_cast<size_t>(b) * p.B + s) * p.Hq + g * p.G + j;
-    float* po = p.part_o + (pr * p.splits + split) * D;
+    return (static_cast<size_t>(b) * p.B + s) * p.Hq + g * p.G + j;
+  };
+  if constexpr (CS == 0) {
 #pragma unroll
-    for (int dt = 0; dt < DT; ++dt)
-      *reinterpret_cast<float2*>(po + dt * 8 + 2 * tq) = make_float2(o[dt][2 * h], o[dt][2 * h + 1]);
-    if (tq == 0) {
-      const float mm = h ? m1 : m0;
-      p.part_ml[(pr * p.splits + split) * 2 + 0] = mm == -INFINITY ? -INFINITY : mm * kLn2;
-      p.part_ml[(pr * p.splits + split) * 2 + 1] = h ? l1 : l0;
+    for (int h = 0; h < 2; ++h) {
+      const int rr = rbase + gq + 8 * h;
+      if (rr >= nrows_all) continue;
+      const size_t pr = out_row(rr);
+      float* po = p.part_o + (pr * p.splits + split) * D;
+#pragma unroll
+      for (int dt = 0; dt < DT; ++dt)
+        *reinterpret_cast<float2*>(po + dt * 8 + 2 * tq) =
+            make_float2(o[dt][2 * h], o[dt][2 * h + 1]);
+      if (tq == 0) {
+        const float mm = h ? m1 : m0;
+        p.part_ml[(pr * p.splits + split) * 2 + 0] = mm == -INFINITY ? -INFINITY : mm * kLn2;
+        p.part_ml[(pr * p.splits + split) * 2 + 1] = h ? l1 : l0;
+      }
     }
+  } else if constexpr (CS == 1) {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int rr = rbase + gq + 8 * h;
+      if (rr >= nrows_all) continue;
+      const float inv = 1.f / (h ? l1 : l0);
+      __nv_bfloat16* orow = out + out_row(rr) * D;
+#pragma unroll
+      for (int dt = 0; dt < DT; ++dt)
+        *reinterpret_cast<__nv_bfloat162*>(orow + dt * 8 + 2 * tq) =
+            __floats2bfloat162_rn(o[dt][2 * h] * inv, o[dt][2 * h + 1] * inv);
+    }
+  } else {
+    // this split's partials into its own shared memory (the K/V ring is free:
+    // the loop ended on a block barrier)
+    constexpr int OS = D + 4;                 // padded row stride (16-byte aligned)
+    constexpr int RPR = kMmaRows / CS;        // rows merged by each CTA
+    float* so = reinterpret_cast<float*>(smraw);            // [64][OS]
+    float* sml = so + kMmaRows * OS;                         // [64][2]
+    __shared__ float w_s[RPR][CS];
+    __shared__ float den_s[RPR];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = warp * 16 + gq + 8 * h;
+#pragma unroll
+      for (int dt = 0; dt < DT; ++dt)
+        *reinterpret_cast<float2*>(so + row * OS + dt * 8 + 2 * tq) =
+            make_float2(o[dt][2 * h], o[dt][2 * h + 1]);
+      if (tq == 0) {
+        const float mm = h ? m1 : m0;
+        sml[row * 2 + 0] = mm == -INFINITY ? -INFINITY : mm * kLn2;
+        sml[row * 2 + 1] = h ? l1 : l0;
+      }
+    }
+    cluster_sync_all();   // every split's partials are now visible cluster-wide
+    const uint32_t rank = cluster_rank();
+    const uint32_t so_u = smem_u32(so), sml_u = smem_u32(sml);
+    if (tid < RPR) {
+      const int row = static_cast<int>(rank) * RPR + tid;
+      float ms[CS], ls[CS];
+#pragma unroll
+      for (int sp = 0; sp < CS; ++sp) {
+        const uint32_t a = dsmem_addr(sml_u + row * 8, sp);
+        ms[sp] = dsmem_ld(a);
+        ls[sp] = dsmem_ld(a + 4);
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int sp = 0; sp < CS; ++sp)
+        if (ls[sp] > 0.f) M = fmaxf(M, ms[sp]);
+      float den = 0.f;
+#pragma unroll
+      for (int sp = 0; sp < CS; ++sp) {
+        const float w = ls[sp] > 0.f ? __expf(ms[sp] - M) : 0.f;
+        den = fmaf(ls[sp], w, den);
+        w_s[tid][sp] = w;
+      }
+      den_s[tid] = den;
+    }
+    __syncthreads();
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+    constexpr int C4 = D / 4;
+    for (int e = tid; e < RPR * C4; e += 128) {
+      const int r = e / C4, c4 = e % C4;
+      const int row = static_cast<int>(rank) * RPR + r;
+      const int rr = blockIdx.z * kMmaRows + row;
+      if (rr >= nrows_all) continue;
+      float4 v[CS];
+#pragma unroll
+      for (int sp = 0; sp < CS; ++sp)
+        v[sp] = dsmem_ld4(dsmem_addr(so_u + (row * OS + c4 * 4) * 4, sp));
+      float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int sp = 0; sp < CS; ++sp) {
+        const float w = w_s[r][sp];
+        num.x = fmaf(v[sp].x, w, num.x);
+        num.y = fmaf(v[sp].y, w, num.y);
+        num.z = fmaf(v[sp].z, w, num.z);
+        num.w = fmaf(v[sp].w, w, num.w);
+      }
+      const float den = den_s[r];
+      __nv_bfloat162 lo = __floats2bfloat162_rn(num.x / den, num.y / den);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(num.z / den, num.w / den);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(out + out_row(rr) * D + c4 * 4) = pk;
+    }
+    cluster_sync_all();   // peers may still be reading this CTA's partials
   }
 }
 
@@ -408,20 +540,56 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
 }
 
 // Opt every attention kernel into large dynamic shared memory once (on the
-// first call, which must come before any stream capture).
+// first call, which must come before any stream capture), allow the
+// 16-CTA clusters, and record the largest cluster the device can schedule.
+static int g_max_cluster = 8;
+
+template <int D>
+static void attn_kernels(const void** ks) {
+  ks[0] = reinterpret_cast<const void*>(attn_mma_kernel<D, 0>);
+  ks[1] = reinterpret_cast<const void*>(attn_mma_kernel<D, 1>);
+  ks[2] = reinterpret_cast<const void*>(attn_mma_kernel<D, 2>);
+  ks[3] = reinterpret_cast<const void*>(attn_mma_kernel<D, 4>);
+  ks[4] = reinterpret_cast<const void*>(attn_mma_kernel<D, 8>);
+  ks[5] = reinterpret_cast<const void*>(attn_mma_kernel<D, 16>);
+  ks[6] = reinterpret_cast<const void*>(attn_simt_kernel<float, D>);
+}
+
 static cudaError_t allow_smem() {
   static std::once_flag once;
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
     const int bytes = 200 * 1024;
-    const void* ks[4] = {reinterpret_cast<const void*>(attn_simt_kernel<float, 64>),
-                         reinterpret_cast<const void*>(attn_simt_kernel<float, 128>),
-                         reinterpret_cast<const void*>(attn_mma_kernel<64>),
-                         reinterpret_cast<const void*>(attn_mma_kernel<128>)};
+    const void* ks[14];
+    attn_kernels<64>(ks);
+    attn_kernels<128>(ks + 7);
     for (const void* k : ks) {
       cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
       if (e != cudaSuccess && err == cudaSuccess) err = e;
     }
+    // 16-CTA clusters are opt-in; keep them only if one can be resident
+    bool ok16 = true;
+    for (const void* k : {ks[5], ks[12]})
+      ok16 = ok16 && cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                         cudaSuccess;
+    if (ok16) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(1, 16, 1);
+      cfg.blockDim = dim3(128);
+      cfg.dynamicSmemBytes = 2 * 2 * kMmaKeys * 128 * sizeof(__nv_bfloat16);
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 1;
+      attr[0].val.clusterDim.y = 16;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      ok16 = cudaOccupancyMaxActiveClusters(&n, attn_mma_kernel<128, 16>, &cfg) == cudaSuccess &&
+             n > 0;
+    }
+    cudaGetLastError();   // a refused probe leaves no error behind
+    g_max_cluster = ok16 ? 16 : 8;
   });
   return err;
 }
@@ -433,6 +601,25 @@ AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d, int64_t max
   const int G = Hq / Hkv;
   p.row_chunks = (B * G + p.rows_per_cta - 1) / p.rows_per_cta;
   const int64_t base = static_cast<int64_t>(nb) * Hkv * p.row_chunks;
+  const int64_t want = (2 * kNumSMs + base - 1) / base;
+  if (dtype == DFLASH_BF16) {
+    // one cluster of 2^k splits (up to 16) per (block, kv head, row chunk);
+    // at least 128 context keys per split
+    p.cluster = 1;
+    if (max_ctx_len <= 0) {
+      p.splits = 1;
+      p.chunk = 64;
+      return p;
+    }
+    const int64_t max_splits = std::min<int64_t>(16, (max_ctx_len + 127) / 128);
+    const int64_t n = std::max<int64_t>(1, std::min(want, max_splits));
+    while (p.cluster < n) p.cluster *= 2;
+    int64_t chunk = (max_ctx_len + p.cluster - 1) / p.cluster;
+    p.chunk = static_cast<int>((chunk + 63) / 64 * 64);
+    p.splits = p.cluster;
+    return p;
+  }
+  p.cluster = 0;
   if (max_ctx_len <= 0) {
     p.splits = 1;
     p.chunk = 64;
@@ -442,7 +629,6 @@ AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d, int64_t max
   // then stay below the K/V bytes it streams
   const int64_t min_chunk = 256;
   const int64_t max_splits = std::min<int64_t>(64, (max_ctx_len + min_chunk - 1) / min_chunk);
-  int64_t want = (2 * kNumSMs + base - 1) / base;
   int64_t splits = std::max<int64_t>(1, std::min(want, max_splits));
   int64_t chunk = (max_ctx_len + splits - 1) / splits;
   chunk = (chunk + 63) / 64 * 64;
@@ -451,9 +637,44 @@ AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d, int64_t max
   return p;
 }
 
+// Partials in global memory are only needed by the fp32 path and by the
+// bf16 fallback when a 16-CTA cluster cannot be scheduled.
 size_t attn_ws_bytes(const AttnPlan& p, int nb, int B, int Hq, int d) {
   const size_t rows = static_cast<size_t>(nb) * B * Hq;
   return rows * p.splits * (d + 2) * sizeof(float);
+}
+
+template <int D, int CS>
+static cudaError_t launch_cluster(const AttnParams& p, dim3 grid, size_t smem, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = CS;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, attn_mma_kernel<D, CS>, p);
+}
+
+template <int D>
+static cudaError_t launch_bf16(const AttnParams& p, int cs, dim3 grid, size_t smem,
+                               cudaStream_t st) {
+  switch (cs) {
+    case 1: return launch_k(attn_mma_kernel<D, 1>, grid, dim3(128), smem, st, p);
+    case 2: return launch_cluster<D, 2>(p, grid, smem, st);
+    case 4: return launch_cluster<D, 4>(p, grid, smem, st);
+    case 8: return launch_cluster<D, 8>(p, grid, smem, st);
+    case 16: return launch_cluster<D, 16>(p, grid, smem, st);
+    default: return launch_k(attn_mma_kernel<D, 0>, grid, dim3(128), smem, st, p);
+  }
 }
 
 cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq, int Hkv, int d,
@@ -471,24 +692,27 @@ cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq, 
   p.chunk = plan.chunk;
   p.rows_per_cta = plan.rows_per_cta;
   p.scale = 1.0f / sqrtf(static_cast<float>(d));
+  p.out = out;
   const int64_t n_rows = static_cast<int64_t>(nb) * B * Hq;
   p.part_o = ws;
   p.part_ml = ws + static_cast<size_t>(n_rows) * plan.splits * d;
   dim3 grid(nb * Hkv, plan.splits, plan.row_chunks);
   cudaError_t e = allow_smem();
   if (e != cudaSuccess) return e;
+  int cs = 0;   // 0: partials through global memory + combine kernel
   if (dtype == DFLASH_BF16) {
+    cs = plan.cluster <= g_max_cluster ? plan.cluster : 0;
     const size_t smem = 2 * 2 * static_cast<size_t>(kMmaKeys) * d * sizeof(__nv_bfloat16);
-    e = d == 64 ? launch_k(attn_mma_kernel<64>, grid, dim3(128), smem, st, p)
-                : launch_k(attn_mma_kernel<128>, grid, dim3(128), smem, st, p);
+    e = d == 64 ? launch_bf16<64>(p, cs, grid, smem, st) : launch_bf16<128>(p, cs, grid, smem, st);
+    if (e != cudaSuccess || cs != 0) return e;
   } else {
     const size_t smem = (static_cast<size_t>(plan.rows_per_cta) * d +
                          kAttnKeyTile * (d + 1) + kAttnKeyTile * d) * sizeof(float);
     e = d == 64 ? launch_k(attn_simt_kernel<float, 64>, grid, dim3(kAttnWarps * 32), smem, st, p)
                 : launch_k(attn_simt_kernel<float, 128>, grid, dim3(kAttnWarps * 32), smem, st,
                            p);
+    if (e != cudaSuccess) return e;
   }
-  if (e != cudaSuccess) return e;
   const int64_t total = n_rows * d;
   const dim3 cgrid(static_cast<unsigned>((total + 255) / 256));
   if (dtype == DFLASH_BF16)

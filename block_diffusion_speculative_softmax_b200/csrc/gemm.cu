@@ -80,6 +80,8 @@ struct Params {
   int kb_per_split;
   int splits;
   int row_tiles;
+  int tok_fast;                     // token-major grid: token tiles on x (weight tile shared
+                                    // by the CTAs that run together), else feature tiles on x
   float* partial;                   // [tiles][splits][BN][BM]
   uint32_t* counters;               // [tiles]
   const int32_t* pos;
@@ -318,30 +320,41 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
       if (do_op) {
         __threadfence();
         // the tile's BN x 128 floats as float4 items (token j, rows 4q..4q+3),
-        // each summed over the splits in fixed order, straight into staging;
-        // every thread keeps 4 items x 2 splits of loads in flight
+        // each summed over the splits in fixed order, straight into staging.
+        // A thread owns 4 items and loads 8 splits of each at once (32 float4
+        // in flight), so the reduction costs ceil(splits / 8) L2 round trips
+        // per 4 items instead of one per split.
         const float4* base = reinterpret_cast<const float4*>(
             p.partial + static_cast<size_t>(tile_lin) * p.splits * BN * BM);
         constexpr int ITEMS = BN * (BM / 4);
         constexpr int NT = 128;
+        constexpr int SB = 8;   // splits per batch of loads
 #pragma unroll 1
         for (int it0 = 0; it0 < ITEMS; it0 += 4 * NT) {
           float4 acc[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-          for (int sp = 0; sp < p.splits; ++sp) {
-            float4 a[4];
+#pragma unroll 1
+          for (int sp0 = 0; sp0 < p.splits; sp0 += SB) {
+            float4 a[4][SB];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int it = it0 + q * NT + tid;
-              a[q] = it < ITEMS ? __ldcg(base + static_cast<size_t>(sp) * ITEMS + it)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+            for (int u = 0; u < SB; ++u)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              acc[q].x += a[q].x; acc[q].y += a[q].y; acc[q].z += a[q].z; acc[q].w += a[q].w;
-            }
+              for (int q = 0; q < 4; ++q) {
+                const int it = it0 + q * NT + tid;
+                a[q][u] = (it < ITEMS && sp0 + u < p.splits)
+                              ? __ldcg(base + static_cast<size_t>(sp0 + u) * ITEMS + it)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+#pragma unroll
+            for (int u = 0; u < SB; ++u)
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                if (sp0 + u < p.splits) {
+                  acc[q].x += a[q][u].x; acc[q].y += a[q][u].y;
+                  acc[q].z += a[q][u].z; acc[q].w += a[q][u].w;
+                }
+              }
           }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -461,13 +474,16 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
   const int lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
 
-  const int tile = blockIdx.x;                // feature tile
+  // the operand with fewer tiles varies fastest, so the CTAs resident
+  // together share the larger operand's tile through L2 and it crosses HBM once
+  const int tile = p.tok_fast ? blockIdx.y : blockIdx.x;       // feature tile
+  const int tok_tile = p.tok_fast ? blockIdx.x : blockIdx.y;
   int sg = 0;
   while (sg + 1 < p.nseg && tile >= p.seg[sg + 1].tile_begin) ++sg;
   const Seg& S = p.seg[sg];
   const int pair = S.pair;
   const int f0 = (tile - S.tile_begin) * (pair ? BW / 2 : BW);   // first output feature
-  const int tok0 = blockIdx.y * BM;
+  const int tok0 = tok_tile * BM;
   const int kb0 = blockIdx.z * p.kb_per_split;
   const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
   const int nkb = kb1 - kb0;
@@ -560,7 +576,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
   const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
   const int t = tok0 + tid;
   const bool tv = t < p.M;
-  const int tile_lin = blockIdx.y * p.row_tiles + blockIdx.x;
+  const int tile_lin = tok_tile * p.row_tiles + tile;
 
   // split-K: every split parks its fp32 tile, the last one sums them
   bool do_op = live;
@@ -633,7 +649,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
         }
       }
       if (tv && best) atomicMax(p.keys + t, best);
-      if (tv && p.lse != nullptr) p.lse[static_cast<size_t>(blockIdx.x) * p.M + t] = make_float2(mx, se);
+      if (tv && p.lse != nullptr) p.lse[static_cast<size_t>(tile) * p.M + t] = make_float2(mx, se);
     } else if (S.op == EPI_SWIGLU) {
       __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out) + static_cast<int64_t>(t) * S.out_stride;
 #pragma unroll 1
@@ -1216,6 +1232,12 @@ cudaError_t launch_tok(const Params& p, dim3 grid, cudaStream_t st) {
   return launch_k(gemm_tok_kernel<BW, STAGES, ARGMAX>, grid, dim3(128), SMEM, st, p);
 }
 
+// Token tiles on grid x when there are fewer of them than feature tiles (and
+// the feature tiles fit grid y): the weights then stream from HBM once.
+inline bool tok_fast(int tok_tiles, int feature_tiles) {
+  return tok_tiles < feature_tiles && feature_tiles <= 65535;
+}
+
 template <bool ARGMAX>
 cudaError_t dispatch_tok(int bw, const Params& p, dim3 grid, cudaStream_t st) {
   switch (bw) {
@@ -1647,7 +1669,11 @@ cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& pl, float* partial,
     return tc::dispatch_sk<false>(pl.bn, p, geo, st);
   }
   dim3 grid(tiles, pl.tok_tiles, pl.splits);
-  if (pl.tok_major) return tc::dispatch_tok<false>(pl.bn, p, grid, st);
+  if (pl.tok_major) {
+    p.tok_fast = tc::tok_fast(pl.tok_tiles, tiles);
+    if (p.tok_fast) grid = dim3(pl.tok_tiles, tiles, pl.splits);
+    return tc::dispatch_tok<false>(pl.bn, p, grid, st);
+  }
   return tc::dispatch<false>(pl.bn, p, grid, st);
 }
 
@@ -1695,7 +1721,9 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X,
     p.keys = keys;
     p.lse = lse;
     p.status = status;
-    dim3 grid(ceil_div(V, BW), ceil_div(M, tc::BM), 1);
+    const int tt = ceil_div(M, tc::BM);
+    p.tok_fast = tc::tok_fast(tt, p.row_tiles);
+    const dim3 grid = p.tok_fast ? dim3(tt, p.row_tiles, 1) : dim3(p.row_tiles, tt, 1);
     return tc::dispatch_tok<true>(BW, p, grid, st);
   }
   if (dtype == DFLASH_BF16 && partial != nullptr) {

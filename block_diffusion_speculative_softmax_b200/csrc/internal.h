@@ -146,6 +146,7 @@ struct AttnPlan {
   int chunk;        // context keys per split (multiple of 64)
   int row_chunks;   // CTAs along the query rows of one (block, kv head)
   int rows_per_cta;
+  int cluster;      // bf16: splits merged in one CTA cluster (power of two); 0: combine kernel
 };
 AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d,
                    int64_t max_ctx_len);

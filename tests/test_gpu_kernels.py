@@ -111,8 +111,10 @@ def test_kv_project(DF, dtype, M, scatter):
     ("bf16", [0, 5, 100, 777], 16, 8, 2, 128, [0, 1, 2, 3, 3]),
     ("bf16", [150, 77], 16, 16, 2, 64, [0, 0, 0, 1, 1]),
     ("bf16", [33], 1, 4, 4, 64, [0]),
+    ("bf16", [400, 13], 16, 16, 4, 64, [1, 0]),
 ])
 def test_block_attn(DF, dtype, lens, B, Hq, Hkv, d, blk_req):
+    # bf16 cases cover split clusters of 16, 8, 2, 1 and 4 CTAs in that order
     cfg = _cfg(dtype, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, block=B)
     rng = np.random.default_rng(sum(lens) + B)
     nb = len(blk_req)
