@@ -34,6 +34,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "draft blocks/s and accepted tok/s per B200; HBM GB/s / tensor util vs peak"
 ACCEPT_DRAWS = 32          # planted target draws averaged for accepted tok/s
+# DRAM bytes (read + write) of one LM-head launch from an ncu capture of
+# `bench.py --op lmhead` (summarised under profiles/), valid only for the
+# GEMM source it was taken with; any later edit of gemm.cu nulls it.
+LMHEAD_TRAFFIC = {}        # workload -> {"bytes": int, "gemm_cu_sha256": str}
 
 
 def parse():
@@ -371,6 +375,19 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def lmhead_traffic(workload):
+    """Measured DRAM bytes per LM-head launch, or None when there is no
+    capture for this workload or the GEMM source changed since."""
+    import hashlib
+    ent = LMHEAD_TRAFFIC.get(workload)
+    if ent is None:
+        return None
+    src = os.path.join(ROOT, "block_diffusion_speculative_softmax_b200", "csrc", "gemm.cu")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    return ent["bytes"] if digest.startswith(ent["gemm_cu_sha256"]) else None
+
+
 def roofline(args, wl, cfg, DF, hbm_peak, tf_burst, peak_src, stream):
     """LM-head argmax (weight streaming, the largest single launch of the
     step), timed alone with CUDA events on its launch stream."""
@@ -397,7 +414,7 @@ def roofline(args, wl, cfg, DF, hbm_peak, tf_burst, peak_src, stream):
     algo = V * H * esz + M * H * esz + M * 8 + M * 4
     flops = 2.0 * M * V * H
     common = {"kernel": "lmhead_argmax (tcgen05 GEMM, argmax epilogue)",
-              "peak_source": peak_src, "traffic": None,
+              "peak_source": peak_src, "traffic": lmhead_traffic(cfg.name),
               "algorithmic_bytes_per_launch": algo, "algorithmic_flops_per_launch": flops,
               "us_per_launch": sec * 1e6,
               "note": "time includes the argmax-key reset and finish launches"}
@@ -507,14 +524,14 @@ def run_op(args):
         tok = torch.empty(M, dtype=torch.int32, device="cuda")
         call = lambda: DF.dflash_lmhead_argmax(cc, x, w, tok, None, ws)
         algo = V * H * e + M * H * e + M * 4
-        kernel = "gemm_kernel<16,6,ARGMAX> (LM head)"
+        kernel = "gemm_sk_kernel<ARGMAX> (<= 64 tokens) / gemm_tok_kernel<ARGMAX> (LM head)"
     elif args.op == "mlp":
         h = rnd(M, H, dtype=torch.float32)
         gm = torch.ones(H, device="cuda")
         wg, wu, wd = rnd(F, H, scale=0.02), rnd(F, H, scale=0.02), rnd(H, F, scale=0.02)
         call = lambda: DF.dflash_mlp(cc, h, gm, wg, wu, wd, ws)
         algo = 3 * F * H * e + 2 * M * H * 4
-        kernel = "rmsnorm + gemm_kernel x2 + finish x2 (SwiGLU MLP)"
+        kernel = "rmsnorm + gemm_kernel x2 (split-K, SwiGLU and residual epilogues)"
     elif args.op == "ctxproj":
         x = rnd(N, H)
         pos = torch.arange(N, dtype=torch.int32, device="cuda")
@@ -524,7 +541,7 @@ def run_op(args):
         call = lambda: DF.dflash_kv_project(cc, x, pos, None, wk, wv, ko, vo, ws)
         algo = N * H * e + 2 * kvd * H * e + 2 * N * kvd * e
         flops = 2.0 * N * H * 2 * kvd
-        kernel = "gemm_kernel<256,4> + finish (context K/V projection, RoPE)"
+        kernel = "gemm_tok_kernel<256,4> (context K/V projection, RoPE epilogue)"
     elif args.op == "attn":
         q, kb, vb = rnd(M, qd), rnd(M, kvd), rnd(M, kvd)
         kc, vc = rnd(N, kvd), rnd(N, kvd)
@@ -536,7 +553,7 @@ def run_op(args):
                                             ws)
         algo = 2 * N * kvd * e + 2 * M * qd * e + 2 * M * kvd * e
         flops = 4.0 * cfg.n_cand * N * cfg.block * qd
-        kernel = "attn_mma_kernel + combine (split-KV block attention)"
+        kernel = "attn_mma_kernel<d, CS> (split-KV block attention, cluster merge)"
     else:  # fuse
         st = rnd(N, T, H)
         wf = torch.randn(D, T, device="cuda", generator=g)

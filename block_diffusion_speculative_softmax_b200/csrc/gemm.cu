@@ -165,13 +165,16 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
   const uint32_t tmem = tmem_slot;
   if (tid == 0) pdl_launch();
 
+  // weights are read once per step: evict them first so L2 keeps what is
+  // reused (activations, K/V, prefetched weights of the next GEMM)
+  const uint64_t pol = policy_evict_first();
   auto load_w = [&](int i, uint8_t* sa) {
     const int kc = (kb0 + i) * BK;
     if (pair) {
-      tma_load_2d(sa, tma, &full_bar[i % STAGES], kc, row0);
-      tma_load_2d(sa + A_BYTES / 2, tmb, &full_bar[i % STAGES], kc, row0);
+      tma_load_2d_hint(sa, tma, &full_bar[i % STAGES], kc, row0, pol);
+      tma_load_2d_hint(sa + A_BYTES / 2, tmb, &full_bar[i % STAGES], kc, row0, pol);
     } else {
-      tma_load_2d(sa, tma, &full_bar[i % STAGES], kc, row0);
+      tma_load_2d_hint(sa, tma, &full_bar[i % STAGES], kc, row0, pol);
     }
   };
 
@@ -451,14 +454,25 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
 // tile, a residual row and an argmax over the tile's vocabulary rows are
 // all formed in that thread's registers, straight out of TMEM.
 // ---------------------------------------------------------------------------
-template <int BW, int STAGES, bool ARGMAX>
+//
+// TWO: a cluster of two CTAs on consecutive token tiles computes one
+// 256-token x BW tile with cta_group::2 MMAs.  Each CTA stages its own 128
+// token rows and HALF of the tile's BW weight rows (gate rows in the even
+// CTA and up rows in the odd one for a SwiGLU tile), so every weight byte
+// reaching shared memory feeds 256 tokens instead of 128 and each CTA moves
+// 2/3 of the bytes per FLOP of the single-CTA tile.  The even CTA counts
+// both CTAs' TMA bytes on its stage barriers and issues the MMAs; their
+// commits arrive on the stage and accumulator barriers of both CTAs.
+template <int BW, int STAGES, bool ARGMAX, bool TWO = false>
 __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant__ Params p) {
   constexpr int X_BYTES = BM * BK * 2;        // 128 tokens x 64 k
-  constexpr int W_BYTES = BW * BK * 2;
+  constexpr int W_ROWS = TWO ? BW / 2 : BW;   // weight rows this CTA stages
+  constexpr int W_BYTES = W_ROWS * BK * 2;
   constexpr int STAGE = X_BYTES + W_BYTES;
   constexpr uint32_t TMEM_COLS = BW;
-  constexpr uint32_t IDESC = idesc_bf16(BM, BW);
+  constexpr uint32_t IDESC = idesc_bf16(TWO ? 2 * BM : BM, BW);
   static_assert(STAGE % 1024 == 0, "stages must stay 1024-byte aligned");
+  static_assert(!TWO || BW == 256, "CTA pairs use 256-feature tiles");
 
   extern __shared__ uint8_t dsmem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -476,8 +490,25 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
 
   // the operand with fewer tiles varies fastest, so the CTAs resident
   // together share the larger operand's tile through L2 and it crosses HBM once
-  const int tile = p.tok_fast ? blockIdx.y : blockIdx.x;       // feature tile
-  const int tok_tile = p.tok_fast ? blockIdx.x : blockIdx.y;
+  // (CTA pairs: a 1-D grid of clusters of two along x; consecutive CTAs are
+  // the two token tiles of one pair, pairs ordered the same way)
+  int tile, tok_tile;
+  if constexpr (TWO) {
+    const int pidx = static_cast<int>(blockIdx.x >> 1);
+    const int tok_pairs = static_cast<int>(gridDim.x >> 1) / p.row_tiles;
+    int tp;
+    if (p.tok_fast) {
+      tp = pidx % tok_pairs;
+      tile = pidx / tok_pairs;
+    } else {
+      tile = pidx % p.row_tiles;
+      tp = pidx / p.row_tiles;
+    }
+    tok_tile = 2 * tp + static_cast<int>(blockIdx.x & 1u);
+  } else {
+    tile = p.tok_fast ? blockIdx.y : blockIdx.x;       // feature tile
+    tok_tile = p.tok_fast ? blockIdx.x : blockIdx.y;
+  }
   int sg = 0;
   while (sg + 1 < p.nseg && tile >= p.seg[sg + 1].tile_begin) ++sg;
   const Seg& S = p.seg[sg];
@@ -487,8 +518,19 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
   const int kb0 = blockIdx.z * p.kb_per_split;
   const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
   const int nkb = kb1 - kb0;
+  const uint32_t rank = TWO ? cluster_rank() : 0u;   // 0: the CTA that issues the MMAs
   const CUtensorMap* tma = &p.tm[S.map];
   const CUtensorMap* tmb = pair ? &p.tm[S.map + 1] : nullptr;
+  // The CTAs that share a weight tile start their k loops at different
+  // k-blocks, so they do not all request the same L2 lines at once.  The
+  // order depends on the token tile only: every feature of a token sums its
+  // k-blocks in the same order, so equal weight rows give equal outputs
+  // (exact argmax ties stay ties).  Both CTAs of a pair walk the same order.
+  const int rot = nkb > 0 ? (TWO ? tok_tile >> 1 : tok_tile) % nkb : 0;
+  auto kblk = [&](int i) {
+    const int j = i + rot;
+    return kb0 + (j >= nkb ? j - nkb : j);
+  };
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -502,33 +544,54 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
     if (tmb) tma_prefetch_desc(tmb);
     tma_prefetch_desc(&p.tm_x);
   }
-  if (warp == 2) tmem_alloc(&tmem_slot, TMEM_COLS);
+  if (warp == 2) {
+    if constexpr (TWO) tmem_alloc_pair(&tmem_slot, TMEM_COLS);
+    else tmem_alloc(&tmem_slot, TMEM_COLS);
+  }
   tc_fence_before();
   __syncthreads();
+  // both CTAs' barriers exist before either CTA's copies or commits reach them
+  if constexpr (TWO) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   if (tid == 0) pdl_launch();
 
-  // stage layout: [X tile 16 KB][W tile BW x 128 B]
+  // stage barrier that counts this CTA's copies: its own, or the even CTA's
+  auto full_addr = [&](int s) -> uint32_t {
+    const uint32_t a = smem_u32(&full_bar[s]);
+    return TWO && rank != 0 ? dsmem_addr(a, 0) : a;
+  };
+  auto load_x = [&](int i, uint8_t* sx) {
+    if constexpr (TWO) tma_load_2d_pair(sx, &p.tm_x, full_addr(i % STAGES), kblk(i) * BK, tok0);
+    else tma_load_2d(sx, &p.tm_x, &full_bar[i % STAGES], kblk(i) * BK, tok0);
+  };
+  // stage layout: [X tile 16 KB][W rows W_ROWS x 128 B]
   auto load_w = [&](int i, uint8_t* sw) {
-    const int kc = (kb0 + i) * BK;
-    if (pair) {
+    const int kc = kblk(i) * BK;
+    if constexpr (TWO) {
+      const uint32_t bar = full_addr(i % STAGES);
+      if (pair) tma_load_2d_pair(sw, rank ? tmb : tma, bar, kc, f0);
+      else tma_load_2d_pair(sw, tma, bar, kc, f0 + static_cast<int>(rank) * W_ROWS);
+    } else if (pair) {
       tma_load_2d(sw, tma, &full_bar[i % STAGES], kc, f0);
       tma_load_2d(sw + W_BYTES / 2, tmb, &full_bar[i % STAGES], kc, f0);
     } else {
       tma_load_2d(sw, tma, &full_bar[i % STAGES], kc, f0);
     }
   };
+  // the even CTA expects both CTAs' bytes of a stage
+  auto expect = [&](int s) {
+    if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], TWO ? 2 * STAGE : STAGE);
+  };
 
   if (warp == 0 && lane == 0) {
     const int npre = min(STAGES, nkb);
     for (int i = 0; i < npre; ++i) {
-      mbar_arrive_expect_tx(&full_bar[i], STAGE);
+      expect(i);
       load_w(i, smem + i * STAGE + X_BYTES);
     }
     pdl_wait();
-    for (int i = 0; i < npre; ++i)
-      tma_load_2d(smem + i * STAGE, &p.tm_x, &full_bar[i], (kb0 + i) * BK, tok0);
+    for (int i = 0; i < npre; ++i) load_x(i, smem + i * STAGE);
     int issued = npre;
     for (int i = npre; i < nkb; ++i) {
       const int s = i % STAGES;
@@ -538,16 +601,16 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
       }
       if (abort_flag) break;
       uint8_t* sa = smem + s * STAGE;
-      mbar_arrive_expect_tx(&full_bar[s], STAGE);
+      expect(s);
       load_w(i, sa + X_BYTES);
-      tma_load_2d(sa, &p.tm_x, &full_bar[s], (kb0 + i) * BK, tok0);
+      load_x(i, sa);
       ++issued;
     }
-    if (abort_flag) {
+    if (abort_flag && rank == 0) {
       for (int i = max(0, issued - STAGES); i < issued; ++i)
         mbar_wait(&full_bar[i % STAGES], (i / STAGES) & 1, p.status, 32);
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0 && rank == 0) {
     for (int i = 0; i < nkb; ++i) {
       const int s = i % STAGES;
       if (!mbar_wait(&full_bar[s], (i / STAGES) & 1, p.status, 33)) {
@@ -560,11 +623,15 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
       const uint64_t da = smem_desc_sw128(sa);
       const uint64_t db = smem_desc_sw128(sa + X_BYTES);
 #pragma unroll
-      for (int k = 0; k < BK / UK; ++k)
-        tc_mma_bf16(tmem, da + 2 * k, db + 2 * k, IDESC, (i > 0 || k > 0) ? 1u : 0u);
-      tc_commit(&empty_bar[s]);
+      for (int k = 0; k < BK / UK; ++k) {
+        if constexpr (TWO) tc_mma_bf16_pair(tmem, da + 2 * k, db + 2 * k, IDESC, (i > 0 || k > 0) ? 1u : 0u);
+        else tc_mma_bf16(tmem, da + 2 * k, db + 2 * k, IDESC, (i > 0 || k > 0) ? 1u : 0u);
+      }
+      if constexpr (TWO) tc_commit_pair(&empty_bar[s]);
+      else tc_commit(&empty_bar[s]);
     }
-    tc_commit(&acc_bar);
+    if constexpr (TWO) tc_commit_pair(&acc_bar);
+    else tc_commit(&acc_bar);
   }
   __syncwarp();
 
@@ -740,9 +807,19 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (TWO) {
+    // after a timed-out wait, give copies that the other CTA issued against
+    // this CTA's barriers time to land (bounded) before the pair tears down
+    if (abort_flag) {
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 200000ull) __nanosleep(1000);
+    }
+    cluster_sync_all();   // neither CTA frees TMEM or exits while the other works
+  }
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    if constexpr (TWO) tmem_dealloc_pair(tmem, TMEM_COLS);
+    else tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -858,11 +935,13 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
           at_tile(c);
         }
       };
+      const uint64_t pol = policy_evict_first();   // weights are read once
       auto load_w = [&](const Cursor& c, int s, uint8_t* sa) {
         const Seg& S = p.seg[c.sg];
         const int kc = c.k * BK;
-        tma_load_2d(sa, &p.tm[S.map], &full_bar[s], kc, c.row0);
-        if (S.pair) tma_load_2d(sa + A_BYTES / 2, &p.tm[S.map + 1], &full_bar[s], kc, c.row0);
+        tma_load_2d_hint(sa, &p.tm[S.map], &full_bar[s], kc, c.row0, pol);
+        if (S.pair)
+          tma_load_2d_hint(sa + A_BYTES / 2, &p.tm[S.map + 1], &full_bar[s], kc, c.row0, pol);
       };
       auto load_x = [&](const Cursor& c, int s, uint8_t* sa) {
         tma_load_2d(sa + A_BYTES, &p.tm_x, &full_bar[s], c.k * BK, c.tok0);
@@ -1232,6 +1311,38 @@ cudaError_t launch_tok(const Params& p, dim3 grid, cudaStream_t st) {
   return launch_k(gemm_tok_kernel<BW, STAGES, ARGMAX>, grid, dim3(128), SMEM, st, p);
 }
 
+// CTA-pair token-major launch: 256-feature tiles, a 6-stage ring of 32 KB
+// stages, a 1-D grid of (feature tiles x even token tiles) CTAs in clusters
+// of two.
+template <bool ARGMAX>
+cudaError_t launch_tok2(const Params& p, dim3 grid, cudaStream_t st) {
+  constexpr int STAGES = 6;
+  constexpr int SMEM = STAGES * (BM * BK * 2 + 128 * BK * 2) + 1024;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_tok_kernel<256, STAGES, ARGMAX, true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, gemm_tok_kernel<256, STAGES, ARGMAX, true>, p);
+}
+
 // Token tiles on grid x when there are fewer of them than feature tiles (and
 // the feature tiles fit grid y): the weights then stream from HBM once.
 inline bool tok_fast(int tok_tiles, int feature_tiles) {
@@ -1522,6 +1633,8 @@ GemmPlan plan_gemm(const GemmJob& job) {
       }
       const int tiles = pl.row_tiles * pl.tok_tiles;
       if (tiles * 2 < kNumSMs) splits = std::min(kb_total, kNumSMs / tiles);
+      // pairs of token tiles share each weight tile's shared-memory traffic
+      pl.two = pl.bn == 256 && splits == 1 && pl.tok_tiles >= 2;
     } else {
       // weight-major (swap-AB): 128 weight rows x BN tokens per tile, split K
       // so about two CTAs per SM stream at once and all fit in one wave
@@ -1631,7 +1744,13 @@ cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& pl, float* partial,
     // rows of one weight box: the tile's feature count (half of it per
     // matrix for a SwiGLU pair)
     const int per_tile = pl.tok_major ? pl.bn : tc::BM;
-    if (S.pair) {
+    if (pl.two) {
+      // each CTA of a pair stages 128 rows: half a tile, or one SwiGLU half
+      if (!encode_tmap_bf16_2d(&p.tm[maps++], o.w0, job.K, o.rows, tc::BK, 128) ||
+          (S.pair && !encode_tmap_bf16_2d(&p.tm[maps++], o.w1, job.K, o.rows, tc::BK, 128)))
+        return cudaErrorInvalidValue;
+      tiles += S.pair ? ceil_div(o.rows, 128) : ceil_div(o.rows, 256);
+    } else if (S.pair) {
       if (!encode_tmap_bf16_2d(&p.tm[maps++], o.w0, job.K, o.rows, tc::BK, per_tile / 2) ||
           !encode_tmap_bf16_2d(&p.tm[maps++], o.w1, job.K, o.rows, tc::BK, per_tile / 2))
         return cudaErrorInvalidValue;
@@ -1671,6 +1790,10 @@ cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& pl, float* partial,
   dim3 grid(tiles, pl.tok_tiles, pl.splits);
   if (pl.tok_major) {
     p.tok_fast = tc::tok_fast(pl.tok_tiles, tiles);
+    if (pl.two) {
+      const int tt = (pl.tok_tiles + 1) & ~1;   // whole pairs; a spare tile is all padding
+      return tc::launch_tok2<false>(p, dim3(static_cast<unsigned>(tiles) * tt), st);
+    }
     if (p.tok_fast) grid = dim3(pl.tok_tiles, tiles, pl.splits);
     return tc::dispatch_tok<false>(pl.bn, p, grid, st);
   }
@@ -1709,7 +1832,10 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X,
   if (dtype == DFLASH_BF16 && M >= tc::kTokMajorMin) {
     tc::Params p{};
     constexpr int BW = 256;
-    if (!encode_tmap_bf16_2d(&p.tm[0], W, K, V, tc::BK, BW)) return cudaErrorInvalidValue;
+    const int tt = ceil_div(M, tc::BM);
+    const bool two = tt >= 2;   // CTA pairs over consecutive token tiles
+    if (!encode_tmap_bf16_2d(&p.tm[0], W, K, V, tc::BK, two ? BW / 2 : BW))
+      return cudaErrorInvalidValue;
     if (!encode_tmap_bf16_2d(&p.tm_x, X, K, M, tc::BK, tc::BM)) return cudaErrorInvalidValue;
     p.seg[0].rows = V;
     p.nseg = 1;
@@ -1721,8 +1847,11 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X,
     p.keys = keys;
     p.lse = lse;
     p.status = status;
-    const int tt = ceil_div(M, tc::BM);
     p.tok_fast = tc::tok_fast(tt, p.row_tiles);
+    if (two) {
+      const int te = (tt + 1) & ~1;
+      return tc::launch_tok2<true>(p, dim3(static_cast<unsigned>(p.row_tiles) * te), st);
+    }
     const dim3 grid = p.tok_fast ? dim3(tt, p.row_tiles, 1) : dim3(p.row_tiles, tt, 1);
     return tc::dispatch_tok<true>(BW, p, grid, st);
   }

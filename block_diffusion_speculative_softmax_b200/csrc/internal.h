@@ -64,6 +64,7 @@ struct GemmPlan {
   int bn;            // token tile (weight-major) or feature tile (token-major)
   int row_tiles;     // tiles along the output features (all segments)
   int tok_tiles;
+  int two;           // token-major on CTA pairs (cta_group::2, 256-feature tiles)
   int splits;        // K splits
   int kb_per_split;  // k-blocks per split
   size_t partial_floats;

@@ -71,8 +71,11 @@ def test_fuse_ctx_zero_rows_is_noop(DF):
 
 # ------------------------------------------------------------------ K/V projection
 @pytest.mark.parametrize("dtype,M,scatter", [("fp32", 8, False), ("bf16", 16, False),
-                                             ("bf16", 37, True), ("bf16", 700, False)])
+                                             ("bf16", 37, True), ("bf16", 700, False),
+                                             ("bf16", 4700, True)])
 def test_kv_project(DF, dtype, M, scatter):
+    # M = 4700: 37 token tiles (odd) x 2 feature tiles runs on CTA pairs with
+    # a padding tile; 700: token-major single CTAs with split K; <= 64: weight-major
     cfg = _cfg(dtype, hidden=576 if dtype == "bf16" else 256,
                n_kv_heads=2, head_dim=128 if dtype == "bf16" else 64)
     rng = np.random.default_rng(M)
