@@ -37,7 +37,9 @@ ACCEPT_DRAWS = 32          # planted target draws averaged for accepted tok/s
 # DRAM bytes (read + write) of one LM-head launch from an ncu capture of
 # `bench.py --op lmhead` (summarised under profiles/), valid only for the
 # GEMM source it was taken with; any later edit of gemm.cu nulls it.
-LMHEAD_TRAFFIC = {}        # workload -> {"bytes": int, "gemm_cu_sha256": str}
+LMHEAD_TRAFFIC = {         # workload -> {"bytes": int, "gemm_cu_sha256": str}
+    "qwen3_4b": {"bytes": 785283584, "gemm_cu_sha256": "ae62e314da1656b0"},
+}
 
 
 def parse():

@@ -107,6 +107,24 @@ __device__ __forceinline__ float2 rope_cs(const Params& p, int pos, int fi) {
   return make_float2(cs, sn);
 }
 
+// (cos, sin) of frequencies i0 .. i0 + 15 at `pos`: eight 16-byte table loads
+// when the table covers the position (i0 is a multiple of 16).
+__device__ __forceinline__ void rope_cs16(const Params& p, int pos, int i0, float2* cs) {
+  if (p.rope_tab != nullptr && pos < p.rope_len) {
+    const float4* t = reinterpret_cast<const float4*>(
+        p.rope_tab + static_cast<size_t>(pos) * (p.head_dim >> 1) + i0);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 v = __ldg(t + q);
+      cs[2 * q] = make_float2(v.x, v.y);
+      cs[2 * q + 1] = make_float2(v.z, v.w);
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 16; ++q) cs[q] = rope_cs(p, pos, i0 + q);
+  }
+}
+
 template <int BN, int STAGES, bool ARGMAX>
 __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Params p) {
   constexpr int B_BYTES = BN * BK * 2;
@@ -774,24 +792,28 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
         }
       };
       if (S.rope) {
-        // chunk c of the first half of a head pairs with chunk c + d/2
+        // 16 frequencies at a time: one (cos, sin) set serves that chunk of
+        // every head in the tile; chunk c of a head's first half pairs with
+        // chunk c + d/2
 #pragma unroll 1
-        for (int c = 0; c < BW; c += 16) {
-          const int i = c % d;
-          if (i >= half) continue;
-          float a[16], b[16];
-          cols(c, a);
-          cols(c + half, b);
-          if (tv) {
+        for (int i0 = 0; i0 < half; i0 += 16) {
+          float2 cs[16];
+          if (tv) rope_cs16(p, pos, i0, cs);
+#pragma unroll 1
+          for (int c = i0; c < BW; c += d) {
+            float a[16], b[16];
+            cols(c, a);
+            cols(c + half, b);
+            if (tv) {
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const float2 cs = rope_cs(p, pos, i + q);
-              const float x1 = a[q], x2 = b[q];
-              a[q] = x1 * cs.x - x2 * cs.y;
-              b[q] = x2 * cs.x + x1 * cs.y;
+              for (int q = 0; q < 16; ++q) {
+                const float x1 = a[q], x2 = b[q];
+                a[q] = x1 * cs[q].x - x2 * cs[q].y;
+                b[q] = x2 * cs[q].x + x1 * cs[q].y;
+              }
+              put16(f0 + c, a);
+              put16(f0 + c + half, b);
             }
-            put16(f0 + c, a);
-            put16(f0 + c + half, b);
           }
         }
       } else {
