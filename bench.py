@@ -330,6 +330,8 @@ def run_ours(args):
     tok_per_step = float(np.mean(tok_draws))
     value = blocks_per_step * world / (ms / 1e3)
     acc_tok_s = tok_per_step * world / (ms / 1e3)
+    # accepted draft tokens only (sum of n, without the bonus token)
+    acc_draft_tok_s = (tok_per_step - wl.R) * world / (ms / 1e3)
 
     # ---- roofline of the dominant kernel, timed alone on its own stream
     roof = roofline(args, wl, cfg, DF, hbm_peak, tf_burst, peak_src, stream)
@@ -352,7 +354,8 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if cfg.dtype == "bf16" else "fp32", "data": "synthetic",
-            "accepted_tok_s": acc_tok_s, "mean_accept_tau": tok_per_step / wl.R,
+            "accepted_tok_s": acc_tok_s, "accepted_draft_tok_s": acc_draft_tok_s,
+            "mean_accept_tau": tok_per_step / wl.R,
             "accept_draws": len(tok_draws),
             "config": {"workload": cfg.name, "mode": args.mode, "n_req": cfg.n_req,
                        "blocks_per_step": blocks_per_step, "block": cfg.block,

@@ -19,7 +19,10 @@ pages give.  Sources (web summaries of three papers):
 * "DFLARE: scaling draft capacity of block-diffusion speculative decoding"
   -- section 2.1 (per-layer softmax fusion alpha^(i) = softmax(W_fuse[i]),
   weighted sum of T target layers, then RMSNorm) and section 2.2 (separate
-  K/V projections W^t for the target context and W^d for the draft block).
+  K/V projections W^t for the target context and W^d for the draft block);
+  section 1 item 1 and section 2.2 also describe the DFlash baseline (one
+  FC-fused context shared by all draft layers, context and block sharing
+  the K/V projections), available here as a variant (``fc_fuse_ctx``).
 
 Readings where the pages are silent (kept identical in the CUDA path):
 RMSNorm y = x / sqrt(mean(x^2) + eps) * g with a learned gain g; rotate-half
@@ -108,6 +111,24 @@ def fuse_ctx(states: np.ndarray, w_fuse: np.ndarray, g_fuse: np.ndarray,
             u += alpha[i, j] * s[:, j, :]
         out[i] = _store(rmsnorm(u, g_fuse[i], eps), bf16_storage)
     return out
+
+
+def fc_fuse_ctx(states: np.ndarray, w_fc: np.ndarray, g_fc: np.ndarray,
+                eps: float, bf16_storage: bool = False) -> np.ndarray:
+    """DFlash-style context fusion (DFLARE summary, section 1 item 1 and
+    section 2.2, describing the DFlash baseline): one fully connected layer
+    maps the T concatenated target hidden states of a row to a single shared
+    representation that every draft layer receives.
+
+    states [N][T][H], w_fc [H][T*H] (nn.Linear layout over the concatenation
+    h_1 | h_2 | ... | h_T), g_fc [H].  The pages do not say whether the FC
+    output is normalised; it is read here as RMSNorm_{g_fc}(concat(h) W_fc^T),
+    the same normalisation the per-layer fusion applies, so both variants
+    hand the K/V projections vectors of the same scale.  Returns [N][H]."""
+    s = _f64(states)
+    N, T, H = s.shape
+    u = s.reshape(N, T * H) @ _f64(w_fc).T
+    return _store(rmsnorm(u, g_fc, eps), bf16_storage)
 
 
 def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
@@ -289,13 +310,22 @@ class Block:
 
 
 def _ctx_kv(cfg, weights, states, bf16_storage):
-    """Per draft layer context K/V of one request: fuse all T target layers
-    with that layer's own alpha, RMSNorm, then W^t projections."""
+    """Per draft layer context K/V of one request.
+
+    DFLARE (default): fuse all T target layers with that layer's own alpha,
+    RMSNorm, then that layer's W^t projections.  DFlash variant (weights
+    carry "w_fc"): one FC-fused context shared by every layer, projected by
+    each layer's W^t -- which the DFlash baseline shares with the block's
+    W^d (pass weights with w_kt = w_kd and w_vt = w_vd for that)."""
     eps, theta = cfg.rms_eps, cfg.rope_theta
     lays = weights["layers"]
-    g_fuse = np.stack([_f64(l["g_fuse"]) for l in lays])
     L = states.shape[0]
-    fused = fuse_ctx(states, weights["w_fuse"], g_fuse, eps, bf16_storage)
+    if "w_fc" in weights:
+        c = fc_fuse_ctx(states, weights["w_fc"], weights["g_fc"], eps, bf16_storage)
+        fused = [c] * len(lays)
+    else:
+        g_fuse = np.stack([_f64(l["g_fuse"]) for l in lays])
+        fused = fuse_ctx(states, weights["w_fuse"], g_fuse, eps, bf16_storage)
     pos = np.arange(L, dtype=np.float64)
     kv = []
     for i, lay in enumerate(lays):

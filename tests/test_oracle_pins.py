@@ -407,6 +407,65 @@ def test_shared_kv_weights_equal_heterogeneous_with_equal_matrices():
     np.testing.assert_array_equal(m_a, m_b)
 
 
+# ------------------------------------------------ DFlash FC-fusion variant
+
+def test_fc_fusion_single_layer_identity_is_rmsnorm():
+    # T = 1 and W_fc = I: the shared context is RMSNorm of the one target layer
+    rng = np.random.default_rng(21)
+    H = 24
+    st = rng.standard_normal((7, 1, H))
+    g = 1 + 0.1 * rng.standard_normal(H)
+    got = O.fc_fuse_ctx(st, np.eye(H), g, 1e-6)
+    want = F.rms_norm(_t(st[:, 0]), (H,), weight=_t(g), eps=1e-6).numpy()
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_fc_fusion_reproduces_softmax_fusion_with_stacked_identities():
+    # W_fc = [a_1 I | ... | a_T I] with a = softmax(w) is the weighted sum of
+    # the per-layer fusion; with the same gain both give the same context
+    rng = np.random.default_rng(22)
+    N, T, H = 6, 4, 16
+    st = rng.standard_normal((N, T, H))
+    w = rng.standard_normal(T)
+    a = np.exp(w - w.max()) / np.exp(w - w.max()).sum()
+    w_fc = np.concatenate([a[j] * np.eye(H) for j in range(T)], axis=1)   # [H][T*H]
+    g = 1 + 0.1 * rng.standard_normal(H)
+    got = O.fc_fuse_ctx(st, w_fc, g, 1e-6)
+    want = O.fuse_ctx(st, w[None, :], g[None, :], 1e-6)[0]
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-13)
+    # a general W_fc is the concatenation times W_fc^T, then RMSNorm
+    w_r = rng.standard_normal((H, T * H))
+    u = st.reshape(N, T * H) @ w_r.T
+    want_r = F.rms_norm(_t(u), (H,), weight=_t(g), eps=1e-6).numpy()
+    np.testing.assert_allclose(O.fc_fuse_ctx(st, w_r, g, 1e-6), want_r, rtol=1e-12)
+
+
+def test_dflash_variant_draft_step_equals_dflare_with_tied_fusion_and_kv():
+    # The DFlash variant (one FC-fused context for all layers, context K/V
+    # through the block's own W^d) must equal the DFLARE step when every
+    # layer's alpha row and gain are the same, W^t = W^d, and W_fc stacks
+    # alpha-scaled identities.
+    cfg = _tiny_cfg()
+    w = synth.make_weights(cfg, seed=6, separate_kv=False)
+    T, H = cfg.n_target_layers, cfg.hidden
+    row = w["w_fuse"][0].astype(np.float64)
+    g = w["layers"][0]["g_fuse"].astype(np.float64)
+    w_dflare = dict(w, w_fuse=np.tile(row, (cfg.n_draft_layers, 1)),
+                    layers=[dict(l, g_fuse=g) for l in w["layers"]])
+    a = np.exp(row - row.max()) / np.exp(row - row.max()).sum()
+    w_dflash = dict(w, w_fc=np.concatenate([a[j] * np.eye(H) for j in range(T)], axis=1),
+                    g_fc=g)
+    st = [synth.make_states(cfg, 6, 0, 8)]
+    blk = [O.Block(0, [9, 0, 0, 0, 0], 1), O.Block(0, [9, 2, 0, 0, 0], 2)]
+    t_a, m_a = O.draft_step(cfg, w_dflare, st, blk)
+    t_b, m_b = O.draft_step(cfg, w_dflash, st, blk)
+    np.testing.assert_array_equal(t_a, t_b)
+    np.testing.assert_allclose(m_a, m_b, rtol=1e-12)
+    # and it genuinely differs once the layers' fusions differ
+    t_c, m_c = O.draft_step(cfg, dict(w_dflare, w_fuse=w["w_fuse"]), st, blk)
+    assert not np.allclose(m_a, m_c)
+
+
 # ---------------------------------------------------------------- losslessness
 
 def speculative_decode(tw, cfg, dw, prompt, n_new, draft_fn, accept_fn, rng,
