@@ -36,9 +36,10 @@ METRIC = "draft blocks/s and accepted tok/s per B200; HBM GB/s / tensor util vs 
 ACCEPT_DRAWS = 32          # planted target draws averaged for accepted tok/s
 # DRAM bytes (read + write) of one LM-head launch from an ncu capture of
 # `bench.py --op lmhead` (summarised under profiles/), valid only for the
-# GEMM source it was taken with; any later edit of gemm.cu nulls it.
+# GEMM code it was taken with (digest of gemm.cu without comments); any
+# later change of that code nulls it.
 LMHEAD_TRAFFIC = {         # workload -> {"bytes": int, "gemm_cu_sha256": str}
-    "qwen3_4b": {"bytes": 785283584, "gemm_cu_sha256": "ae62e314da1656b0"},
+    "qwen3_4b": {"bytes": 785283584, "gemm_cu_sha256": "c631e555a25cd81b"},
 }
 
 
@@ -380,17 +381,29 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def code_digest(text):
+    """sha256 of C/C++ source with comments removed and whitespace collapsed,
+    so only a change of the code itself changes it."""
+    import hashlib
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()
+
+
+def gemm_source_digest():
+    src = os.path.join(ROOT, "block_diffusion_speculative_softmax_b200", "csrc", "gemm.cu")
+    with open(src) as f:
+        return code_digest(f.read())
+
+
 def lmhead_traffic(workload):
     """Measured DRAM bytes per LM-head launch, or None when there is no
-    capture for this workload or the GEMM source changed since."""
-    import hashlib
+    capture for this workload or the GEMM code changed since."""
     ent = LMHEAD_TRAFFIC.get(workload)
     if ent is None:
         return None
-    src = os.path.join(ROOT, "block_diffusion_speculative_softmax_b200", "csrc", "gemm.cu")
-    with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()
-    return ent["bytes"] if digest.startswith(ent["gemm_cu_sha256"]) else None
+    return ent["bytes"] if gemm_source_digest().startswith(ent["gemm_cu_sha256"]) else None
 
 
 def roofline(args, wl, cfg, DF, hbm_peak, tf_burst, peak_src, stream):

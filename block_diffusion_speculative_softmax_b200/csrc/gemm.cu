@@ -33,6 +33,14 @@
 // with one 64-bit atomicMax, so logits never reach global memory.  fp32
 // models run on a SIMT FFMA kernel (partials + finish kernel): tensor-core
 // tf32 would miss a 1e-4 tolerance.
+//
+// Three bf16 kernels share this structure:
+//   gemm_kernel     weight-major split-K (above), block GEMMs with <= 64 tokens;
+//   gemm_sk_kernel  weight-major stream-K: a persistent grid whose CTAs take
+//                   equal shares of the (tile, k-block) units, used for the
+//                   LM head with <= 64 tokens;
+//   gemm_tok_kernel token-major (tokens on M, features on N) for >= 65 tokens,
+//                   on CTA pairs (cta_group::2) when tiles are plentiful.
 #include <algorithm>
 #include <cstdlib>
 #include <cmath>

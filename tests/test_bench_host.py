@@ -106,3 +106,13 @@ def test_every_python_module_compiles():
     for f in files:
         with open(f) as fh:
             compile(fh.read(), f, "exec")
+
+
+def test_traffic_digest_ignores_comments_but_not_code():
+    base = "int f(int a) {\n  return a + 1;  // one\n}\n/* block */\n"
+    assert bench.code_digest(base) == bench.code_digest(base.replace("// one", "// two"))
+    assert bench.code_digest(base) == bench.code_digest(base.replace("/* block */", ""))
+    assert bench.code_digest(base) != bench.code_digest(base.replace("a + 1", "a + 2"))
+    # the recorded LM-head traffic belongs to the GEMM code in this tree
+    for ent in bench.LMHEAD_TRAFFIC.values():
+        assert bench.gemm_source_digest().startswith(ent["gemm_cu_sha256"])
