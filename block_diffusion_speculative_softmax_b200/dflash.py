@@ -4,6 +4,27 @@ Argument marshalling only: every step of the draft pass runs in the CUDA
 kernels behind the C ABI declared in include/dflash.h.  PyTorch provides
 device memory and streams.  There is no fallback: if the library cannot be
 loaded, every call raises.
+
+Typical use (one draft step + verification per decoding step)::
+
+    from block_diffusion_speculative_softmax_b200 import build, dflash as DF
+    build.build()                                   # compiles libdflash.so once
+    cfg = DF.make_config(hidden=2560, n_q_heads=32, n_kv_heads=8, head_dim=128,
+                         ffn=9728, n_draft_layers=5, n_target_layers=5, block=16,
+                         vocab=151936)              # bf16, mask id V-1, theta 1e6
+    w = DF.DeviceWeights(cfg, host_weights)         # dict of numpy arrays, see synth.make_weights
+    buf = DF.StepBuffers(cfg, ctx_lens, n_blocks)   # KV caches, block and output buffers
+    ws = DF.alloc_workspace(DF.dflash_workspace_size(cfg, len(ctx_lens), n_blocks,
+                                                     n_ctx_new, max(ctx_lens)))
+    # fill buf.block_tokens (anchor in slot 0), buf.block_req, buf.known_len,
+    # and buf.target_tokens with the target's argmax tokens; new_states holds
+    # the target states [n_ctx_new][T][H] of the context rows to (re)fuse:
+    DF.dflash_draft_step(cfg, w, buf, new_states, ws, verify=True)
+    DF.dflash_check(ws)                              # device-side errors, if any
+    # buf.draft_tokens, buf.n_acc, buf.best_k and buf.out_tok hold the result
+
+``block_diffusion_speculative_softmax_b200.workload.Workload`` builds all of
+this from the seeded synthetic inputs of a named configuration.
 """
 from __future__ import annotations
 
