@@ -88,6 +88,15 @@ dflash_status check_config(const dflash_config* c) {
     if (!aligned16(p)) return fail(DFLASH_EINVAL, "%s is not 16-byte aligned", name); \
   } while (0)
 
+// Index and per-token arrays (int32 / fp32 / int64, nullable): naturally
+// aligned, so a misaligned pointer is refused on the host and never reaches
+// a kernel.
+#define DFL_ALIGNED(p, n, name)                                                  \
+  do {                                                                           \
+    if ((p) != nullptr && (reinterpret_cast<uintptr_t>(p) % (n)) != 0)           \
+      return fail(DFLASH_EINVAL, "%s is not %d-byte aligned", name, n);          \
+  } while (0)
+
 // ------------------------------------------------------------------ jobs
 GemmJob job_base(const dflash_config* c, const void* x, int64_t M, int K) {
   GemmJob j;
@@ -350,6 +359,8 @@ dflash_status dflash_kv_project(const dflash_config* cfg, const void* x, int64_t
   DFL_PTR(k_out, "k_out");
   DFL_PTR(v_out, "v_out");
   DFL_CHECK(pos != nullptr, DFLASH_EINVAL, "pos is NULL");
+  DFL_ALIGNED(pos, 4, "pos");
+  DFL_ALIGNED(dst_row, 8, "dst_row");
   const GemmJob j = job_kv(cfg, x, M, pos, dst_row, w_k, w_v, k_out, v_out);
   const GemmPlan pl = plan_gemm(j);
   const size_t off_cnt = align256(sizeof(DevStatus) + pl.partial_floats * 4);
@@ -378,6 +389,8 @@ dflash_status dflash_block_attn(const dflash_config* cfg, int32_t n_blocks, cons
   DFL_PTR(out, "out");
   DFL_CHECK(ctx_off != nullptr && block_req != nullptr, DFLASH_EINVAL,
             "ctx_off / block_req is NULL");
+  DFL_ALIGNED(ctx_off, 8, "ctx_off");
+  DFL_ALIGNED(block_req, 4, "block_req");
   if (max_ctx_len > 0) {
     DFL_PTR(k_ctx, "k_ctx");
     DFL_PTR(v_ctx, "v_ctx");
@@ -440,6 +453,9 @@ dflash_status dflash_lmhead_argmax(const dflash_config* cfg, int64_t M, const vo
   DFL_PTR(x, "x");
   DFL_PTR(w_lm, "w_lm");
   DFL_CHECK(tok != nullptr, DFLASH_EINVAL, "tok is NULL");
+  DFL_ALIGNED(tok, 4, "tok");
+  DFL_ALIGNED(max_logit, 4, "max_logit");
+  DFL_ALIGNED(conf, 4, "conf");
   const GemmPlan pl = plan_lmhead(cfg->dtype, cfg->vocab, M, cfg->hidden);
   const size_t off_keys = sizeof(DevStatus);
   const size_t off_cnt = align256(off_keys + M * 8);
@@ -473,6 +489,11 @@ dflash_status dflash_accept(int32_t R, int32_t K, int32_t B, const int32_t* draf
   if (R == 0) return DFLASH_OK;
   DFL_CHECK(draft && target && n_acc && best_k && out_tok, DFLASH_EINVAL,
             "a pointer argument is NULL");
+  DFL_ALIGNED(draft, 4, "draft");
+  DFL_ALIGNED(target, 4, "target");
+  DFL_ALIGNED(n_acc, 4, "n_acc");
+  DFL_ALIGNED(best_k, 4, "best_k");
+  DFL_ALIGNED(out_tok, 4, "out_tok");
   DFL_CUDA(launch_accept(R, K, B, draft, target, n_acc, best_k, out_tok,
                          static_cast<cudaStream_t>(stream)),
            "accept kernel");
@@ -489,6 +510,11 @@ dflash_status dflash_d2sd_candidates(int32_t R, int32_t B, int32_t K, int32_t ma
   if (R == 0) return DFLASH_OK;
   DFL_CHECK(base_tokens && conf && known_len && cand_tokens, DFLASH_EINVAL,
             "a pointer argument is NULL");
+  DFL_ALIGNED(base_tokens, 4, "base_tokens");
+  DFL_ALIGNED(conf, 4, "conf");
+  DFL_ALIGNED(known_len, 4, "known_len");
+  DFL_ALIGNED(cand_tokens, 4, "cand_tokens");
+  DFL_ALIGNED(block_req, 4, "block_req");
   DFL_CUDA(launch_d2sd(R, B, K, mask_token_id, base_tokens, conf, known_len, cand_tokens,
                        block_req, static_cast<cudaStream_t>(stream)),
            "D2SD cut kernel");
@@ -519,6 +545,19 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
   DFL_CHECK(a->block_req && a->block_tokens && a->ctx_off && a->draft_tokens, DFLASH_EINVAL,
             "block_req / block_tokens / ctx_off / draft_tokens is NULL");
   DFL_CHECK(a->k_cache && a->v_cache, DFLASH_EINVAL, "k_cache / v_cache is NULL");
+  DFL_ALIGNED(a->block_req, 4, "block_req");
+  DFL_ALIGNED(a->block_tokens, 4, "block_tokens");
+  DFL_ALIGNED(a->known_len, 4, "known_len");
+  DFL_ALIGNED(a->ctx_off, 8, "ctx_off");
+  DFL_ALIGNED(a->new_off, 8, "new_off");
+  DFL_ALIGNED(a->ctx_cached, 4, "ctx_cached");
+  DFL_ALIGNED(a->draft_tokens, 4, "draft_tokens");
+  DFL_ALIGNED(a->max_logit, 4, "max_logit");
+  DFL_ALIGNED(a->confidence, 4, "confidence");
+  DFL_ALIGNED(a->target_tokens, 4, "target_tokens");
+  DFL_ALIGNED(a->n_acc, 4, "n_acc");
+  DFL_ALIGNED(a->best_k, 4, "best_k");
+  DFL_ALIGNED(a->out_tok, 4, "out_tok");
   if (a->n_ctx_new > 0) DFL_PTR(a->new_states, "new_states");
   DFL_CHECK(w->w_fuse && w->layers, DFLASH_EINVAL, "w_fuse / layers is NULL");
   DFL_PTR(w->embed, "embed");
@@ -712,6 +751,8 @@ extern "C" dflash_status dflash_lmhead_argmax_noalloc(const dflash_config* cfg, 
   DFL_PTR(x, "x");
   DFL_PTR(w_lm, "w_lm");
   DFL_CHECK(tok != nullptr, DFLASH_EINVAL, "tok is NULL");
+  DFL_ALIGNED(tok, 4, "tok");
+  DFL_ALIGNED(max_logit, 4, "max_logit");
   unsigned long long* keys = nullptr;
   if ((s = noalloc_scratch(&keys)) != DFLASH_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

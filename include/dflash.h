@@ -37,8 +37,11 @@
  *     dflash_check() synchronises the stream and returns them.
  *   - Calls are stateless and thread-safe as long as concurrent calls use
  *     different workspaces.
- *   - Device pointers must be 16-byte aligned; hidden, ffn and head_dim
- *     must be multiples of 8 (bf16) or 4 (fp32).
+ *   - Weight, activation, state and cache pointers must be 16-byte aligned;
+ *     token, index and per-token arrays (int32, fp32, int64) must be
+ *     naturally aligned (4 or 8 bytes); hidden, ffn and head_dim must be
+ *     multiples of 8 (bf16) or 4 (fp32).  A misaligned pointer is refused
+ *     with DFLASH_EINVAL before any launch.
  */
 #ifndef DFLASH_H_
 #define DFLASH_H_

@@ -115,3 +115,31 @@ def test_draft_step_argument_checks(lib):
                                None)
     assert st == DF.EINVAL
     assert DF.dflash_launch_count() == 0
+
+
+def test_misaligned_index_and_output_pointers_rejected(lib):
+    """int32 / fp32 / int64 arrays must be naturally aligned; a misaligned
+    one is refused on the host (it would fault a kernel)."""
+    cfg = _cfg()
+    odd = C.c_void_p(258)     # 2 mod 4
+    ok = C.c_void_p(256)
+    st = lib.dflash_lmhead_argmax(C.byref(cfg), 4, ok, ok, odd, None, None, ok, 1 << 30, None)
+    assert st == DF.EINVAL and b"tok is not 4-byte aligned" in lib.dflash_last_error()
+    st = lib.dflash_lmhead_argmax(C.byref(cfg), 4, ok, ok, ok, None, odd, ok, 1 << 30, None)
+    assert st == DF.EINVAL and b"conf is not 4-byte aligned" in lib.dflash_last_error()
+    assert lib.dflash_accept(1, 1, 8, ok, ok, ok, ok, odd, None) == DF.EINVAL
+    assert b"out_tok" in lib.dflash_last_error()
+    assert lib.dflash_d2sd_candidates(1, 16, 4, 5, ok, odd, ok, ok, None, None) == DF.EINVAL
+    st = lib.dflash_kv_project(C.byref(cfg), ok, 4, ok, C.c_void_p(260), ok, ok, ok, ok, ok,
+                               1 << 30, None)
+    assert st == DF.EINVAL and b"dst_row is not 8-byte aligned" in lib.dflash_last_error()
+    w = DF.Weights()
+    a = DF.StepArgs()
+    a.n_req, a.n_blocks = 1, 1
+    a.block_req, a.block_tokens, a.ctx_off, a.draft_tokens = 256, 256, 260, 256
+    kc = (C.c_void_p * 16)(*([256] * 16))
+    a.k_cache = kc
+    a.v_cache = kc
+    st = lib.dflash_draft_step(C.byref(cfg), C.byref(w), C.byref(a), ok, 1 << 30, None)
+    assert st == DF.EINVAL and b"ctx_off is not 8-byte aligned" in lib.dflash_last_error()
+    assert DF.dflash_launch_count() == 0
