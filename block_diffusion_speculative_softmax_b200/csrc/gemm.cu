@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
   if (tid == 0) pdl_launch();
 
   // weights are read once per step: evict them first so L2 keeps what is
-  // reused (activations, K/V, prefetched weights of the next GEMM)
+  // reused (activations, partial tiles, the K/V caches)
   const uint64_t pol = policy_evict_first();
   auto load_w = [&](int i, uint8_t* sa) {
     const int kc = (kb0 + i) * BK;
