@@ -533,3 +533,112 @@ def test_draft_confidence_is_top1_softmax_probability():
     assert abs(O.draft_confidence(big)[0] - 1.0) < 1e-15
     # invariant to a constant shift of all logits
     np.testing.assert_allclose(O.draft_confidence(z + 123.0), O.draft_confidence(z), rtol=1e-12)
+
+
+# ------------------------------------------- composed step, restated in torch
+
+def _rope_complex(x, pos, theta):
+    """Rotate-half RoPE written as a complex rotation: the pair
+    (x_i, x_{i+d/2}) is the complex number x_i + i x_{i+d/2}, turned by the
+    angle pos * theta^(-2i/d).  x [M][heads][d] (torch fp64), pos [M]."""
+    d = x.shape[-1]
+    half = d // 2
+    freq = theta ** (-2.0 * torch.arange(half, dtype=torch.float64) / d)
+    ang = pos.to(torch.float64)[:, None, None] * freq[None, None, :]
+    z = torch.complex(x[..., :half], x[..., half:]) * torch.polar(torch.ones_like(ang), ang)
+    return torch.cat([z.real, z.imag], dim=-1)
+
+
+def _torch_draft_block(cfg, w, states, tokens, known_len, blk_pos0=None, swap_kv=False,
+                       rope_q=True):
+    """One draft block written with torch library routines, independently of
+    the oracle (DFLARE summary sections 2.1-2.2; DFlash summary methodology
+    step 2): per layer softmax fusion + RMSNorm of the T target states,
+    context K/V through W^t at positions 0..L-1, block Q and K/V through W^d
+    at positions L..L+B-1, unmasked GQA attention over [context ; block] by
+    scaled_dot_product_attention, O projection and SwiGLU MLP with
+    residuals, final RMSNorm and the LM head.  The keyword arguments plant
+    plausible slips (block positions from 0, W^t and W^d swapped, no RoPE on
+    Q) to show the comparison notices them.  Returns (x_final, logits)."""
+    H, B, eps, theta = cfg.hidden, cfg.block, cfg.rms_eps, cfg.rope_theta
+    Hq, Hkv, d = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+    st = _t(states)
+    L = st.shape[0]
+    ids = torch.tensor([int(tokens[s]) if s < known_len else cfg.mask_token_id
+                        for s in range(B)])
+    h = _t(w["embed"])[ids]
+    pos_c = torch.arange(L)
+    pos_b = torch.arange(B) + (L if blk_pos0 is None else blk_pos0)
+    for i, lay in enumerate(w["layers"]):
+        wkt, wvt, wkd, wvd = (_t(lay[n]) for n in ("w_kt", "w_vt", "w_kd", "w_vd"))
+        if swap_kv:
+            wkt, wkd, wvt, wvd = wkd, wkt, wvd, wvt
+        a = torch.softmax(_t(w["w_fuse"][i]), dim=0)
+        f = F.rms_norm(torch.einsum("t,lth->lh", a, st), (H,), weight=_t(lay["g_fuse"]),
+                       eps=eps)
+        kc = _rope_complex(F.linear(f, wkt).reshape(L, Hkv, d), pos_c, theta)
+        vc = F.linear(f, wvt).reshape(L, Hkv, d)
+        x = F.rms_norm(h, (H,), weight=_t(lay["g_attn"]), eps=eps)
+        q = F.linear(x, _t(lay["w_q"])).reshape(B, Hq, d)
+        if rope_q:
+            q = _rope_complex(q, pos_b, theta)
+        kb = _rope_complex(F.linear(x, wkd).reshape(B, Hkv, d), pos_b, theta)
+        vb = F.linear(x, wvd).reshape(B, Hkv, d)
+        keys = torch.cat([kc, kb]).repeat_interleave(Hq // Hkv, dim=1).permute(1, 0, 2)
+        vals = torch.cat([vc, vb]).repeat_interleave(Hq // Hkv, dim=1).permute(1, 0, 2)
+        o = F.scaled_dot_product_attention(q.permute(1, 0, 2), keys, vals)   # [Hq][B][d]
+        h = h + F.linear(o.permute(1, 0, 2).reshape(B, Hq * d), _t(lay["w_o"]))
+        x = F.rms_norm(h, (H,), weight=_t(lay["g_mlp"]), eps=eps)
+        act = F.silu(F.linear(x, _t(lay["w_gate"]))) * F.linear(x, _t(lay["w_up"]))
+        h = h + F.linear(act, _t(lay["w_down"]))
+    xf = F.rms_norm(h, (H,), weight=_t(w["g_final"]), eps=eps)
+    return xf.numpy(), F.linear(xf, _t(w["lm_head"])).numpy()
+
+
+def _strong_weights(cfg, seed):
+    """Synthetic draft weights with matrices scaled to std 0.2, so attention
+    scores are O(1) and every path (positions, W^t vs W^d, the MLP) moves
+    the logits by far more than rounding."""
+    w = synth.make_weights(cfg, seed)
+    for lay in w["layers"]:
+        for n in ("w_q", "w_kt", "w_vt", "w_kd", "w_vd", "w_o", "w_gate", "w_up", "w_down"):
+            lay[n] = lay[n] * 10.0
+    w["embed"] = w["embed"] * 50.0
+    w["lm_head"] = w["lm_head"] * 10.0
+    return w
+
+
+@pytest.mark.parametrize("theta", [1.0e6, 100.0])
+def test_whole_draft_step_matches_torch_restatement(theta):
+    cfg = _tiny_cfg(rope_theta=theta)
+    w = _strong_weights(cfg, seed=31)
+    lens = [9, 4]
+    st = [synth.make_states(cfg, 31, r, lens[r]) for r in range(2)]
+    blocks = [O.Block(0, [5, 0, 0, 0, 0], 1), O.Block(1, [11, 0, 0, 0, 0], 1),
+              O.Block(0, [5, 17, 3, 0, 0], 3)]
+    keep = {}
+    tok, zmax = O.draft_step(cfg, w, st, blocks, keep=keep)
+    for i, blk in enumerate(blocks):
+        xf, z = _torch_draft_block(cfg, w, st[blk.req], blk.tokens, blk.known_len)
+        np.testing.assert_allclose(keep["x_final"][i], xf, rtol=1e-10, atol=1e-11)
+        np.testing.assert_allclose(keep["logits"][i], z, rtol=1e-10, atol=1e-11)
+        np.testing.assert_allclose(zmax[i], z.max(1), rtol=1e-10, atol=1e-11)
+        want = z.argmax(1)
+        want[:blk.known_len] = blk.tokens[:blk.known_len]
+        np.testing.assert_array_equal(tok[i], want)
+
+
+def test_torch_restatement_notices_position_and_projection_slips():
+    # each planted slip moves the logits by far more than the 1e-10 the
+    # comparison above allows, so the oracle cannot carry any of them
+    cfg = _tiny_cfg(rope_theta=100.0)
+    w = _strong_weights(cfg, seed=32)
+    st = synth.make_states(cfg, 32, 0, 9)
+    blk = O.Block(0, [5, 0, 0, 0, 0], 1)
+    keep = {}
+    O.draft_step(cfg, w, [st], [blk], keep=keep)
+    ref = keep["logits"][0]
+    scale = np.abs(ref).max()
+    for slip in (dict(blk_pos0=0), dict(swap_kv=True), dict(rope_q=False)):
+        _, z = _torch_draft_block(cfg, w, st, blk.tokens, blk.known_len, **slip)
+        assert np.abs(z - ref).max() > 1e-3 * scale, slip
