@@ -8,7 +8,7 @@ final norm, LM-head argmax and acceptance against planted target tokens
 (for the D2SD workload: first draft, lowest-confidence cuts, batched
 re-anchored second draft over K candidates, acceptance).
 
-    python bench.py [--gpus N --steps K --warmup W] [--config qwen3_4b]
+    python bench.py [--gpus N --steps K --warmup W] [--config serving32]
                     [--mode full|steady] [--impl ours|reference]
 
 Prints one JSON line (rank 0).  Under torchrun every rank runs an
@@ -34,13 +34,11 @@ sys.path.insert(0, ROOT)
 
 METRIC = "draft blocks/s and accepted tok/s per B200; HBM GB/s / tensor util vs peak"
 ACCEPT_DRAWS = 32          # planted target draws averaged for accepted tok/s
-# DRAM bytes (read + write) of one LM-head launch from an ncu capture of
-# `bench.py --op lmhead` (summarised under profiles/), valid only for the
-# GEMM code it was taken with (digest of gemm.cu without comments); any
-# later change of that code nulls it.
-LMHEAD_TRAFFIC = {         # workload -> {"bytes": int, "gemm_cu_sha256": str}
-    "qwen3_4b": {"bytes": 785283584, "gemm_cu_sha256": "c631e555a25cd81b"},
-}
+# DRAM bytes (read + write) of one launch of a kernel from an ncu capture
+# (summarised under profiles/), valid only for the source file it was taken
+# with (digest of the file without comments); any later change of that code
+# nulls it.  Key: (workload, mode, kernel-table name).
+TRAFFIC = {}
 
 
 def parse():
@@ -49,11 +47,13 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="qwen3_4b")
+    ap.add_argument("--config", default="serving32")
     ap.add_argument("--mode", choices=["full", "steady"], default="full")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the step time and kernel table of the other workloads")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the step eagerly instead of replaying a CUDA graph")
     ap.add_argument("--profile", action="store_true",
@@ -246,28 +246,33 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- our arm
-def run_ours(args):
+def _ev():
     import torch
-    rank, world, lr = dist_init("nccl")
-    from block_diffusion_speculative_softmax_b200 import build as B
-    if rank == 0:
-        B.build()
-    barrier(world)
-    from block_diffusion_speculative_softmax_b200 import dflash as DF
-    from block_diffusion_speculative_softmax_b200 import synth, workload
-    DF.load()
-    cfg = synth.get_config(args.config)
-    hbm_peak, tf_burst, tf_sust, peak_src = load_peaks()
+    return torch.cuda.Event(enable_timing=True)
 
-    wl = workload.Workload(cfg, seed=args.seed + rank, mode=args.mode)
-    # pass once, plant target tokens against the drafted blocks
-    wl.step(verify=False)
-    torch.cuda.synchronize()
-    n_plant = wl.plant_targets()
-    stream = torch.cuda.Stream()
-    clocks = Clocks(torch.cuda.current_device())
-    clocks.start()
-    clocks.mark("warm_start")
+
+def time_calls(call, stream, reps, warm=2):
+    """Mean device time (s) of ``call()`` over ``reps`` calls, CUDA events on
+    the launching stream, after ``warm`` untimed calls."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            call()
+        e0, e1 = _ev(), _ev()
+        e0.record(stream)
+        for _ in range(reps):
+            call()
+        e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps / 1e3
+
+
+def measure_step(wl, args, stream, steps, warmup, world, clocks=None):
+    """Graph-captured step replayed ``steps`` times between CUDA events on its
+    stream (after ``warmup`` replays), max over ranks.  Returns (ms, graph,
+    launches per step)."""
+    import torch
+    from block_diffusion_speculative_softmax_b200 import dflash as DF
     with torch.cuda.stream(stream):
         wl.step(verify=True)
     stream.synchronize()
@@ -281,7 +286,7 @@ def run_ours(args):
     else:
         with torch.cuda.stream(stream):
             wl.step(verify=True)
-    launches_per_step = DF.dflash_launch_count() - c0
+    launches = DF.dflash_launch_count() - c0
 
     def one_step():
         if graph is not None:
@@ -290,36 +295,39 @@ def run_ours(args):
             wl.step(verify=True)
 
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
+        for _ in range(warmup):
             one_step()
     stream.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    clocks.mark("timed_start")
+    e0, e1 = _ev(), _ev()
+    if clocks:
+        clocks.mark("timed_start")
     with torch.cuda.stream(stream):
-        ev0.record(stream)
-        for _ in range(args.steps):
+        e0.record(stream)
+        for _ in range(steps):
             one_step()
-        ev1.record(stream)
-    ev1.synchronize()
-    clocks.mark("timed_end")
+        e1.record(stream)
+    e1.synchronize()
+    if clocks:
+        clocks.mark("timed_end")
     torch.cuda.synchronize()
     barrier(world)
-    ms = ev0.elapsed_time(ev1) / args.steps
-    ms = max_over_ranks(ms, world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
     wl.check()
+    return ms, graph, launches
+
+
+def accepted_tokens(wl, stream, n_plant, draws):
+    """Mean emitted tokens per step over ``draws`` planted target draws, each
+    run through verification on the GPU (and checked for K = 1).  The step's
+    work does not depend on the targets."""
+    import torch
     fb = wl.final_buf
     n_acc = fb.n_acc.cpu().numpy()
     assert (n_acc == n_plant).all() or wl.K > 1, "accept lengths differ from the planted ones"
-    blocks_per_step = fb.nb
-    # The step's work does not depend on the targets, so the accepted tokens
-    # per step are averaged over several planted draws (each run through
-    # verification on the GPU, and checked) rather than the single draw the
-    # timed steps used.
     tok_draws = [int((n_acc + 1).sum())]
-    for draw in range(1, ACCEPT_DRAWS):
+    for draw in range(1, draws):
         n_pl = wl.plant_targets(seed_offset=draw)
         with torch.cuda.stream(stream):
             wl.step(verify=True)
@@ -328,24 +336,185 @@ def run_ours(args):
         na = fb.n_acc.cpu().numpy()
         assert (na == n_pl).all() or wl.K > 1, "accept lengths differ from the planted ones"
         tok_draws.append(int((na + 1).sum()))
-    tok_per_step = float(np.mean(tok_draws))
+    return float(np.mean(tok_draws)), len(tok_draws)
+
+
+def _entry(name, kernel, sec, count, algo_bytes, flops, peaks, ms_step):
+    """One row of the kernel table: bound and roofline fraction from the
+    algorithmic bytes / FLOPs of one call and its measured duration."""
+    hbm, tf_burst, _, src = peaks
+    ridge = tf_burst * 1e12 / (hbm * 1e9)
+    tensor = flops > 0 and flops / max(algo_bytes, 1) > ridge
+    row = {"kernel": name, "impl": kernel, "us_per_call": sec * 1e6, "calls_per_step": count,
+           "algorithmic_bytes_per_call": int(algo_bytes), "algorithmic_flops_per_call": flops,
+           "step_share_est": sec * count * 1e3 / ms_step if ms_step else None,
+           "peak_source": src}
+    if tensor:
+        a = flops / sec / 1e12
+        row.update(bound="tensor", achieved=a, peak=tf_burst, unit="TFLOP/s", frac=a / tf_burst)
+    else:
+        a = algo_bytes / sec / 1e9
+        row.update(bound="hbm", achieved=a, peak=hbm, unit="GB/s", frac=a / hbm)
+    return row
+
+
+def kernel_table(wl, cfg, DF, peaks, stream, reps, ms_step):
+    """Every entry point of the step timed alone on the workload's own device
+    buffers (weights, states, KV caches) with CUDA events on its launch
+    stream; algorithmic bytes / FLOPs per call from the path's formulas:
+    fusion reads the new rows' T states once and writes D fused rows; the
+    context K/V projection reads its rows and both weight matrices and
+    writes K and V; attention reads every request's context K/V once (its
+    candidates share it) plus Q, block K/V and the output; the MLP streams
+    its three weight matrices; the LM head streams the vocabulary."""
+    import torch
+    e = 2 if cfg.dtype == "bf16" else 4
+    H, F, V, T, D = cfg.hidden, cfg.ffn, cfg.vocab, cfg.n_target_layers, cfg.n_draft_layers
+    kvd, qd = cfg.kv_dim, cfg.q_dim
+    fb = wl.final_buf
+    nb = fb.nb
+    M = nb * cfg.block
+    cc = wl.ccfg
+    dt = wl.dt
+    rows = []
+    g = torch.Generator(device="cuda").manual_seed(1234)
+
+    def rnd(*shape, scale=1.0, dtype=dt):
+        return (torch.randn(*shape, device="cuda", generator=g) * scale).to(dtype)
+
+    n_new = wl.n_new
+    ws = DF.alloc_workspace(DF.dflash_workspace_size(cc, wl.R, nb, max(n_new, 1),
+                                                     max(wl.ctx_lens)))
+    if n_new > 0 and wl.w.w_fc is None:
+        fused = torch.empty(D, n_new, H, dtype=dt, device="cuda")
+        gl = [l["g_fuse"] for l in wl.w.layers]
+        sec = time_calls(lambda: DF.dflash_fuse_ctx(cc, wl.new_states, wl.w.w_fuse, gl, fused),
+                         stream, reps)
+        rows.append(_entry("fuse", "fuse_rows_kernel", sec, 1,
+                           n_new * T * H * e + D * n_new * H * e, 0.0, peaks, ms_step))
+        pos = torch.arange(n_new, dtype=torch.int32, device="cuda")
+        lay = wl.w.layers[0]
+        kc, vc = fb.k_cache[0], fb.v_cache[0]
+        sec = time_calls(lambda: DF.dflash_kv_project(cc, fused[0], pos, None, lay["w_kt"],
+                                                      lay["w_vt"], kc, vc, ws), stream, reps)
+        rows.append(_entry("ctx_kv_proj", "gemm_tok_kernel (RoPE epilogue)", sec, D,
+                           n_new * H * e + 2 * kvd * H * e + 2 * n_new * kvd * e,
+                           2.0 * n_new * H * 2 * kvd, peaks, ms_step))
+        del fused
+    sum_L = int(sum(wl.ctx_lens))
+    q, kb, vb = rnd(M, qd), rnd(M, kvd), rnd(M, kvd)
+    out = torch.empty(M, qd, dtype=dt, device="cuda")
+    sec = time_calls(lambda: DF.dflash_block_attn(cc, nb, q, kb, vb, fb.k_cache[0],
+                                                  fb.v_cache[0], fb.ctx_off, fb.block_req,
+                                                  fb.max_L, out, ws), stream, reps)
+    rows.append(_entry("block_attn", "attn_mma_kernel (split-KV, cluster merge)", sec, D,
+                       2 * sum_L * kvd * e + 2 * M * qd * e + 2 * M * kvd * e,
+                       4.0 * cfg.n_cand * sum_L * cfg.block * qd + 4.0 * M * cfg.block * qd,
+                       peaks, ms_step))
+    h = torch.randn(M, H, device="cuda", generator=g)
+    lay = wl.w.layers[0]
+    sec = time_calls(lambda: DF.dflash_mlp(cc, h, lay["g_mlp"], lay["w_gate"], lay["w_up"],
+                                           lay["w_down"], ws), stream, reps)
+    rows.append(_entry("mlp", "rmsnorm + SwiGLU GEMM + down GEMM", sec, D,
+                       3 * F * H * e + M * H * 4 * 2 + M * F * e * 2, 6.0 * M * H * F,
+                       peaks, ms_step))
+    x = rnd(M, H)
+    tok = torch.empty(M, dtype=torch.int32, device="cuda")
+    sec = time_calls(lambda: DF.dflash_lmhead_argmax(cc, x, wl.w.lm_head, tok, None, ws),
+                     stream, reps)
+    rows.append(_entry("lmhead_argmax", "LM-head GEMM with argmax epilogue", sec, 1,
+                       V * H * e + M * H * e + M * 12, 2.0 * M * V * H, peaks, ms_step))
+    DF.dflash_check(ws, stream=stream)
+    del ws
+    torch.cuda.empty_cache()
+    return rows
+
+
+def dominant(rows):
+    return max(rows, key=lambda r: r["us_per_call"] * r["calls_per_step"])
+
+
+def run_ours(args):
+    import torch
+    rank, world, lr = dist_init("nccl")
+    from block_diffusion_speculative_softmax_b200 import build as B
+    if rank == 0:
+        B.build()
+    barrier(world)
+    from block_diffusion_speculative_softmax_b200 import dflash as DF
+    from block_diffusion_speculative_softmax_b200 import synth, workload
+    DF.load()
+    cfg = synth.get_config(args.config)
+    peaks = load_peaks()
+    stream = torch.cuda.Stream()
+
+    wl = workload.Workload(cfg, seed=args.seed + rank, mode=args.mode)
+    # pass once, plant target tokens against the drafted blocks
+    wl.step(verify=False)
+    torch.cuda.synchronize()
+    n_plant = wl.plant_targets()
+    clocks = Clocks(torch.cuda.current_device())
+    clocks.start()
+    clocks.mark("warm_start")
+    ms, graph, launches_per_step = measure_step(wl, args, stream, args.steps, args.warmup,
+                                                world, clocks)
+    tok_per_step, n_draws = accepted_tokens(wl, stream, n_plant, ACCEPT_DRAWS)
+    blocks_per_step = wl.final_buf.nb
     value = blocks_per_step * world / (ms / 1e3)
     acc_tok_s = tok_per_step * world / (ms / 1e3)
-    # accepted draft tokens only (sum of n, without the bonus token)
     acc_draft_tok_s = (tok_per_step - wl.R) * world / (ms / 1e3)
 
-    # ---- roofline of the dominant kernel, timed alone on its own stream
-    roof = roofline(args, wl, cfg, DF, hbm_peak, tf_burst, peak_src, stream)
+    # ---- every kernel against its roofline; the dominant one is `roofline`
+    rows = kernel_table(wl, cfg, DF, peaks, stream, max(5, min(50, args.steps)), ms)
+    dom = dominant(rows)
+    roof = dict(dom)
+    roof["traffic"] = recorded_traffic(cfg.name, dom["kernel"], args.mode)
     clk = clocks.stop()
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = end_to_end(args, wl, DF, stream, world, blocks_per_step)
-
+        e2e = end_to_end(args, wl, DF, stream, world, blocks_per_step, graph)
     used_graph = graph is not None
     if graph is not None:
         del graph
+    cfg_line = {"workload": cfg.name, "mode": args.mode, "n_req": cfg.n_req,
+                "blocks_per_step": blocks_per_step, "block": cfg.block,
+                "ctx_len": cfg.ctx_len if cfg.ctx_len_min == 0 else
+                f"U[{cfg.ctx_len_min},{cfg.ctx_len}] (sum {int(sum(wl.ctx_lens))})",
+                "draft_layers": cfg.n_draft_layers, "target_layers": cfg.n_target_layers,
+                "hidden": cfg.hidden, "vocab": cfg.vocab, "parallelism": f"replicas{world}",
+                "cuda_graph": used_graph,
+                "l2": "inputs larger than L2 (weights %.2f GB streamed per step)"
+                      % (wl.w.nbytes() / 1e9)}
+    del wl
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads (rank-local, no collectives): step time and
+    # dominant-kernel roofline of each
+    per_config = {}
+    if world == 1 and not args.no_per_config:
+        for name in synth.CONFIG_ORDER:
+            if name == cfg.name:
+                continue
+            c2 = synth.get_config(name)
+            w2 = workload.Workload(c2, seed=args.seed, mode=args.mode)
+            w2.step(verify=False)
+            torch.cuda.synchronize()
+            n2 = w2.plant_targets()
+            steps2 = max(5, min(args.steps, 30))
+            ms2, g2, _ = measure_step(w2, args, stream, steps2, max(3, args.warmup), 1)
+            del g2
+            t2, _ = accepted_tokens(w2, stream, n2, 4)
+            r2 = kernel_table(w2, c2, DF, peaks, stream, 10, ms2)
+            d2 = dominant(r2)
+            per_config[name] = {"ms_per_step": ms2, "blocks_s": w2.final_buf.nb / (ms2 / 1e3),
+                                "accepted_tok_s": t2 / (ms2 / 1e3), "steps": steps2,
+                                "dominant_kernel": d2["kernel"], "dominant_bound": d2["bound"],
+                                "dominant_frac": d2["frac"],
+                                "kernels": {r["kernel"]: round(r["frac"], 4) for r in r2}}
+            del w2
+            torch.cuda.empty_cache()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(cfg, args.seed)
@@ -356,21 +525,14 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if cfg.dtype == "bf16" else "fp32", "data": "synthetic",
             "accepted_tok_s": acc_tok_s, "accepted_draft_tok_s": acc_draft_tok_s,
-            "mean_accept_tau": tok_per_step / wl.R,
-            "accept_draws": len(tok_draws),
-            "config": {"workload": cfg.name, "mode": args.mode, "n_req": cfg.n_req,
-                       "blocks_per_step": blocks_per_step, "block": cfg.block,
-                       "ctx_len": cfg.ctx_len if cfg.ctx_len_min == 0 else
-                       f"U[{cfg.ctx_len_min},{cfg.ctx_len}]",
-                       "draft_layers": cfg.n_draft_layers, "target_layers": cfg.n_target_layers,
-                       "hidden": cfg.hidden, "vocab": cfg.vocab,
-                       "parallelism": f"replicas{world}",
-                       "cuda_graph": used_graph,
-                       "l2": "inputs larger than L2 (weights %.2f GB streamed per step)"
-                             % (wl.w.nbytes() / 1e9)},
+            "mean_accept_tau": tok_per_step / cfg.n_req,
+            "accept_draws": n_draws,
+            "config": cfg_line,
             "gpu_launches": launches_per_step * args.steps,
             "launches_per_step": launches_per_step,
             "roofline": roof,
+            "kernels": rows,
+            "per_config": per_config or None,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
@@ -391,67 +553,28 @@ def code_digest(text):
     return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()
 
 
-def gemm_source_digest():
-    src = os.path.join(ROOT, "block_diffusion_speculative_softmax_b200", "csrc", "gemm.cu")
+def source_digest(fname):
+    src = os.path.join(ROOT, "block_diffusion_speculative_softmax_b200", "csrc", fname)
     with open(src) as f:
         return code_digest(f.read())
 
 
-def lmhead_traffic(workload):
-    """Measured DRAM bytes per LM-head launch, or None when there is no
-    capture for this workload or the GEMM code changed since."""
-    ent = LMHEAD_TRAFFIC.get(workload)
+def recorded_traffic(workload, kernel, mode="full"):
+    """Measured DRAM bytes (read + write) per launch of ``kernel`` on
+    ``workload``, or None when there is no capture for it or its source file
+    changed since the capture."""
+    ent = TRAFFIC.get((workload, mode, kernel))
     if ent is None:
         return None
-    return ent["bytes"] if gemm_source_digest().startswith(ent["gemm_cu_sha256"]) else None
+    return ent["bytes"] if source_digest(ent["file"]).startswith(ent["sha256"]) else None
 
 
-def roofline(args, wl, cfg, DF, hbm_peak, tf_burst, peak_src, stream):
-    """LM-head argmax (weight streaming, the largest single launch of the
-    step), timed alone with CUDA events on its launch stream."""
-    import torch
-    M = wl.final_buf.nb * cfg.block
-    H, V = cfg.hidden, cfg.vocab
-    x = torch.randn(M, H, device="cuda").to(wl.dt)
-    tok = torch.empty(M, dtype=torch.int32, device="cuda")
-    ws = DF.alloc_workspace(DF.dflash_workspace_size(wl.ccfg, 1, wl.final_buf.nb, 0, 0))
-    reps = max(10, min(200, args.steps))
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            DF.dflash_lmhead_argmax(wl.ccfg, x, wl.w.lm_head, tok, None, ws, stream=stream)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            DF.dflash_lmhead_argmax(wl.ccfg, x, wl.w.lm_head, tok, None, ws, stream=stream)
-        e1.record(stream)
-    e1.synchronize()
-    DF.dflash_check(ws, stream=stream)
-    sec = e0.elapsed_time(e1) / reps / 1e3
-    esz = 2 if cfg.dtype == "bf16" else 4
-    algo = V * H * esz + M * H * esz + M * 8 + M * 4
-    flops = 2.0 * M * V * H
-    common = {"kernel": "lmhead_argmax (tcgen05 GEMM, argmax epilogue)",
-              "peak_source": peak_src, "traffic": lmhead_traffic(cfg.name),
-              "algorithmic_bytes_per_launch": algo, "algorithmic_flops_per_launch": flops,
-              "us_per_launch": sec * 1e6,
-              "note": "time includes the argmax-key reset and finish launches"}
-    # bf16 with enough tokens per weight byte to pass the ridge point is
-    # bounded by the tensor pipe (burst peak: the kernel is timed alone)
-    if cfg.dtype == "bf16" and flops / algo > tf_burst * 1e12 / (hbm_peak * 1e9):
-        tf = flops / sec / 1e12
-        return dict(common, bound="tensor", achieved=tf, peak=tf_burst, unit="TFLOP/s",
-                    frac=tf / tf_burst)
-    gbs = algo / sec / 1e9
-    return dict(common, bound="hbm", achieved=gbs, peak=hbm_peak, unit="GB/s",
-                frac=gbs / hbm_peak)
-
-
-def end_to_end(args, wl, DF, stream, world, blocks_per_step):
+def end_to_end(args, wl, DF, stream, world, blocks_per_step, graph=None):
     """Per step: pinned host -> device copy of the step's inputs (the target
     states of the new context rows, the block tokens and the target tokens),
-    the draft step + verification through the public API, and a device ->
-    host read of the accepted tokens and lengths."""
+    the draft step + verification (the captured graph of the public API's
+    calls when there is one, else the calls themselves), and a device -> host
+    read of the accepted tokens and lengths."""
     import torch
     fb = wl.final_buf
     dev_in = [t for t in (wl.new_states, wl.buf.block_tokens, fb.target_tokens) if t is not None]
@@ -460,25 +583,27 @@ def end_to_end(args, wl, DF, stream, world, blocks_per_step):
                 torch.empty_like(fb.n_acc, device="cpu").pin_memory()]
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
-    steps = max(3, min(args.steps, 50))
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
+    steps = max(3, min(args.steps, 20))
+    e0, e1 = _ev(), _ev()
     with torch.cuda.stream(stream):
         for i in range(steps + 2):
             if i == 2:
                 e0.record(stream)
             for d, h in zip(dev_in, host_in):
                 d.copy_(h, non_blocking=True)
-            wl.step(verify=True, stream=stream)
+            if graph is not None:
+                graph.replay()
+            else:
+                wl.step(verify=True, stream=stream)
             host_out[0].copy_(fb.out_tok, non_blocking=True)
             host_out[1].copy_(fb.n_acc, non_blocking=True)
         e1.record(stream)
     e1.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    ms = max_over_ranks(ms, world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
     return {"value": blocks_per_step * world / (ms / 1e3), "unit": "blocks/s",
             "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "api": "dflash_draft_step via the Python binding, eager launches"}
+            "api": "dflash_draft_step (graph-replayed) with pinned host copies in and out"
+                   if graph is not None else "dflash_draft_step via the Python binding"}
 
 
 # ---------------------------------------------------------------- profiling modes

@@ -142,6 +142,15 @@ GemmJob job_resid(const dflash_config* c, const void* w, const void* x, int64_t 
   return j;
 }
 
+// DFlash FC fusion: fp32 u = states[N][T*H] W_fc^T (RMSNorm follows).
+GemmJob job_fc(const dflash_config* c, const void* states, int64_t N, const void* w_fc,
+               float* u) {
+  GemmJob j = job_base(c, states, N, c->n_target_layers * c->hidden);
+  j.nseg = 1;
+  j.seg[0] = {w_fc, nullptr, c->hidden, EPI_STORE_F32, 0, u, c->hidden, 0};
+  return j;
+}
+
 GemmJob job_swiglu(const dflash_config* c, const void* wg, const void* wu, const void* x,
                    int64_t M, void* act) {
   GemmJob j = job_base(c, x, M, c->hidden);
@@ -171,7 +180,10 @@ struct Needs {
 Needs step_needs(const dflash_config* c, int64_t M, int64_t n_new) {
   Needs n;
   dflash_layer_weights l{};
-  if (n_new > 0) n.take(plan_gemm(job_kv(c, nullptr, n_new, nullptr, nullptr, 0, 0, 0, 0)));
+  if (n_new > 0) {
+    n.take(plan_gemm(job_kv(c, nullptr, n_new, nullptr, nullptr, 0, 0, 0, 0)));
+    n.take(plan_gemm(job_fc(c, nullptr, n_new, nullptr, nullptr)));
+  }
   if (M > 0) {
     n.take(plan_gemm(job_kv(c, nullptr, M, nullptr, nullptr, 0, 0, 0, 0)));
     n.take(plan_gemm(job_qkv(c, l, nullptr, M, nullptr, 0, 0, 0)));
@@ -207,13 +219,18 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
   L.vb = take(M * kvd * e);
   L.attn = take(M * qd * e);
   L.act = take(M * F * e);
-  L.fused = take(static_cast<size_t>(c->n_draft_layers) * n_new * H * e);
+  // per-layer fused contexts [D][N][H]; the FC variant keeps one [N][H]
+  // context behind its fp32 product [N][H] in the same region
+  L.fused = take(std::max(static_cast<size_t>(c->n_draft_layers) * e, 4 + e) * n_new * H);
   L.partial = take(nd.partial_floats * 4);
   L.attn_ws = take(attn_ws_bytes(ap, nb, c->block, c->n_q_heads, c->head_dim));
   const size_t ncount = nd.counters;
   // the context branch runs on a second stream: its own split-K scratch
   Needs side;
-  if (n_new > 0) side.take(plan_gemm(job_kv(c, nullptr, n_new, nullptr, nullptr, 0, 0, 0, 0)));
+  if (n_new > 0) {
+    side.take(plan_gemm(job_kv(c, nullptr, n_new, nullptr, nullptr, 0, 0, 0, 0)));
+    side.take(plan_gemm(job_fc(c, nullptr, n_new, nullptr, nullptr)));
+  }
   L.partial_side = take(side.partial_floats * 4);
   L.zero = off;
   L.keys = take(M * 8);
@@ -342,6 +359,36 @@ dflash_status dflash_fuse_ctx(const dflash_config* cfg, const void* states, int6
                        cfg->n_draft_layers, w_fuse, g_fuse, fused, cfg->rms_eps, nullptr,
                        static_cast<cudaStream_t>(stream)),
            "fusion kernel");
+  return DFLASH_OK;
+}
+
+dflash_status dflash_fc_fuse_ctx(const dflash_config* cfg, const void* states, int64_t n_rows,
+                                 const void* w_fc, const float* g_fc, void* fused, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  dflash_status s = check_config(cfg);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(n_rows >= 0 && n_rows < (int64_t(1) << 31), DFLASH_EINVAL, "n_rows out of range");
+  if (n_rows == 0) return DFLASH_OK;
+  DFL_PTR(states, "states");
+  DFL_PTR(w_fc, "w_fc");
+  DFL_PTR(g_fc, "g_fc");
+  DFL_PTR(fused, "fused");
+  const int H = cfg->hidden;
+  const size_t off_u = sizeof(DevStatus);
+  const GemmJob j = job_fc(cfg, states, n_rows, w_fc, at<float>(ws, off_u));
+  const GemmPlan pl = plan_gemm(j);
+  const size_t off_part = align256(off_u + static_cast<size_t>(n_rows) * H * 4);
+  const size_t off_cnt = align256(off_part + pl.partial_floats * 4);
+  const size_t need = off_cnt + pl.counters * 4;
+  if ((s = check_ws(ws, ws_bytes, need)) != DFLASH_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DFL_CUDA(launch_zero(at<void>(ws, off_cnt), pl.counters * 4, st), "counter reset");
+  DFL_CUDA(launch_gemm(j, pl, at<float>(ws, off_part), at<uint32_t>(ws, off_cnt),
+                       status_word(ws), st),
+           "FC fusion GEMM");
+  DFL_CUDA(launch_rmsnorm(cfg->dtype, at<float>(ws, off_u), n_rows, H, g_fc, cfg->rms_eps, fused,
+                          st),
+           "FC fusion rmsnorm");
   return DFLASH_OK;
 }
 
@@ -559,7 +606,14 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
   DFL_ALIGNED(a->best_k, 4, "best_k");
   DFL_ALIGNED(a->out_tok, 4, "out_tok");
   if (a->n_ctx_new > 0) DFL_PTR(a->new_states, "new_states");
-  DFL_CHECK(w->w_fuse && w->layers, DFLASH_EINVAL, "w_fuse / layers is NULL");
+  DFL_CHECK(w->layers, DFLASH_EINVAL, "layers is NULL");
+  const bool fc = w->w_fc != nullptr;
+  if (fc) {
+    DFL_PTR(w->w_fc, "w_fc");
+    DFL_PTR(w->g_fc, "g_fc");
+  } else {
+    DFL_CHECK(w->w_fuse != nullptr, DFLASH_EINVAL, "w_fuse is NULL");
+  }
   DFL_PTR(w->embed, "embed");
   DFL_PTR(w->lm_head, "lm_head");
   DFL_PTR(w->g_final, "g_final");
@@ -575,7 +629,7 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
     DFL_PTR(l.w_gate, "w_gate");
     DFL_PTR(l.w_up, "w_up");
     DFL_PTR(l.w_down, "w_down");
-    DFL_PTR(l.g_fuse, "g_fuse");
+    if (!fc) DFL_PTR(l.g_fuse, "g_fuse");
     DFL_PTR(l.g_attn, "g_attn");
     DFL_PTR(l.g_mlp, "g_mlp");
     if (a->max_ctx_len > 0) {
@@ -629,21 +683,34 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
       DFL_CUDA(cudaStreamWaitEvent(side->stream, side->fork, 0), "fork");
       cs = side->stream;
     }
-    const float* gf[kMaxLayers];
-    for (int i = 0; i < D; ++i) gf[i] = w->layers[i].g_fuse;
-    DFL_CUDA(launch_fuse(dt, a->new_states, a->n_ctx_new, c->n_target_layers, H, D, w->w_fuse,
-                         gf, fused, c->rms_eps, status, cs),
-             "fusion kernel");
+    float* part_c = side ? at<float>(ws, L.partial_side) : partial;
+    uint32_t* cnt_c = side ? at<uint32_t>(ws, L.counters_side) : counters;
+    // FC variant: fp32 product at the start of the fused region, the one
+    // shared context right behind it
+    uint8_t* fc_ctx = fused + static_cast<size_t>(a->n_ctx_new) * H * 4;
+    if (fc) {
+      s = run_job(job_fc(c, a->new_states, a->n_ctx_new, w->w_fc, reinterpret_cast<float*>(fused)),
+                  part_c, cnt_c, status, cs, "FC fusion GEMM");
+      if (s != DFLASH_OK) return s;
+      DFL_CUDA(launch_rmsnorm(dt, reinterpret_cast<float*>(fused), a->n_ctx_new, H, w->g_fc,
+                              c->rms_eps, fc_ctx, cs),
+               "FC fusion rmsnorm");
+    } else {
+      const float* gf[kMaxLayers];
+      for (int i = 0; i < D; ++i) gf[i] = w->layers[i].g_fuse;
+      DFL_CUDA(launch_fuse(dt, a->new_states, a->n_ctx_new, c->n_target_layers, H, D, w->w_fuse,
+                           gf, fused, c->rms_eps, status, cs),
+               "fusion kernel");
+    }
     for (int i = 0; i < D; ++i) {
       const dflash_layer_weights& l = w->layers[i];
-      GemmJob jc = job_kv(c, fused + static_cast<size_t>(i) * a->n_ctx_new * H * e,
-                          a->n_ctx_new, new_pos, new_dst, l.w_kt, l.w_vt, a->k_cache[i],
-                          a->v_cache[i]);
+      const void* ctx_i = fc ? static_cast<const void*>(fc_ctx)
+                             : fused + static_cast<size_t>(i) * a->n_ctx_new * H * e;
+      GemmJob jc = job_kv(c, ctx_i, a->n_ctx_new, new_pos, new_dst, l.w_kt, l.w_vt,
+                          a->k_cache[i], a->v_cache[i]);
       jc.rope_tab = rope_tab;
       jc.rope_len = L.rope_len;
-      s = run_job(jc, side ? at<float>(ws, L.partial_side) : partial,
-                  side ? at<uint32_t>(ws, L.counters_side) : counters, status, cs,
-                  "context K/V GEMM");
+      s = run_job(jc, part_c, cnt_c, status, cs, "context K/V GEMM");
       if (s != DFLASH_OK) return s;
       if (side) DFL_CUDA(cudaEventRecord(side->done[i], side->stream), "context done");
     }

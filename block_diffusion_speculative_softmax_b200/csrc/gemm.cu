@@ -457,7 +457,10 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
               const float pv = st[(j0 + q) * SROW + prt];
               v = i < half ? v * cs[q].x - pv * cs[q].y : v * cs[q].x + pv * cs[q].y;
             }
-            o[orow[q] * S.out_stride + f] = __float2bfloat16_rn(v);
+            if (S.op == EPI_STORE_F32)
+              static_cast<float*>(S.out)[orow[q] * S.out_stride + f] = v;
+            else
+              o[orow[q] * S.out_stride + f] = __float2bfloat16_rn(v);
           }
         }
       }
@@ -789,6 +792,17 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
       const int d = p.head_dim, half = d >> 1;
       const int pos = (tv && S.rope) ? p.pos[t] : 0;
       auto put16 = [&](int f, const float* v) {
+        if (S.op == EPI_STORE_F32) {
+          float* of = static_cast<float*>(S.out) + orow * S.out_stride;
+          if (f + 16 <= S.rows) {
+#pragma unroll
+            for (int q = 0; q < 16; q += 4)
+              *reinterpret_cast<float4*>(of + f + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+          } else {
+            for (int q = 0; q < 16 && f + q < S.rows; ++q) of[f + q] = v[q];
+          }
+          return;
+        }
         alignas(16) __nv_bfloat16 r[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) r[q] = __float2bfloat16_rn(v[q]);
@@ -1242,7 +1256,10 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
                 const float pv = st[(j0 + q) * SROW + prt];
                 x = i < half ? x * cs[q].x - pv * cs[q].y : x * cs[q].x + pv * cs[q].y;
               }
-              o[orow[q] * S.out_stride + f] = __float2bfloat16_rn(x);
+              if (S.op == EPI_STORE_F32)
+                static_cast<float*>(S.out)[orow[q] * S.out_stride + f] = x;
+              else
+                o[orow[q] * S.out_stride + f] = __float2bfloat16_rn(x);
             }
           }
         }

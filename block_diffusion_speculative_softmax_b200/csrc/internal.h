@@ -26,7 +26,7 @@ void count_launch(int n = 1);
 // token m of X [M][K]:  y[m][r] = sum_k X[m][k] W_s[r][k], then the
 // segment's epilogue op writes the result.
 constexpr int kMaxSegs = 3;
-enum EpiOp { EPI_NONE = 0, EPI_STORE = 1, EPI_RESID = 2, EPI_SWIGLU = 3 };
+enum EpiOp { EPI_NONE = 0, EPI_STORE = 1, EPI_RESID = 2, EPI_SWIGLU = 3, EPI_STORE_F32 = 4 };
 
 struct GemmOut {
   const void* w0;      // weights [rows][K]; the gate matrix for EPI_SWIGLU
@@ -35,6 +35,7 @@ struct GemmOut {
   int op;              // EPI_STORE: out = y (dtype), optional RoPE and row scatter
                        // EPI_RESID: fp32 out += y
                        // EPI_SWIGLU: out = silu(y_gate) * y_up (dtype)
+                       // EPI_STORE_F32: fp32 out = y (no RoPE, no scatter)
   int rope;            // EPI_STORE: rotate-half RoPE over heads of head_dim
   void* out;
   int64_t out_stride;  // elements between output rows

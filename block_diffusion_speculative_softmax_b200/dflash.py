@@ -65,7 +65,8 @@ class LayerWeights(C.Structure):
 
 class Weights(C.Structure):
     _fields_ = [("w_fuse", C.c_void_p), ("layers", C.POINTER(LayerWeights)),
-                ("embed", C.c_void_p), ("g_final", C.c_void_p), ("lm_head", C.c_void_p)]
+                ("embed", C.c_void_p), ("g_final", C.c_void_p), ("lm_head", C.c_void_p),
+                ("w_fc", C.c_void_p), ("g_fc", C.c_void_p)]
 
 
 class StepArgs(C.Structure):
@@ -93,6 +94,7 @@ SIGNATURES = {
     "dflash_launch_count": (C.c_uint64, []),
     "dflash_version": (C.c_char_p, []),
     "dflash_fuse_ctx": (C.c_int, [_CFG, _VP, _I64, _VP, C.POINTER(_VP), _VP, _VP]),
+    "dflash_fc_fuse_ctx": (C.c_int, [_CFG, _VP, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "dflash_kv_project": (C.c_int, [_CFG, _VP, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ,
                                     _VP]),
     "dflash_block_attn": (C.c_int, [_CFG, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _VP,
@@ -208,6 +210,12 @@ def dflash_fuse_ctx(cfg: Config, states: torch.Tensor, w_fuse: torch.Tensor,
                                   _p(fused), _stream(stream)))
 
 
+def dflash_fc_fuse_ctx(cfg: Config, states: torch.Tensor, w_fc: torch.Tensor,
+                       g_fc: torch.Tensor, fused: torch.Tensor, ws, stream=None):
+    _check(load().dflash_fc_fuse_ctx(C.byref(cfg), _p(states), states.shape[0], _p(w_fc),
+                                     _p(g_fc), _p(fused), _p(ws), ws.numel(), _stream(stream)))
+
+
 def dflash_kv_project(cfg: Config, x, pos, dst_row, w_k, w_v, k_out, v_out, ws, stream=None):
     _check(load().dflash_kv_project(C.byref(cfg), _p(x), x.shape[0], _p(pos), _p(dst_row),
                                     _p(w_k), _p(w_v), _p(k_out), _p(v_out), _p(ws), ws.numel(),
@@ -273,6 +281,9 @@ class DeviceWeights:
             return torch.as_tensor(a).to(device=device, dtype=dtype).contiguous()
 
         self.w_fuse = dev(host["w_fuse"], f32)
+        # DFlash FC fusion (optional): one shared context for every layer
+        self.w_fc = dev(host["w_fc"], dt) if "w_fc" in host else None
+        self.g_fc = dev(host["g_fc"], f32) if "w_fc" in host else None
         self.embed = dev(host["embed"], dt)
         self.lm_head = dev(host["lm_head"], dt)
         self.g_final = dev(host["g_final"], f32)
@@ -290,11 +301,14 @@ class DeviceWeights:
                 "w_q", "w_kt", "w_vt", "w_kd", "w_vd", "w_o", "w_gate", "w_up", "w_down",
                 "g_fuse", "g_attn", "g_mlp")]) for d in self.layers])
         self.struct = Weights(self.w_fuse.data_ptr(), self._lw, self.embed.data_ptr(),
-                              self.g_final.data_ptr(), self.lm_head.data_ptr())
+                              self.g_final.data_ptr(), self.lm_head.data_ptr(),
+                              None if self.w_fc is None else self.w_fc.data_ptr(),
+                              None if self.g_fc is None else self.g_fc.data_ptr())
 
     def nbytes(self) -> int:
         tot = sum(t.numel() * t.element_size() for t in (self.w_fuse, self.embed, self.lm_head,
-                                                        self.g_final))
+                                                        self.g_final, self.w_fc, self.g_fc)
+                  if t is not None)
         for d in self.layers:
             tot += sum(t.numel() * t.element_size() for t in d.values())
         return tot

@@ -31,7 +31,7 @@ import numpy as np
 
 __all__ = [
     "DraftConfig", "CONFIGS", "CONFIG_ORDER", "get_config", "to_bf16_bits",
-    "round_bf16", "make_weights", "make_states", "ctx_lengths", "make_anchors",
+    "round_bf16", "make_weights", "make_fc_weights", "make_states", "ctx_lengths", "make_anchors",
     "make_confidence", "geometric_lengths", "plant_targets",
     "plant_targets_d2sd", "small_config",
 ]
@@ -181,6 +181,15 @@ def make_weights(cfg: DraftConfig, seed: int = 0,
             lay["w_vt"] = lay["w_vd"]
         w["layers"].append(lay)
     return w
+
+
+def make_fc_weights(cfg: DraftConfig, seed: int = 0) -> dict:
+    """Weights of the DFlash-style FC context fusion: w_fc [H][T*H] ~
+    N(0, 0.02) and its RMSNorm gain g_fc = 1 + N(0, 0.02) (streams 14, 15).
+    Add them to a ``make_weights`` dict to select that variant."""
+    H, T = cfg.hidden, cfg.n_target_layers
+    return {"w_fc": _draw(_rng(cfg, seed, 14), (H, T * H), 0.02, cfg),
+            "g_fc": _draw(_rng(cfg, seed, 15), (H,), 0.02, cfg, 1.0)}
 
 
 def ctx_lengths(cfg: DraftConfig, seed: int = 0) -> List[int]:

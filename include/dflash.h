@@ -104,6 +104,16 @@ typedef struct {
   const void* embed;                  /* [V][H] slot embeddings */
   const float* g_final;               /* [H] final RMSNorm gain */
   const void* lm_head;                /* [V][H] */
+  /* DFlash-style context fusion (DFLARE summary, section 1 item 1 and
+   * section 2.2, describing the DFlash baseline).  NULL (the default): every
+   * draft layer fuses the T target layers with its own softmax weights
+   * (w_fuse, g_fuse).  Non-NULL: ONE fully connected layer maps the
+   * concatenated target states of a row to a single context shared by all
+   * draft layers, c = RMSNorm_{g_fc}(concat(h_1..h_T) W_fc^T); w_fuse and the
+   * layers' g_fuse are then unused.  (DFlash also shares the K/V projection
+   * between context and block: pass w_kt = w_kd and w_vt = w_vd.) */
+  const void* w_fc;                   /* [H][T*H] (nullable) */
+  const float* g_fc;                  /* [H] fp32 (required with w_fc) */
 } dflash_weights;
 
 /* ------------------------------------------------------------------------
@@ -149,6 +159,16 @@ dflash_status dflash_fuse_ctx(const dflash_config* cfg, const void* states,
                               int64_t n_rows, const float* w_fuse,
                               const float* const* g_fuse, void* fused,
                               void* stream);
+
+/* DFlash-style FC context fusion (DFLARE summary, section 1 item 1 and
+ * section 2.2): states [N][T][H] (dtype), viewed as [N][T*H] ->
+ *   fused[n, :] = RMSNorm_{g_fc}(states[n] W_fc^T)   [N][H] (dtype)
+ * w_fc [H][T*H] (dtype), g_fc [H] fp32.  The fp32 product is staged in the
+ * workspace (N*H*4 bytes after the header); N may be 0 (no launch). */
+dflash_status dflash_fc_fuse_ctx(const dflash_config* cfg, const void* states,
+                                 int64_t n_rows, const void* w_fc,
+                                 const float* g_fc, void* fused, void* ws,
+                                 size_t ws_bytes, void* stream);
 
 /* K/V projection, DFLARE summary section 2.2 (called with W^t for context
  * rows and with W^d for block rows):

@@ -113,6 +113,6 @@ def test_traffic_digest_ignores_comments_but_not_code():
     assert bench.code_digest(base) == bench.code_digest(base.replace("// one", "// two"))
     assert bench.code_digest(base) == bench.code_digest(base.replace("/* block */", ""))
     assert bench.code_digest(base) != bench.code_digest(base.replace("a + 1", "a + 2"))
-    # the recorded LM-head traffic belongs to the GEMM code in this tree
-    for ent in bench.LMHEAD_TRAFFIC.values():
-        assert bench.gemm_source_digest().startswith(ent["gemm_cu_sha256"])
+    # every recorded DRAM traffic figure belongs to the code in this tree
+    for ent in bench.TRAFFIC.values():
+        assert bench.source_digest(ent["file"]).startswith(ent["sha256"])

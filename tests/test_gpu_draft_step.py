@@ -98,6 +98,18 @@ def test_small_shapes(W, name):
         _verify_planted(wl)
 
 
+@pytest.mark.parametrize("name", ["bf16_ragged", "bf16_multi_req", "fp32_b1"])
+def test_small_dflash_fc_variant(W, name):
+    # DFlash baseline: one FC-fused context for every layer, context and block
+    # sharing the K/V projections (DFLARE summary, section 1 item 1, 2.2)
+    cfg = synth.small_config("qwen3_4b", **SMALL[name])
+    hw = synth.make_weights(cfg, 0, separate_kv=False)
+    hw.update(synth.make_fc_weights(cfg, 0))
+    wl, rep, _ = _run_pass1(W, cfg, host_weights=hw)
+    if cfg.block > 1:
+        _verify_planted(wl)
+
+
 def test_small_steady_state_matches_full(W):
     cfg = synth.small_config("qwen3_4b", **SMALL["bf16_multi_req"])
     _run_pass1(W, cfg, mode="steady", steady_new_rows=7)

@@ -59,6 +59,28 @@ def test_fuse_ctx(DF, dtype, H, T, D, N):
     assert rel_err(out.float().cpu().numpy(), want) <= TOL[dtype]
 
 
+# DFlash-style FC fusion: one Linear(T*H -> H) + RMSNorm shared by all layers
+@pytest.mark.parametrize("dtype,H,T,N", [("fp32", 256, 3, 37), ("bf16", 576, 5, 300),
+                                         ("bf16", 2560, 5, 2048), ("bf16", 4096, 9, 65),
+                                         ("bf16", 2880, 5, 16)])
+def test_fc_fuse_ctx(DF, dtype, H, T, N):
+    # N = 2048 / 300 / 65: token-major tiles (2048: CTA pairs); 16: weight-major
+    cfg = _cfg(dtype, hidden=H, n_target_layers=T)
+    rng = np.random.default_rng(H + T + N)
+    st = _round(cfg, rng.standard_normal((N, T, H)))
+    w_fc = _round(cfg, 0.02 * rng.standard_normal((H, T * H)))
+    g = _round(cfg, 1 + 0.02 * rng.standard_normal(H))
+    ccfg = DF.config_from(cfg)
+    dt = _tdt(cfg)
+    out = torch.empty(N, H, dtype=dt, device="cuda")
+    ws = DF.alloc_workspace(DF.dflash_workspace_size(ccfg, 1, 1, N, N))
+    DF.dflash_fc_fuse_ctx(ccfg, to_dev(st, dt), to_dev(w_fc, dt), to_dev(g, torch.float32),
+                          out, ws)
+    DF.dflash_check(ws)
+    want = O.fc_fuse_ctx(st, w_fc, g, cfg.rms_eps, bf16_storage=(dtype == "bf16"))
+    assert rel_err(out.float().cpu().numpy(), want) <= TOL[dtype]
+
+
 def test_fuse_ctx_zero_rows_is_noop(DF):
     cfg = _cfg()
     ccfg = DF.config_from(cfg)
