@@ -256,7 +256,17 @@ dflash_status dflash_d2sd_candidates(int32_t R, int32_t B, int32_t K,
  *     that device current); make that first call before any stream capture;
  *   - all calls share the array: calls that overlap on the GPU (different
  *     streams, or different host threads on one device) race;
- *   - non-finite logits are not reported (there is no workspace header). */
+ *   - the cached address stays valid until the device's primary context is
+ *     reset (cudaDeviceReset); do not call this entry point after a reset;
+ *   - device-side errors are NOT reported: there is no workspace header, so
+ *     neither a non-finite logit (DFLASH_ENUMERIC) nor a bounded wait that
+ *     ran out (DFLASH_ETIMEOUT) reaches the caller, and the tokens of such a
+ *     call are undefined; callers that need those checks use
+ *     dflash_lmhead_argmax with a workspace and dflash_check;
+ *   - with at most 64 tokens it runs the one-CTA-per-tile weight-streaming
+ *     kernel (the stream-K kernel of dflash_lmhead_argmax needs workspace
+ *     partials), so at batch 1 it is somewhat slower than that entry point;
+ *     65 tokens and more take the same token-major kernel as it does. */
 dflash_status dflash_lmhead_argmax_noalloc(const dflash_config* cfg, int64_t M,
                                            const void* x, const void* w_lm,
                                            int32_t* tok, float* max_logit,
