@@ -151,6 +151,15 @@ GemmJob job_fc(const dflash_config* c, const void* states, int64_t N, const void
   return j;
 }
 
+// LM head writing fp32 logits [M][V] (temperature-1 mode).
+GemmJob job_logits(const dflash_config* c, const void* x, int64_t M, const void* w_lm,
+                   float* logits) {
+  GemmJob j = job_base(c, x, M, c->hidden);
+  j.nseg = 1;
+  j.seg[0] = {w_lm, nullptr, c->vocab, EPI_STORE_F32, 0, logits, c->vocab, 0};
+  return j;
+}
+
 GemmJob job_swiglu(const dflash_config* c, const void* wg, const void* wu, const void* x,
                    int64_t M, void* act) {
   GemmJob j = job_base(c, x, M, c->hidden);
@@ -163,7 +172,7 @@ GemmJob job_swiglu(const dflash_config* c, const void* wg, const void* wu, const
 struct Layout {
   size_t h = 0, x = 0, q = 0, kb = 0, vb = 0, attn = 0, act = 0, fused = 0, partial = 0,
          attn_ws = 0, zero = 0, keys = 0, counters = 0, blk_pos = 0, new_pos = 0, new_dst = 0,
-         rope = 0, partial_side = 0, counters_side = 0, lse = 0, total = 0;
+         rope = 0, partial_side = 0, counters_side = 0, lse = 0, row_lse = 0, total = 0;
   int rope_len = 0;
   size_t zero_bytes = 0;   // [keys | counters], zeroed at the start of a step
 };
@@ -191,6 +200,7 @@ Needs step_needs(const dflash_config* c, int64_t M, int64_t n_new) {
     n.take(plan_gemm(job_swiglu(c, nullptr, nullptr, nullptr, M, 0)));
     n.take(plan_gemm(job_resid(c, nullptr, nullptr, M, c->ffn, 0)));
     n.take(plan_lmhead(c->dtype, c->vocab, M, c->hidden));
+    n.take(plan_gemm(job_logits(c, nullptr, M, nullptr, nullptr)));
   }
   return n;
 }
@@ -241,6 +251,7 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
   L.new_pos = take(n_new * 4);
   L.new_dst = take(n_new * 8);
   L.lse = take(static_cast<size_t>(lmhead_tiles(c->dtype, c->vocab, M)) * M * 8);
+  L.row_lse = take(M * 4);   // temperature-1 mode: logsumexp of each logit row
   L.rope_len = static_cast<int>(max_ctx + c->block);
   L.rope = take(static_cast<size_t>(L.rope_len) * (c->head_dim / 2) * 8);
   L.total = off;
@@ -527,6 +538,75 @@ dflash_status dflash_lmhead_argmax(const dflash_config* cfg, int64_t M, const vo
   return DFLASH_OK;
 }
 
+dflash_status dflash_lmhead_logits(const dflash_config* cfg, int64_t M, const void* x,
+                                   const void* w_lm, float* logits, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  dflash_status s = check_config(cfg);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(M >= 0 && M < (int64_t(1) << 31), DFLASH_EINVAL, "M out of range");
+  if (M == 0) return DFLASH_OK;
+  DFL_PTR(x, "x");
+  DFL_PTR(w_lm, "w_lm");
+  DFL_PTR(logits, "logits");
+  const GemmJob j = job_logits(cfg, x, M, w_lm, logits);
+  const GemmPlan pl = plan_gemm(j);
+  const size_t off_part = sizeof(DevStatus);
+  const size_t off_cnt = align256(off_part + pl.partial_floats * 4);
+  if ((s = check_ws(ws, ws_bytes, off_cnt + pl.counters * 4)) != DFLASH_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DFL_CUDA(launch_zero(at<void>(ws, off_cnt), pl.counters * 4, st), "counter reset");
+  DFL_CUDA(launch_gemm(j, pl, at<float>(ws, off_part), at<uint32_t>(ws, off_cnt),
+                       status_word(ws), st),
+           "LM head logits GEMM");
+  return DFLASH_OK;
+}
+
+dflash_status dflash_sample(const dflash_config* cfg, int64_t M, const float* logits,
+                            uint64_t seed, uint32_t offset, int32_t* tok, float* logq, float* lse,
+                            void* stream) {
+  dflash_status s = check_config(cfg);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(M >= 0 && M < (int64_t(1) << 31), DFLASH_EINVAL, "M out of range");
+  if (M == 0) return DFLASH_OK;
+  DFL_CHECK(logits != nullptr && tok != nullptr, DFLASH_EINVAL, "logits / tok is NULL");
+  DFL_ALIGNED(logits, 4, "logits");
+  DFL_ALIGNED(tok, 4, "tok");
+  DFL_ALIGNED(logq, 4, "logq");
+  DFL_ALIGNED(lse, 4, "lse");
+  DFL_CUDA(launch_sample_rows(logits, M, cfg->vocab, seed, offset, cfg->block, nullptr, nullptr,
+                              tok, logq, lse, static_cast<cudaStream_t>(stream)),
+           "sampling kernel");
+  return DFLASH_OK;
+}
+
+dflash_status dflash_accept_stochastic(int32_t R, int32_t B, int32_t V, const int32_t* draft,
+                                       const float* draft_logits, const float* draft_lse,
+                                       const float* target_logp, uint64_t seed, uint32_t offset,
+                                       int32_t* n_acc, int32_t* out_tok, void* ws,
+                                       size_t ws_bytes, void* stream) {
+  DFL_CHECK(R >= 0, DFLASH_EINVAL, "R must be >= 0");
+  DFL_CHECK(B >= 1 && B <= kMaxBlock, DFLASH_EINVAL, "B must be in [1, %d], got %d", kMaxBlock, B);
+  DFL_CHECK(V >= 2, DFLASH_EINVAL, "V must be >= 2, got %d", V);
+  if (R == 0) return DFLASH_OK;
+  DFL_CHECK(R < (1 << 26), DFLASH_EINVAL, "R too large for the random-number counters");
+  DFL_CHECK(draft && draft_logits && draft_lse && target_logp && n_acc && out_tok, DFLASH_EINVAL,
+            "a pointer argument is NULL");
+  DFL_ALIGNED(draft, 4, "draft");
+  DFL_ALIGNED(draft_logits, 4, "draft_logits");
+  DFL_ALIGNED(draft_lse, 4, "draft_lse");
+  DFL_ALIGNED(target_logp, 4, "target_logp");
+  DFL_ALIGNED(n_acc, 4, "n_acc");
+  DFL_ALIGNED(out_tok, 4, "out_tok");
+  dflash_status s = check_ws(ws, ws_bytes, sizeof(DevStatus) + static_cast<size_t>(R) * 8);
+  if (s != DFLASH_OK) return s;
+  DFL_CUDA(launch_accept_stochastic(R, B, V, draft, draft_logits, draft_lse, target_logp, seed,
+                                    offset, n_acc, out_tok,
+                                    at<unsigned long long>(ws, sizeof(DevStatus)),
+                                    static_cast<cudaStream_t>(stream)),
+           "stochastic accept");
+  return DFLASH_OK;
+}
+
 dflash_status dflash_accept(int32_t R, int32_t K, int32_t B, const int32_t* draft,
                             const int32_t* target, int32_t* n_acc, int32_t* best_k,
                             int32_t* out_tok, void* stream) {
@@ -637,7 +717,21 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
       DFL_PTR(a->v_cache[i], "v_cache[i]");
     }
   }
-  if (a->target_tokens) {
+  DFL_CHECK(a->sample == 0 || a->sample == 1, DFLASH_EINVAL, "sample must be 0 or 1");
+  const bool sampling = a->sample == 1;
+  if (sampling) {
+    DFL_CHECK(a->draft_logits != nullptr, DFLASH_EINVAL, "sample = 1 needs draft_logits");
+    DFL_ALIGNED(a->draft_logits, 16, "draft_logits");
+    DFL_ALIGNED(a->draft_logq, 4, "draft_logq");
+    DFL_ALIGNED(a->target_logp, 4, "target_logp");
+    if (a->target_logp) {
+      DFL_CHECK(a->n_cand == 1 && a->n_blocks == a->n_req, DFLASH_EINVAL,
+                "stochastic verification takes one candidate per request (n_cand = 1)");
+      DFL_CHECK(a->n_acc && a->out_tok, DFLASH_EINVAL, "n_acc / out_tok is NULL");
+      DFL_CHECK(a->n_req < (1 << 26), DFLASH_EINVAL, "n_req too large for the counters");
+    }
+  }
+  if (a->target_tokens && !sampling) {
     DFL_CHECK(a->n_cand >= 1 && a->n_cand <= 32 && a->n_blocks == a->n_req * a->n_cand,
               DFLASH_EINVAL, "verification needs n_blocks == n_req * n_cand (n_cand in [1,32])");
     DFL_CHECK(a->n_acc && a->best_k && a->out_tok, DFLASH_EINVAL,
@@ -745,6 +839,25 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
       return s;
   }
   DFL_CUDA(launch_rmsnorm(dt, h, M, H, w->g_final, c->rms_eps, x, st), "final rmsnorm");
+  if (sampling) {
+    // temperature 1: logits to the caller's buffer, a Gumbel-max draw per
+    // slot, then (optionally) stochastic verification
+    float* row_lse = at<float>(ws, L.row_lse);
+    s = run_job(job_logits(c, x, M, w->lm_head, a->draft_logits), partial, counters, status, st,
+                "LM head logits GEMM");
+    if (s != DFLASH_OK) return s;
+    DFL_CUDA(launch_sample_rows(a->draft_logits, M, c->vocab, a->seed, a->rng_offset, c->block,
+                                a->block_tokens, a->known_len, a->draft_tokens, a->draft_logq,
+                                row_lse, st),
+             "sampling kernel");
+    if (a->target_logp) {
+      DFL_CUDA(launch_accept_stochastic(a->n_req, c->block, c->vocab, a->draft_tokens,
+                                        a->draft_logits, row_lse, a->target_logp, a->seed,
+                                        a->rng_offset, a->n_acc, a->out_tok, keys, st),
+               "stochastic accept");
+    }
+    return DFLASH_OK;
+  }
   float2* lse = a->confidence ? at<float2>(ws, L.lse) : nullptr;
   DFL_CUDA(launch_lmhead_argmax(dt, w->lm_head, c->vocab, x, M, H, keys, status, st, partial,
                                 counters, lse),

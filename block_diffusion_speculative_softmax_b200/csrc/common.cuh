@@ -341,3 +341,45 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
 }
 
 }  // namespace dfl
+
+namespace dfl {
+
+// ---------------------------------------------------------------------------
+// Counter-based random numbers: Philox4x32 with 10 rounds (Salmon, Moraes,
+// Dror and Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011).
+// A round multiplies c0 by M0 and c2 by M1 (64-bit products, hi/lo halves)
+// and outputs (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0); the key is bumped by
+// the Weyl constants between rounds.
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+    const uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
+    const uint32_t hi1 = static_cast<uint32_t>(p1 >> 32), lo1 = static_cast<uint32_t>(p1);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// Purpose tags of the counters (fourth word): ASCII "DRFT", "ACPT", "RESD".
+constexpr uint32_t kRngDraft = 0x44524654u;
+constexpr uint32_t kRngAccept = 0x41435054u;
+constexpr uint32_t kRngResid = 0x52455344u;
+
+// 32-bit word -> U = (floor(x / 2^9) + 1/2) / 2^23, an odd multiple of 2^-24
+// in (0, 1); the integer 2 floor(x / 2^9) + 1 < 2^24 converts exactly.
+__device__ __forceinline__ float uniform_from_word(uint32_t x) {
+  return __uint2float_rn(((x >> 9) << 1) | 1u) * 5.9604644775390625e-8f;
+}
+// Standard Gumbel variate -log(-log U).
+__device__ __forceinline__ float gumbel_from_word(uint32_t x) {
+  return -logf(-logf(uniform_from_word(x)));
+}
+
+}  // namespace dfl

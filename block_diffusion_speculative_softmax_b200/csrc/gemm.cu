@@ -474,6 +474,142 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
   }
 }
 
+// Epilogue of one token row of a token-major tile: thread = token t (valid
+// when tv), features f0 .. f0 + BW - 1 of segment S; cols(c, v) yields the
+// accumulator columns [c, c + 16) of the row.  ARGMAX: argmax key (and the
+// tile's log-sum-exp share); else the segment's op (SwiGLU halves, residual
+// row, or a store with optional RoPE over heads and row scatter).
+template <int BW, bool ARGMAX, typename ColsFn>
+__device__ __forceinline__ void tok_row_epilogue(const Params& p, const Seg& S, int tile, int f0,
+                                                 int t, bool tv, ColsFn&& cols) {
+  if constexpr (ARGMAX) {
+    unsigned long long best = 0ull;
+    float mx = -INFINITY, se = 0.f;   // running log-sum-exp share of this tile
+#pragma unroll 1
+    for (int c = 0; c < BW; c += 16) {
+      float v[16];
+      cols(c, v);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const int f = f0 + c + q;
+        if (f < S.rows) {
+          if (!isfinite(v[q]) && tv) report(p.status, DFLASH_ENUMERIC, 35);
+          const unsigned long long k = argmax_key(v[q], static_cast<uint32_t>(f));
+          best = k > best ? k : best;
+          if (v[q] > mx) {
+            se = se * __expf(mx - v[q]) + 1.f;
+            mx = v[q];
+          } else {
+            se += __expf(v[q] - mx);
+          }
+        }
+      }
+    }
+    if (tv && best) atomicMax(p.keys + t, best);
+    if (tv && p.lse != nullptr) p.lse[static_cast<size_t>(tile) * p.M + t] = make_float2(mx, se);
+  } else if (S.op == EPI_SWIGLU) {
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out) + static_cast<int64_t>(t) * S.out_stride;
+#pragma unroll 1
+    for (int c = 0; c < BW / 2; c += 16) {
+      float g[16], u[16];
+      cols(c, g);
+      cols(BW / 2 + c, u);
+      if (tv) {
+        alignas(16) __nv_bfloat16 r[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) r[q] = __float2bfloat16_rn(g[q] / (1.f + __expf(-g[q])) * u[q]);
+        const int f = f0 + c;
+        if (f + 16 <= S.rows) {
+          reinterpret_cast<uint4*>(o + f)[0] = reinterpret_cast<const uint4*>(r)[0];
+          reinterpret_cast<uint4*>(o + f)[1] = reinterpret_cast<const uint4*>(r)[1];
+        } else {
+          for (int q = 0; q < 16 && f + q < S.rows; ++q) o[f + q] = r[q];
+        }
+      }
+    }
+  } else if (S.op == EPI_RESID) {
+    float* h = static_cast<float*>(S.out) + static_cast<int64_t>(t) * S.out_stride;
+#pragma unroll 1
+    for (int c = 0; c < BW; c += 16) {
+      float v[16];
+      cols(c, v);
+      const int f = f0 + c;
+      if (tv) {
+        if (f + 16 <= S.rows) {
+#pragma unroll
+          for (int q = 0; q < 16; q += 4) {
+            float4 a = *reinterpret_cast<float4*>(h + f + q);
+            a.x += v[q]; a.y += v[q + 1]; a.z += v[q + 2]; a.w += v[q + 3];
+            *reinterpret_cast<float4*>(h + f + q) = a;
+          }
+        } else {
+          for (int q = 0; q < 16 && f + q < S.rows; ++q) h[f + q] += v[q];
+        }
+      }
+    }
+  } else {   // EPI_STORE, optional RoPE over heads of head_dim
+    const int64_t orow = tv ? (S.use_dst ? p.dst[t] : t) : 0;
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out) + orow * S.out_stride;
+    const int d = p.head_dim, half = d >> 1;
+    const int pos = (tv && S.rope) ? p.pos[t] : 0;
+    auto put16 = [&](int f, const float* v) {
+      if (S.op == EPI_STORE_F32) {
+        float* of = static_cast<float*>(S.out) + orow * S.out_stride;
+        if (f + 16 <= S.rows) {
+#pragma unroll
+          for (int q = 0; q < 16; q += 4)
+            *reinterpret_cast<float4*>(of + f + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+        } else {
+          for (int q = 0; q < 16 && f + q < S.rows; ++q) of[f + q] = v[q];
+        }
+        return;
+      }
+      alignas(16) __nv_bfloat16 r[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) r[q] = __float2bfloat16_rn(v[q]);
+      if (f + 16 <= S.rows) {
+        reinterpret_cast<uint4*>(o + f)[0] = reinterpret_cast<const uint4*>(r)[0];
+        reinterpret_cast<uint4*>(o + f)[1] = reinterpret_cast<const uint4*>(r)[1];
+      } else {
+        for (int q = 0; q < 16 && f + q < S.rows; ++q) o[f + q] = r[q];
+      }
+    };
+    if (S.rope) {
+      // 16 frequencies at a time: one (cos, sin) set serves that chunk of
+      // every head in the tile; chunk c of a head's first half pairs with
+      // chunk c + d/2
+#pragma unroll 1
+      for (int i0 = 0; i0 < half; i0 += 16) {
+        float2 cs[16];
+        if (tv) rope_cs16(p, pos, i0, cs);
+#pragma unroll 1
+        for (int c = i0; c < BW; c += d) {
+          float a[16], b[16];
+          cols(c, a);
+          cols(c + half, b);
+          if (tv) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const float x1 = a[q], x2 = b[q];
+              a[q] = x1 * cs[q].x - x2 * cs[q].y;
+              b[q] = x2 * cs[q].x + x1 * cs[q].y;
+            }
+            put16(f0 + c, a);
+            put16(f0 + c + half, b);
+          }
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int c = 0; c < BW; c += 16) {
+        float v[16];
+        cols(c, v);
+        if (tv) put16(f0 + c, v);
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Token-major variant for M >= 128 tokens (the context K/V projection over
 // L rows, and every GEMM when many blocks are drafted together): the TOKENS
@@ -721,132 +857,7 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
   };
 
   if (do_op) {
-    if constexpr (ARGMAX) {
-      unsigned long long best = 0ull;
-      float mx = -INFINITY, se = 0.f;   // running log-sum-exp share of this tile
-#pragma unroll 1
-      for (int c = 0; c < BW; c += 16) {
-        float v[16];
-        cols(c, v);
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const int f = f0 + c + q;
-          if (f < S.rows) {
-            if (!isfinite(v[q]) && tv) report(p.status, DFLASH_ENUMERIC, 35);
-            const unsigned long long k = argmax_key(v[q], static_cast<uint32_t>(f));
-            best = k > best ? k : best;
-            if (v[q] > mx) {
-              se = se * __expf(mx - v[q]) + 1.f;
-              mx = v[q];
-            } else {
-              se += __expf(v[q] - mx);
-            }
-          }
-        }
-      }
-      if (tv && best) atomicMax(p.keys + t, best);
-      if (tv && p.lse != nullptr) p.lse[static_cast<size_t>(tile) * p.M + t] = make_float2(mx, se);
-    } else if (S.op == EPI_SWIGLU) {
-      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out) + static_cast<int64_t>(t) * S.out_stride;
-#pragma unroll 1
-      for (int c = 0; c < BW / 2; c += 16) {
-        float g[16], u[16];
-        cols(c, g);
-        cols(BW / 2 + c, u);
-        if (tv) {
-          alignas(16) __nv_bfloat16 r[16];
-#pragma unroll
-          for (int q = 0; q < 16; ++q) r[q] = __float2bfloat16_rn(g[q] / (1.f + __expf(-g[q])) * u[q]);
-          const int f = f0 + c;
-          if (f + 16 <= S.rows) {
-            reinterpret_cast<uint4*>(o + f)[0] = reinterpret_cast<const uint4*>(r)[0];
-            reinterpret_cast<uint4*>(o + f)[1] = reinterpret_cast<const uint4*>(r)[1];
-          } else {
-            for (int q = 0; q < 16 && f + q < S.rows; ++q) o[f + q] = r[q];
-          }
-        }
-      }
-    } else if (S.op == EPI_RESID) {
-      float* h = static_cast<float*>(S.out) + static_cast<int64_t>(t) * S.out_stride;
-#pragma unroll 1
-      for (int c = 0; c < BW; c += 16) {
-        float v[16];
-        cols(c, v);
-        const int f = f0 + c;
-        if (tv) {
-          if (f + 16 <= S.rows) {
-#pragma unroll
-            for (int q = 0; q < 16; q += 4) {
-              float4 a = *reinterpret_cast<float4*>(h + f + q);
-              a.x += v[q]; a.y += v[q + 1]; a.z += v[q + 2]; a.w += v[q + 3];
-              *reinterpret_cast<float4*>(h + f + q) = a;
-            }
-          } else {
-            for (int q = 0; q < 16 && f + q < S.rows; ++q) h[f + q] += v[q];
-          }
-        }
-      }
-    } else {   // EPI_STORE, optional RoPE over heads of head_dim
-      const int64_t orow = tv ? (S.use_dst ? p.dst[t] : t) : 0;
-      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out) + orow * S.out_stride;
-      const int d = p.head_dim, half = d >> 1;
-      const int pos = (tv && S.rope) ? p.pos[t] : 0;
-      auto put16 = [&](int f, const float* v) {
-        if (S.op == EPI_STORE_F32) {
-          float* of = static_cast<float*>(S.out) + orow * S.out_stride;
-          if (f + 16 <= S.rows) {
-#pragma unroll
-            for (int q = 0; q < 16; q += 4)
-              *reinterpret_cast<float4*>(of + f + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
-          } else {
-            for (int q = 0; q < 16 && f + q < S.rows; ++q) of[f + q] = v[q];
-          }
-          return;
-        }
-        alignas(16) __nv_bfloat16 r[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) r[q] = __float2bfloat16_rn(v[q]);
-        if (f + 16 <= S.rows) {
-          reinterpret_cast<uint4*>(o + f)[0] = reinterpret_cast<const uint4*>(r)[0];
-          reinterpret_cast<uint4*>(o + f)[1] = reinterpret_cast<const uint4*>(r)[1];
-        } else {
-          for (int q = 0; q < 16 && f + q < S.rows; ++q) o[f + q] = r[q];
-        }
-      };
-      if (S.rope) {
-        // 16 frequencies at a time: one (cos, sin) set serves that chunk of
-        // every head in the tile; chunk c of a head's first half pairs with
-        // chunk c + d/2
-#pragma unroll 1
-        for (int i0 = 0; i0 < half; i0 += 16) {
-          float2 cs[16];
-          if (tv) rope_cs16(p, pos, i0, cs);
-#pragma unroll 1
-          for (int c = i0; c < BW; c += d) {
-            float a[16], b[16];
-            cols(c, a);
-            cols(c + half, b);
-            if (tv) {
-#pragma unroll
-              for (int q = 0; q < 16; ++q) {
-                const float x1 = a[q], x2 = b[q];
-                a[q] = x1 * cs[q].x - x2 * cs[q].y;
-                b[q] = x2 * cs[q].x + x1 * cs[q].y;
-              }
-              put16(f0 + c, a);
-              put16(f0 + c + half, b);
-            }
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < BW; c += 16) {
-          float v[16];
-          cols(c, v);
-          if (tv) put16(f0 + c, v);
-        }
-      }
-    }
+    tok_row_epilogue<BW, ARGMAX>(p, S, tile, f0, t, tv, cols);
     if (p.splits > 1 && tid == 0) p.counters[tile_lin] = 0u;
   }
   tc_fence_before();
@@ -864,6 +875,213 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
     tc_fence_after();
     if constexpr (TWO) tmem_dealloc_pair(tmem, TMEM_COLS);
     else tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Persistent token-major GEMM on CTA pairs (many tiles, no K split).  One
+// cluster of two CTAs per pair of SMs walks the pair tiles t = pair,
+// pair + pairs, ... (same raster as the non-persistent kernel).  Warp 0
+// streams TMA stages through the ring without stopping at tile boundaries,
+// warp 1 of the even CTA issues the pair MMAs, and warps 2..5 of both CTAs
+// drain the accumulator: TMEM holds TWO 256-column accumulators, so tile
+// i's epilogue (tcgen05.ld, RoPE / SwiGLU / residual / argmax, global
+// stores) runs while tile i + 1 accumulates in the other buffer.  The
+// accumulator-empty barrier lives in the even CTA and counts one arrival
+// per CTA (each CTA's 128 epilogue threads meet at a named barrier first).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+               ::"r"(bar_cluster_addr) : "memory");
+}
+
+template <bool ARGMAX>
+__global__ void __launch_bounds__(192, 1) gemm_tokp_kernel(const __grid_constant__ Params p,
+                                                           const int n_tiles) {
+  constexpr int BW = 256;
+  constexpr int STAGES = 6;
+  constexpr int X_BYTES = BM * BK * 2;        // 128 tokens x 64 k
+  constexpr int W_BYTES = (BW / 2) * BK * 2;  // this CTA's half of the 256 feature rows
+  constexpr int STAGE = X_BYTES + W_BYTES;
+  constexpr uint32_t TMEM_COLS = 2 * BW;
+  constexpr uint32_t IDESC = idesc_bf16(2 * BM, BW);
+  constexpr int EPI = 128;
+  static_assert(STAGE % 1024 == 0, "stages must stay 1024-byte aligned");
+
+  extern __shared__ uint8_t dsmem[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t accf_bar[2];
+  __shared__ __align__(8) uint64_t acce_bar[2];
+  __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int pairs = static_cast<int>(gridDim.x >> 1);
+  const int nkb = p.kb_total;
+  const int tok_pairs = static_cast<int>((p.M + 2 * BM - 1) / (2 * BM));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf_bar[b], 1);
+      mbar_init(&acce_bar[b], 2);   // one arrival per CTA of the pair
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+    for (int g = 0; g < p.nseg; ++g) {
+      tma_prefetch_desc(&p.tm[p.seg[g].map]);
+      if (p.seg[g].pair) tma_prefetch_desc(&p.tm[p.seg[g].map + 1]);
+    }
+    tma_prefetch_desc(&p.tm_x);
+  }
+  if (warp == 2) tmem_alloc_pair(&tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();   // both CTAs' barriers exist before copies or commits reach them
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  if (threadIdx.x == 0) pdl_launch();
+
+  // pair tile -> (feature tile, pair of token tiles)
+  auto decode = [&](int t, int& ftile, int& tp) {
+    if (p.tok_fast) {
+      tp = t % tok_pairs;
+      ftile = t / tok_pairs;
+    } else {
+      ftile = t % p.row_tiles;
+      tp = t / p.row_tiles;
+    }
+  };
+  auto seg_of = [&](int ftile) {
+    int sg = 0;
+    while (sg + 1 < p.nseg && ftile >= p.seg[sg + 1].tile_begin) ++sg;
+    return sg;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs): its token rows and its
+      // half of the feature rows; the even CTA's stage barrier counts both
+      pdl_wait();
+      int s = 0;
+      uint32_t ph = 0;
+      for (int t = pair; t < n_tiles && !abort_flag; t += pairs) {
+        int ftile, tp;
+        decode(t, ftile, tp);
+        const Seg& S = p.seg[seg_of(ftile)];
+        const int f0 = (ftile - S.tile_begin) * (S.pair ? BW / 2 : BW);
+        const int tok0 = (2 * tp + static_cast<int>(rank)) * BM;
+        const CUtensorMap* tmw = S.pair ? &p.tm[S.map + (rank ? 1 : 0)] : &p.tm[S.map];
+        const int wrow = S.pair ? f0 : f0 + static_cast<int>(rank) * (BW / 2);
+        const int rot = tp % nkb;
+        for (int i = 0; i < nkb; ++i) {
+          if (!mbar_wait(&empty_bar[s], ph ^ 1, p.status, 51)) {
+            abort_flag = 1;
+            break;
+          }
+          int kb = i + rot;
+          if (kb >= nkb) kb -= nkb;
+          const uint32_t fb = rank ? dsmem_addr(smem_u32(&full_bar[s]), 0)
+                                   : smem_u32(&full_bar[s]);
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * STAGE);
+          uint8_t* st = smem + s * STAGE;
+          tma_load_2d_pair(st + X_BYTES, tmw, fb, kb * BK, wrow);
+          tma_load_2d_pair(st, &p.tm_x, fb, kb * BK, tok0);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (even CTA)
+      int s = 0;
+      uint32_t ph = 0;
+      int i = 0;
+      for (int t = pair; t < n_tiles; t += pairs, ++i) {
+        const int b = i & 1;
+        if (!abort_flag && !mbar_wait(&acce_bar[b], ((i >> 1) & 1) ^ 1, p.status, 52))
+          abort_flag = 1;
+        tc_fence_after();
+        for (int k = 0; k < nkb; ++k) {
+          if (!abort_flag && !mbar_wait(&full_bar[s], ph, p.status, 53)) abort_flag = 1;
+          if (!abort_flag) {
+            tc_fence_after();
+            const uint8_t* st = smem + s * STAGE;
+            const uint64_t da = smem_desc_sw128(st);
+            const uint64_t db = smem_desc_sw128(st + X_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < BK / UK; ++kk)
+              tc_mma_bf16_pair(tmem + b * BW, da + 2 * kk, db + 2 * kk, IDESC,
+                               (k > 0 || kk > 0) ? 1u : 0u);
+            tc_commit_pair(&empty_bar[s]);
+          }
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        tc_commit_pair(&accf_bar[b]);   // also after an abort, so nobody waits long
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 (both CTAs): TMEM lane = token row
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t acce0 = dsmem_addr(smem_u32(&acce_bar[0]), 0);
+    const uint32_t acce1 = dsmem_addr(smem_u32(&acce_bar[1]), 0);
+    pdl_wait();
+    int i = 0;
+    for (int t = pair; t < n_tiles; t += pairs, ++i) {
+      const int b = i & 1;
+      const bool ok = mbar_wait(&accf_bar[b], (i >> 1) & 1, p.status, 54);
+      tc_fence_after();
+      int ftile, tp;
+      decode(t, ftile, tp);
+      const Seg& S = p.seg[seg_of(ftile)];
+      const int f0 = (ftile - S.tile_begin) * (S.pair ? BW / 2 : BW);
+      const int tok = (2 * tp + static_cast<int>(rank)) * BM + r;
+      const bool tv = tok < p.M;
+      const uint32_t acc = lane_addr + static_cast<uint32_t>(b * BW);
+      if (ok && !abort_flag) {
+        auto cols = [&](int c, float* v) { tmem_ld16(acc + c, v); };
+        tok_row_epilogue<BW, ARGMAX>(p, S, ftile, f0, tok, tv, cols);
+      }
+      tc_fence_before();
+      named_sync(1, EPI);
+      if (threadIdx.x == 64) mbar_arrive_cluster(b ? acce1 : acce0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (abort_flag) {
+    // give copies that the other CTA issued against this CTA's barriers
+    // time to land (bounded) before the pair tears down
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) __nanosleep(1000);
+  }
+  cluster_sync_all();   // neither CTA frees TMEM or exits while the other works
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
@@ -892,12 +1110,6 @@ __device__ __forceinline__ int sk_cta_of(int64_t units, int grid, int64_t u) {
   return static_cast<int>(((u + 1) * grid - 1) / units);
 }
 
-__device__ __forceinline__ void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 
 template <int BN, int STAGES, bool ARGMAX>
 __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__ Params p,
@@ -1390,6 +1602,40 @@ cudaError_t launch_tok2(const Params& p, dim3 grid, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, gemm_tok_kernel<256, STAGES, ARGMAX, true>, p);
 }
 
+// Persistent CTA-pair launch: one cluster of two CTAs per pair of SMs.
+template <bool ARGMAX>
+cudaError_t launch_tokp(const Params& p, int n_tiles, cudaStream_t st) {
+  constexpr int SMEM = 6 * (BM * BK * 2 + 128 * BK * 2) + 1024;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_tokp_kernel<ARGMAX>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const int pairs = std::min(n_tiles, kNumSMs / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, gemm_tokp_kernel<ARGMAX>, p, n_tiles);
+}
+
+// The persistent kernel pays off once there is more than one wave of pair
+// tiles (otherwise every pair runs a single tile anyway).
+inline bool use_persistent(int pair_tiles) { return pair_tiles > kNumSMs / 2; }
+
 // Token tiles on grid x when there are fewer of them than feature tiles (and
 // the feature tiles fit grid y): the weights then stream from HBM once.
 inline bool tok_fast(int tok_tiles, int feature_tiles) {
@@ -1839,6 +2085,8 @@ cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& pl, float* partial,
     p.tok_fast = tc::tok_fast(pl.tok_tiles, tiles);
     if (pl.two) {
       const int tt = (pl.tok_tiles + 1) & ~1;   // whole pairs; a spare tile is all padding
+      if (tc::use_persistent(tiles * (tt / 2)))
+        return tc::launch_tokp<false>(p, tiles * (tt / 2), st);
       return tc::launch_tok2<false>(p, dim3(static_cast<unsigned>(tiles) * tt), st);
     }
     if (p.tok_fast) grid = dim3(pl.tok_tiles, tiles, pl.splits);
@@ -1897,6 +2145,8 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V, const void* X,
     p.tok_fast = tc::tok_fast(tt, p.row_tiles);
     if (two) {
       const int te = (tt + 1) & ~1;
+      if (tc::use_persistent(p.row_tiles * (te / 2)))
+        return tc::launch_tokp<true>(p, p.row_tiles * (te / 2), st);
       return tc::launch_tok2<true>(p, dim3(static_cast<unsigned>(p.row_tiles) * te), st);
     }
     const dim3 grid = p.tok_fast ? dim3(tt, p.row_tiles, 1) : dim3(p.row_tiles, tt, 1);

@@ -165,6 +165,18 @@ cudaError_t launch_accept(int R, int K, int B, const int32_t* draft,
 cudaError_t launch_d2sd(int R, int B, int K, int mask_id, const int32_t* base,
                         const float* conf, int32_t* known_len, int32_t* cand,
                         int32_t* block_req, cudaStream_t st);
+// Temperature-1 sampling (sampling.cu): Gumbel-max draw per stored logit
+// row (row ids 0..M-1 select the noise); known-prefix slots keep their input.
+cudaError_t launch_sample_rows(const float* logits, int64_t M, int V, uint64_t seed,
+                               uint32_t offset, int B, const int32_t* block_tokens,
+                               const int32_t* known_len, int32_t* tok, float* logq,
+                               float* lse, cudaStream_t st);
+// Stochastic acceptance of one candidate per request; keys [R] scratch.
+cudaError_t launch_accept_stochastic(int R, int B, int V, const int32_t* draft,
+                                     const float* draft_logits, const float* draft_lse,
+                                     const float* target_logp, uint64_t seed, uint32_t offset,
+                                     int32_t* n_acc, int32_t* out_tok,
+                                     unsigned long long* keys, cudaStream_t st);
 cudaError_t launch_wait_selftest(uint32_t* status, int64_t limit_ns,
                                  cudaStream_t st);
 

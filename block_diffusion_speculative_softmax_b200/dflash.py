@@ -79,7 +79,9 @@ class StepArgs(C.Structure):
                 ("max_logit", C.c_void_p), ("confidence", C.c_void_p),
                 ("target_tokens", C.c_void_p),
                 ("n_cand", C.c_int32), ("n_acc", C.c_void_p), ("best_k", C.c_void_p),
-                ("out_tok", C.c_void_p)]
+                ("out_tok", C.c_void_p), ("sample", C.c_int32), ("rng_offset", C.c_uint32),
+                ("seed", C.c_uint64), ("draft_logits", C.c_void_p), ("draft_logq", C.c_void_p),
+                ("target_logp", C.c_void_p)]
 
 
 _VP, _I32, _I64, _SZ = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
@@ -101,6 +103,10 @@ SIGNATURES = {
                                     _VP, _SZ, _VP]),
     "dflash_mlp": (C.c_int, [_CFG, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "dflash_lmhead_argmax": (C.c_int, [_CFG, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "dflash_lmhead_logits": (C.c_int, [_CFG, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "dflash_sample": (C.c_int, [_CFG, _I64, _VP, C.c_uint64, C.c_uint32, _VP, _VP, _VP, _VP]),
+    "dflash_accept_stochastic": (C.c_int, [_I32, _I32, _I32, _VP, _VP, _VP, _VP, C.c_uint64,
+                                           C.c_uint32, _VP, _VP, _VP, _SZ, _VP]),
     "dflash_accept": (C.c_int, [_I32, _I32, _I32, _VP, _VP, _VP, _VP, _VP, _VP]),
     "dflash_d2sd_candidates": (C.c_int, [_I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP, _VP,
                                          _VP]),
@@ -248,6 +254,25 @@ def dflash_lmhead_argmax_noalloc(cfg: Config, x, w_lm, tok, max_logit=None, stre
                                                _p(tok), _p(max_logit), _stream(stream)))
 
 
+def dflash_lmhead_logits(cfg: Config, x, w_lm, logits, ws, stream=None):
+    _check(load().dflash_lmhead_logits(C.byref(cfg), x.shape[0], _p(x), _p(w_lm), _p(logits),
+                                       _p(ws), ws.numel(), _stream(stream)))
+
+
+def dflash_sample(cfg: Config, logits, seed: int, offset: int, tok, logq=None, lse=None,
+                  stream=None):
+    _check(load().dflash_sample(C.byref(cfg), logits.shape[0], _p(logits), seed, offset,
+                                _p(tok), _p(logq), _p(lse), _stream(stream)))
+
+
+def dflash_accept_stochastic(draft, draft_logits, draft_lse, target_logp, seed: int,
+                             offset: int, n_acc, out_tok, ws, stream=None):
+    R, B, V = draft_logits.shape
+    _check(load().dflash_accept_stochastic(R, B, V, _p(draft), _p(draft_logits), _p(draft_lse),
+                                           _p(target_logp), seed, offset, _p(n_acc),
+                                           _p(out_tok), _p(ws), ws.numel(), _stream(stream)))
+
+
 def dflash_accept(draft: torch.Tensor, target: torch.Tensor, n_acc, best_k, out_tok,
                   stream=None):
     R, K, B = draft.shape
@@ -352,13 +377,25 @@ class StepBuffers:
         self.n_acc = torch.zeros(self.R, dtype=torch.int32, device=device)
         self.best_k = torch.zeros(self.R, dtype=torch.int32, device=device)
         self.out_tok = torch.zeros(self.R, B, dtype=torch.int32, device=device)
+        self.draft_logits = None      # temperature-1 mode buffers (alloc_sampling)
+        self.draft_logq = None
+        self.target_logp = None
+
+    def alloc_sampling(self, device="cuda"):
+        """Buffers of the temperature-1 mode: the draft's logits and log
+        probabilities per slot and the target's log probabilities."""
+        B, V = self.cfg.block, self.cfg.vocab
+        self.draft_logits = torch.zeros(self.nb, B, V, dtype=torch.float32, device=device)
+        self.draft_logq = torch.zeros(self.nb, B, dtype=torch.float32, device=device)
+        self.target_logp = torch.zeros(self.nb, B, V, dtype=torch.float32, device=device)
 
 
 def dflash_draft_step(cfg: Config, w: DeviceWeights, buf: StepBuffers,
                       new_states: Optional[torch.Tensor], ws: torch.Tensor,
                       new_off: Optional[torch.Tensor] = None,
                       ctx_cached: Optional[torch.Tensor] = None, verify: bool = False,
-                      stream=None, confidence: bool = False):
+                      stream=None, confidence: bool = False, sample: bool = False,
+                      seed: int = 0, rng_offset: int = 0):
     """One draft step over ``buf``'s blocks.  ``new_states`` [n_new][T][H]
     holds the target states of the context rows to (re)compute: all rows
     (``ctx_cached`` None) or rows [cached_r, L_r) of every request."""
@@ -385,5 +422,13 @@ def dflash_draft_step(cfg: Config, w: DeviceWeights, buf: StepBuffers,
     a.n_acc = buf.n_acc.data_ptr()
     a.best_k = buf.best_k.data_ptr()
     a.out_tok = buf.out_tok.data_ptr()
+    if sample:
+        a.sample = 1
+        a.seed = seed
+        a.rng_offset = rng_offset
+        a.draft_logits = buf.draft_logits.data_ptr()
+        a.draft_logq = buf.draft_logq.data_ptr()
+        a.target_logp = buf.target_logp.data_ptr() if verify else None
+        a.target_tokens = None
     _check(load().dflash_draft_step(C.byref(cfg), C.byref(w.struct), C.byref(a), _p(ws),
                                     ws.numel(), _stream(stream)))

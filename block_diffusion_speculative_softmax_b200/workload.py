@@ -31,7 +31,7 @@ class Workload:
     def __init__(self, cfg: synth.DraftConfig, seed: int = 0, device: str = "cuda",
                  mode: str = "full", steady_new_rows: int = 6, host_weights: Optional[dict] = None,
                  keep_host: bool = False, ctx_lens: Optional[List[int]] = None,
-                 conf_source: str = "synthetic"):
+                 conf_source: str = "synthetic", sample: bool = False, rng_seed: int = 1):
         self.cfg = cfg
         self.seed = seed
         self.device = device
@@ -94,6 +94,13 @@ class Workload:
                 self.conf = torch.from_numpy(synth.make_confidence(cfg, seed)).to(device)
             self.cached_all = torch.tensor(self.ctx_lens, dtype=torch.int32, device=device)
         self.conf_source = conf_source if K > 1 else None
+        # temperature-1 mode: sampled drafts, stochastic verification
+        self.sample = sample
+        self.rng_seed = rng_seed
+        self.rng_offset = 0
+        if sample:
+            assert K == 1, "stochastic verification takes one candidate per request"
+            self.buf.alloc_sampling(device)
         nb_max = R * K
         self.ws_bytes = DF.dflash_workspace_size(self.ccfg, R, nb_max, n_new, max(self.ctx_lens))
         self.ws = DF.alloc_workspace(self.ws_bytes, device)
@@ -105,7 +112,8 @@ class Workload:
         DF.dflash_draft_step(self.ccfg, self.w, self.buf, self.new_states, self.ws,
                              new_off=self.new_off, ctx_cached=self.ctx_cached,
                              verify=verify, stream=stream,
-                             confidence=self.conf_source == "draft")
+                             confidence=self.conf_source == "draft", sample=self.sample,
+                             seed=self.rng_seed, rng_offset=self.rng_offset)
 
     def candidates(self, stream=None):
         """D2SD cuts from pass-1 tokens into the pass-2 block buffers."""
@@ -147,6 +155,21 @@ class Workload:
             t = synth.plant_targets(d, n, cfg.vocab, rng)
             self.buf.target_tokens.copy_(torch.from_numpy(t))
         return n
+
+    def plant_target_logp(self, sigma: float = 0.5, seed_offset: int = 0):
+        """Temperature-1 stand-in for the target model: its distribution for
+        slot j+1 is the draft's slot j+1 logits perturbed by N(0, sigma^2)
+        noise (so drafts are often, not always, accepted), and for the slot
+        after the block an unrelated random distribution; stored as log
+        probabilities.  Needs the draft logits of a previous step."""
+        b = self.buf
+        g = torch.Generator(device=b.draft_logits.device)
+        g.manual_seed(int(self.seed) * 1000003 + 7919 + seed_offset)
+        z = torch.empty_like(b.target_logp)
+        z[:, :-1] = b.draft_logits[:, 1:] + sigma * torch.randn(
+            b.draft_logits[:, 1:].shape, device=z.device, generator=g)
+        z[:, -1] = 2.0 * torch.randn(z[:, -1].shape, device=z.device, generator=g)
+        b.target_logp.copy_(torch.log_softmax(z, dim=-1))
 
     @property
     def final_buf(self):

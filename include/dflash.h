@@ -273,6 +273,57 @@ dflash_status dflash_lmhead_argmax_noalloc(const dflash_config* cfg, int64_t M,
                                            void* stream);
 
 /* ------------------------------------------------------------------------
+ * Temperature-1 drafting and stochastic verification
+ *
+ * DFlash summary, methodology step 3 (the standard speculative acceptance
+ * test, a comparison of log probabilities; the first rejected slot is filled
+ * by the target's own generation) and DFLARE summary, section 4 (stochastic
+ * decoding at temperature 1).  Readings: each drafted slot is sampled from
+ * the draft's softmax q_j by the Gumbel-max rule; slot j is accepted while
+ * log U_j < log p_j(d_j) - log q_j(d_j); the token at the first rejected
+ * slot is drawn from norm(max(0, p_j - q_j)) (the draw that keeps the
+ * emitted tokens distributed as the target's), and when every slot passes
+ * one more token is drawn from the target's distribution for the next slot.
+ * Every uniform is a Philox4x32-10 draw (Salmon et al., SC 2011) with key
+ * (seed low 32 bits, seed high 32 bits) and counter words (c0, c1, c2, c3):
+ *   draft noise, token row m, id v:      (v >> 2, m, offset, 0x44524654) word v & 3
+ *   acceptance, request r, slot j:       (j, r, offset, 0x41435054)      word 0
+ *   residual / next-slot noise, r, j, v: (v >> 2, 64 r + j, offset, 0x52455344) word v & 3
+ * and a word x becomes U = (floor(x / 2^9) + 1/2) / 2^23 in (0, 1); the
+ * Gumbel variate is -log(-log U).
+ * ----------------------------------------------------------------------*/
+
+/* LM head writing its logits: logits[m][v] = x[m] . w_lm[v] (fp32 [M][V]). */
+dflash_status dflash_lmhead_logits(const dflash_config* cfg, int64_t M,
+                                   const void* x, const void* w_lm,
+                                   float* logits, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/* Gumbel-max draw of every row of logits [M][V] (fp32):
+ *   tok[m] = argmax_v (logits[m][v] + G(seed, offset, m, v)) (lowest id on
+ *   an exact tie); logq[m] = logits[m][tok[m]] - lse[m] (nullable);
+ *   lse[m] = log sum_v exp(logits[m][v]) (nullable).  No workspace. */
+dflash_status dflash_sample(const dflash_config* cfg, int64_t M,
+                            const float* logits, uint64_t seed, uint32_t offset,
+                            int32_t* tok, float* logq, float* lse, void* stream);
+
+/* Stochastic acceptance, one candidate block per request.  draft [R][B]
+ * int32 (slot 0 = anchor); draft_logits [R][B][V] fp32 with row logsumexp
+ * draft_lse [R][B]; target_logp [R][B][V] fp32 log probabilities, row j =
+ * the target's distribution for slot j+1 (after reading slots 0..j).
+ *   n_acc[r] = accepted drafted slots; out_tok[r] = draft[r][1..n], the
+ *   drawn token, then -1 up to B.
+ * Needs 8 * R bytes of workspace after the header.  B <= 32. */
+dflash_status dflash_accept_stochastic(int32_t R, int32_t B, int32_t V,
+                                       const int32_t* draft,
+                                       const float* draft_logits,
+                                       const float* draft_lse,
+                                       const float* target_logp, uint64_t seed,
+                                       uint32_t offset, int32_t* n_acc,
+                                       int32_t* out_tok, void* ws,
+                                       size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * The whole draft step (+ optional verification)
  * ----------------------------------------------------------------------*/
 
@@ -299,6 +350,18 @@ typedef struct {
   int32_t* n_acc;              /* out [R] */
   int32_t* best_k;             /* out [R] */
   int32_t* out_tok;            /* out [R][B] */
+  /* Temperature-1 mode (see dflash_sample / dflash_accept_stochastic).
+   * sample = 0: greedy argmax drafting, greedy verification (the fields
+   * below are unused).  sample = 1: the LM head writes draft_logits, every
+   * drafted slot is a Gumbel-max draw (row ids b*B + s), and with
+   * target_logp set the step verifies stochastically (n_cand must be 1);
+   * target_tokens, max_logit and confidence are then unused. */
+  int32_t sample;
+  uint32_t rng_offset;         /* counter word c2 of every draw (e.g. the step number) */
+  uint64_t seed;               /* Philox key */
+  float* draft_logits;         /* out [nb][B][V] fp32 (required with sample = 1) */
+  float* draft_logq;           /* out [nb][B] (nullable): log q of each drafted token */
+  const float* target_logp;    /* [nb][B][V] fp32 (nullable: no verification) */
 } dflash_step_args;
 
 /* One draft step (DFlash summary, methodology step 2; DFLARE sections
