@@ -648,6 +648,37 @@ dflash_status dflash_d2sd_candidates(int32_t R, int32_t B, int32_t K, int32_t ma
   return DFLASH_OK;
 }
 
+dflash_status dflash_advance(const dflash_config* cfg, int32_t R, int32_t K, const int32_t* n_acc,
+                             const int32_t* best_k, const int32_t* out_tok,
+                             const void* verify_states, int32_t* ctx_len, const int64_t* ctx_off,
+                             void* new_states, int32_t* new_count, int32_t* block_tokens,
+                             int32_t* known_len, void* ws, size_t ws_bytes, void* stream) {
+  dflash_status s = check_config(cfg);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(R >= 0, DFLASH_EINVAL, "R must be >= 0");
+  DFL_CHECK(K >= 1 && K <= 32, DFLASH_EINVAL, "K must be in [1, 32], got %d", K);
+  if (R == 0) return DFLASH_OK;
+  DFL_CHECK(n_acc && out_tok && ctx_len && ctx_off && new_count && block_tokens && known_len,
+            DFLASH_EINVAL, "a pointer argument is NULL");
+  DFL_PTR(verify_states, "verify_states");
+  DFL_PTR(new_states, "new_states");
+  DFL_ALIGNED(n_acc, 4, "n_acc");
+  DFL_ALIGNED(best_k, 4, "best_k");
+  DFL_ALIGNED(out_tok, 4, "out_tok");
+  DFL_ALIGNED(ctx_len, 4, "ctx_len");
+  DFL_ALIGNED(ctx_off, 8, "ctx_off");
+  DFL_ALIGNED(new_count, 4, "new_count");
+  DFL_ALIGNED(block_tokens, 4, "block_tokens");
+  DFL_ALIGNED(known_len, 4, "known_len");
+  if ((s = check_ws(ws, ws_bytes, sizeof(DevStatus))) != DFLASH_OK) return s;
+  const int64_t row_bytes = static_cast<int64_t>(cfg->n_target_layers) * cfg->hidden * esize(cfg);
+  DFL_CUDA(launch_advance(R, K, cfg->block, row_bytes, n_acc, best_k, out_tok, verify_states,
+                          ctx_len, ctx_off, new_states, new_count, block_tokens, known_len,
+                          cfg->mask_token_id, status_word(ws), static_cast<cudaStream_t>(stream)),
+           "advance kernel");
+  return DFLASH_OK;
+}
+
 dflash_status dflash_selftest_wait_timeout(void* ws, size_t ws_bytes, int64_t limit_ns,
                                            void* stream) {
   dflash_status s = check_ws(ws, ws_bytes, sizeof(DevStatus));
@@ -717,6 +748,14 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
       DFL_PTR(a->v_cache[i], "v_cache[i]");
     }
   }
+  DFL_ALIGNED(a->ctx_len, 4, "ctx_len");
+  DFL_ALIGNED(a->new_count, 4, "new_count");
+  if (a->new_count) {
+    DFL_CHECK(a->ctx_len != nullptr, DFLASH_EINVAL, "new_count needs ctx_len");
+    DFL_CHECK(a->n_ctx_new == static_cast<int64_t>(a->n_req) * c->block, DFLASH_EINVAL,
+              "with new_count, n_ctx_new must be n_req * block (%lld != %d * %d)",
+              static_cast<long long>(a->n_ctx_new), a->n_req, c->block);
+  }
   DFL_CHECK(a->sample == 0 || a->sample == 1, DFLASH_EINVAL, "sample must be 0 or 1");
   const bool sampling = a->sample == 1;
   if (sampling) {
@@ -762,7 +801,8 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
 
   // positions, cache rows, and zeroed argmax keys / tile counters
   DFL_CUDA(launch_prep_rows(a->n_req, a->n_blocks, c->block, a->block_req, a->ctx_off,
-                            a->new_off, a->ctx_cached, a->n_ctx_new, blk_pos, new_pos, new_dst,
+                            a->new_off, a->ctx_cached, a->ctx_len, a->new_count, a->n_ctx_new,
+                            blk_pos, new_pos, new_dst,
                             at<uint32_t>(ws, L.zero), static_cast<int64_t>(L.zero_bytes / 4), st),
            "row bookkeeping");
   float2* rope_tab = at<float2>(ws, L.rope);
@@ -825,7 +865,7 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
     if (side) DFL_CUDA(cudaStreamWaitEvent(st, side->done[i], 0), "join context");
     DFL_CUDA(launch_attn(dt, ap, a->n_blocks, c->block, c->n_q_heads, c->n_kv_heads,
                          c->head_dim, q, kb, vb, a->k_cache[i], a->v_cache[i], a->ctx_off,
-                         a->block_req, attn, at<float>(ws, L.attn_ws), status, st),
+                         a->block_req, attn, at<float>(ws, L.attn_ws), status, st, a->ctx_len),
              "attention");
     if ((s = run_job(job_resid(c, l.w_o, attn, M, qd, h), partial, counters, status, st,
                      "O GEMM")) != DFLASH_OK)

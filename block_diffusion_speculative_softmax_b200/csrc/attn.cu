@@ -27,6 +27,7 @@ struct AttnParams {
   const void* kc;
   const void* vc;
   const int64_t* ctx_off;
+  const int32_t* ctx_len;    // nullable: rows of request r = ctx_len[r]
   const int32_t* block_req;
   int B, Hq, Hkv, G;
   int splits, chunk, rows_per_cta;
@@ -53,7 +54,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_simt_kernel(const AttnPa
   const int split = blockIdx.y;
   const int r = p.block_req[b];
   const int64_t c_begin = p.ctx_off[r];
-  const int64_t L = p.ctx_off[r + 1] - c_begin;
+  const int64_t L = p.ctx_len ? static_cast<int64_t>(p.ctx_len[r]) : p.ctx_off[r + 1] - c_begin;
   const int64_t k_lo = static_cast<int64_t>(split) * p.chunk;
   const int n_ctx = static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(L, k_lo + p.chunk) - k_lo));
   const int n_blk = split == 0 ? p.B : 0;
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnParams p) {
   const int split = blockIdx.y;
   const int r = p.block_req[b];
   const int64_t c_begin = p.ctx_off[r];
-  const int64_t L = p.ctx_off[r + 1] - c_begin;
+  const int64_t L = p.ctx_len ? static_cast<int64_t>(p.ctx_len[r]) : p.ctx_off[r + 1] - c_begin;
   const int64_t k_lo = static_cast<int64_t>(split) * p.chunk;
   const int n_ctx = static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(L, k_lo + p.chunk) - k_lo));
   const int total = n_ctx + (split == 0 ? p.B : 0);
@@ -665,12 +666,14 @@ static cudaError_t launch_bf16(const AttnParams& p, int cs, dim3 grid, size_t sm
 cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq, int Hkv, int d,
                         const void* q, const void* kb, const void* vb, const void* kc,
                         const void* vc, const int64_t* ctx_off, const int32_t* block_req,
-                        void* out, float* ws, uint32_t* status, cudaStream_t st) {
+                        void* out, float* ws, uint32_t* status, cudaStream_t st,
+                        const int32_t* ctx_len) {
   (void)status;
   if (nb <= 0) return cudaSuccess;
   AttnParams p{};
   p.q = q; p.kb = kb; p.vb = vb; p.kc = kc; p.vc = vc;
   p.ctx_off = ctx_off;
+  p.ctx_len = ctx_len;
   p.block_req = block_req;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = Hq / Hkv;
   p.splits = plan.splits;

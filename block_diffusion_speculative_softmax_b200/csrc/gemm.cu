@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
 #pragma unroll
           for (int q = 0; q < JU; ++q) {
             const int t = tok0 + j0 + q;
-            if (f >= S.rows || t >= p.M) continue;
+            if (f >= S.rows || t >= p.M || orow[q] < 0) continue;
             float v = st[(j0 + q) * SROW + tid];
             if (S.rope) {
               const float pv = st[(j0 + q) * SROW + prt];
@@ -548,7 +548,9 @@ __device__ __forceinline__ void tok_row_epilogue(const Params& p, const Seg& S, 
       }
     }
   } else {   // EPI_STORE, optional RoPE over heads of head_dim
+    // a negative destination row marks a token to skip
     const int64_t orow = tv ? (S.use_dst ? p.dst[t] : t) : 0;
+    tv = tv && orow >= 0;
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out) + orow * S.out_stride;
     const int d = p.head_dim, half = d >> 1;
     const int pos = (tv && S.rope) ? p.pos[t] : 0;
@@ -1462,7 +1464,7 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const int t = tok0 + j0 + q;
-              if (j0 + q >= BN || f >= S.rows || t >= p.M) continue;
+              if (j0 + q >= BN || f >= S.rows || t >= p.M || orow[q] < 0) continue;
               float x = st[(j0 + q) * SROW + et];
               if (S.rope) {
                 const float pv = st[(j0 + q) * SROW + prt];
@@ -1850,7 +1852,7 @@ __global__ void __launch_bounds__(256) finish_kernel(const __grid_constant__ Fin
       v = i < half ? v * cs - pv * sn : v * cs + pv * sn;
     }
     const int64_t orow = sg.use_dst ? p.dst[m] : m;
-    static_cast<float*>(sg.out)[orow * sg.out_stride + c] = v;
+    if (orow >= 0) static_cast<float*>(sg.out)[orow * sg.out_stride + c] = v;
   }
 }
 

@@ -106,10 +106,16 @@ cudaError_t launch_rmsnorm(int dtype, const float* h, int64_t M, int H,
                            const float* g, float eps, void* x, cudaStream_t st);
 cudaError_t launch_prep_rows(int R, int nb, int B, const int32_t* block_req,
                              const int64_t* ctx_off, const int64_t* new_off,
-                             const int32_t* ctx_cached, int64_t n_new,
+                             const int32_t* ctx_cached, const int32_t* ctx_len,
+                             const int32_t* new_count, int64_t n_new,
                              int32_t* blk_pos, int32_t* new_pos,
                              int64_t* new_dst, uint32_t* zero, int64_t n_zero,
                              cudaStream_t st);
+cudaError_t launch_advance(int R, int K, int B, int64_t row_bytes, const int32_t* n_acc,
+                           const int32_t* best_k, const int32_t* out_tok, const void* verify_states,
+                           int32_t* ctx_len, const int64_t* ctx_off, void* new_states,
+                           int32_t* new_count, int32_t* block_tokens, int32_t* known_len,
+                           int mask_id, uint32_t* status, cudaStream_t st);
 // tokens (+ max logit) from the argmax keys; resets the keys to zero.
 cudaError_t launch_argmax_finish(unsigned long long* keys, int64_t M,
                                  int B, const int32_t* block_tokens,
@@ -153,11 +159,14 @@ struct AttnPlan {
 AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d,
                    int64_t max_ctx_len);
 size_t attn_ws_bytes(const AttnPlan& p, int nb, int B, int Hq, int d);
+// ctx_len (nullable): request r has ctx_len[r] context rows from ctx_off[r]
+// (else ctx_off[r + 1] - ctx_off[r]).
 cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq,
                         int Hkv, int d, const void* q, const void* kb,
                         const void* vb, const void* kc, const void* vc,
                         const int64_t* ctx_off, const int32_t* block_req,
-                        void* out, float* ws, uint32_t* status, cudaStream_t st);
+                        void* out, float* ws, uint32_t* status, cudaStream_t st,
+                        const int32_t* ctx_len = nullptr);
 
 cudaError_t launch_accept(int R, int K, int B, const int32_t* draft,
                           const int32_t* target, int32_t* n_acc,

@@ -331,7 +331,9 @@ cudaError_t launch_rmsnorm(int dtype, const float* h, int64_t M, int H, const fl
 __global__ void prep_rows_kernel(int R, int nb, int B, const int32_t* __restrict__ block_req,
                                  const int64_t* __restrict__ ctx_off,
                                  const int64_t* __restrict__ new_off,
-                                 const int32_t* __restrict__ ctx_cached, int64_t n_new,
+                                 const int32_t* __restrict__ ctx_cached,
+                                 const int32_t* __restrict__ ctx_len,
+                                 const int32_t* __restrict__ new_count, int64_t n_new,
                                  int32_t* __restrict__ blk_pos, int32_t* __restrict__ new_pos,
                                  int64_t* __restrict__ new_dst, uint32_t* __restrict__ zero,
                                  int64_t n_zero) {
@@ -342,7 +344,25 @@ __global__ void prep_rows_kernel(int R, int nb, int B, const int32_t* __restrict
   for (int64_t i = tid; i < n_zero; i += stride) zero[i] = 0u;
   for (int64_t m = tid; m < static_cast<int64_t>(nb) * B; m += stride) {
     const int r = block_req[m / B];
-    blk_pos[m] = static_cast<int32_t>(ctx_off[r + 1] - ctx_off[r] + m % B);
+    const int64_t L = ctx_len ? static_cast<int64_t>(ctx_len[r]) : ctx_off[r + 1] - ctx_off[r];
+    blk_pos[m] = static_cast<int32_t>(L + m % B);
+  }
+  if (new_count != nullptr) {
+    // fixed slots: B per request, the first new_count[r] are the last rows
+    // of its context; the others are skipped (destination -1)
+    for (int64_t n = tid; n < n_new; n += stride) {
+      const int r = static_cast<int>(n / B), j = static_cast<int>(n % B);
+      const int c = new_count[r];
+      if (j < c) {
+        const int64_t p = static_cast<int64_t>(ctx_len[r]) - c + j;
+        new_pos[n] = static_cast<int32_t>(p);
+        new_dst[n] = ctx_off[r] + p;
+      } else {
+        new_pos[n] = 0;
+        new_dst[n] = -1;
+      }
+    }
+    return;
   }
   const int64_t* off = new_off ? new_off : ctx_off;
   for (int64_t n = tid; n < n_new; n += stride) {
@@ -359,7 +379,8 @@ __global__ void prep_rows_kernel(int R, int nb, int B, const int32_t* __restrict
 
 cudaError_t launch_prep_rows(int R, int nb, int B, const int32_t* block_req,
                              const int64_t* ctx_off, const int64_t* new_off,
-                             const int32_t* ctx_cached, int64_t n_new, int32_t* blk_pos,
+                             const int32_t* ctx_cached, const int32_t* ctx_len,
+                             const int32_t* new_count, int64_t n_new, int32_t* blk_pos,
                              int32_t* new_pos, int64_t* new_dst, uint32_t* zero, int64_t n_zero,
                              cudaStream_t st) {
   const int64_t work =
@@ -367,7 +388,8 @@ cudaError_t launch_prep_rows(int R, int nb, int B, const int32_t* block_req,
   if (work <= 0) return cudaSuccess;
   const int grid = static_cast<int>(std::min<int64_t>((work + 255) / 256, kNumSMs * 8));
   return launch_k(prep_rows_kernel, dim3(grid), dim3(256), 0, st, R, nb, B, block_req, ctx_off,
-                  new_off, ctx_cached, n_new, blk_pos, new_pos, new_dst, zero, n_zero);
+                  new_off, ctx_cached, ctx_len, new_count, n_new, blk_pos, new_pos, new_dst, zero,
+                  n_zero);
 }
 
 struct InvFreq {
@@ -558,6 +580,63 @@ cudaError_t launch_d2sd(int R, int B, int K, int mask_id, const int32_t* base, c
   const int wpb = 4;
   return launch_k(d2sd_kernel, dim3((R + wpb - 1) / wpb), dim3(wpb * 32), 0, st, R, B, K, mask_id,
                   base, conf, known_len, cand, block_req);
+}
+
+// ===========================================================================
+// Roll the speculative window forward on the device (DFlash summary,
+// methodology step 4): request r accepted n = n_acc[r] drafted tokens of
+// candidate k = best_k[r]; the target states of that block's slots 0..n
+// (anchor + accepted tokens, from the target's verification pass) become the
+// newest context rows, the context grows by n + 1 and the emitted token
+// out_tok[r][n] is the next anchor.  Grid (R, B): CTA (r, j) copies slot j.
+// ===========================================================================
+__global__ void advance_kernel(int R, int K, int B, int64_t row_bytes,
+                               const int32_t* __restrict__ n_acc,
+                               const int32_t* __restrict__ best_k,
+                               const int32_t* __restrict__ out_tok,
+                               const uint8_t* __restrict__ verify_states,
+                               int32_t* __restrict__ ctx_len, const int64_t* __restrict__ ctx_off,
+                               uint8_t* __restrict__ new_states, int32_t* __restrict__ new_count,
+                               int32_t* __restrict__ block_tokens, int32_t* __restrict__ known_len,
+                               int mask_id, uint32_t* status) {
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch();
+  const int r = blockIdx.x, j = blockIdx.y;
+  const int n = n_acc[r];
+  const int k = best_k ? best_k[r] : 0;
+  if (j <= n) {
+    const uint4* src = reinterpret_cast<const uint4*>(
+        verify_states + ((static_cast<int64_t>(r) * K + k) * B + j) * row_bytes);
+    uint4* dst = reinterpret_cast<uint4*>(new_states + (static_cast<int64_t>(r) * B + j) * row_bytes);
+    for (int64_t i = threadIdx.x; i < row_bytes / 16; i += blockDim.x) dst[i] = __ldg(src + i);
+  }
+  if (threadIdx.x == 0) {
+    block_tokens[static_cast<int64_t>(r) * B + j] =
+        j == 0 ? out_tok[static_cast<int64_t>(r) * B + n] : mask_id;
+    if (j == 0) {
+      const int64_t cap = ctx_off[r + 1] - ctx_off[r];
+      int64_t L = static_cast<int64_t>(ctx_len[r]) + n + 1;
+      if (L > cap) {   // the caller's capacity is exhausted: keep what fits
+        report(status, DFLASH_EINVAL, 61);
+        L = cap;
+      }
+      new_count[r] = static_cast<int32_t>(min(static_cast<int64_t>(n + 1), L - ctx_len[r]));
+      ctx_len[r] = static_cast<int32_t>(L);
+      known_len[r] = 1;
+    }
+  }
+}
+
+cudaError_t launch_advance(int R, int K, int B, int64_t row_bytes, const int32_t* n_acc,
+                           const int32_t* best_k, const int32_t* out_tok, const void* verify_states,
+                           int32_t* ctx_len, const int64_t* ctx_off, void* new_states,
+                           int32_t* new_count, int32_t* block_tokens, int32_t* known_len,
+                           int mask_id, uint32_t* status, cudaStream_t st) {
+  if (R <= 0) return cudaSuccess;
+  return launch_k(advance_kernel, dim3(R, B), dim3(256), 0, st, R, K, B, row_bytes, n_acc, best_k,
+                  out_tok, static_cast<const uint8_t*>(verify_states), ctx_len, ctx_off,
+                  static_cast<uint8_t*>(new_states), new_count, block_tokens, known_len, mask_id,
+                  status);
 }
 
 // ===========================================================================

@@ -81,7 +81,8 @@ class StepArgs(C.Structure):
                 ("n_cand", C.c_int32), ("n_acc", C.c_void_p), ("best_k", C.c_void_p),
                 ("out_tok", C.c_void_p), ("sample", C.c_int32), ("rng_offset", C.c_uint32),
                 ("seed", C.c_uint64), ("draft_logits", C.c_void_p), ("draft_logq", C.c_void_p),
-                ("target_logp", C.c_void_p)]
+                ("target_logp", C.c_void_p), ("ctx_len", C.c_void_p),
+                ("new_count", C.c_void_p)]
 
 
 _VP, _I32, _I64, _SZ = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
@@ -113,6 +114,8 @@ SIGNATURES = {
     "dflash_draft_step": (C.c_int, [_CFG, C.POINTER(Weights), C.POINTER(StepArgs), _VP, _SZ,
                                     _VP]),
     "dflash_selftest_wait_timeout": (C.c_int, [_VP, _SZ, _I64, _VP]),
+    "dflash_advance": (C.c_int, [_CFG, _I32, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                 _VP, _VP, _SZ, _VP]),
     "dflash_lmhead_argmax_noalloc": (C.c_int, [_CFG, _I64, _VP, _VP, _VP, _VP, _VP]),
 }
 
@@ -288,6 +291,17 @@ def dflash_d2sd_candidates(base_tokens, conf, K, mask_token_id, known_len, cand_
                                          _stream(stream)))
 
 
+def dflash_advance(cfg: Config, n_acc, best_k, out_tok, verify_states, ctx_len, ctx_off,
+                   new_states, new_count, block_tokens, known_len, ws, stream=None):
+    """Roll every request's window forward on the device (see dflash.h).
+    verify_states [R][K][B][T][H]; new_states [R][B][T][H]."""
+    R, K = verify_states.shape[0], verify_states.shape[1]
+    _check(load().dflash_advance(C.byref(cfg), R, K, _p(n_acc), _p(best_k), _p(out_tok),
+                                 _p(verify_states), _p(ctx_len), _p(ctx_off), _p(new_states),
+                                 _p(new_count), _p(block_tokens), _p(known_len), _p(ws),
+                                 ws.numel(), _stream(stream)))
+
+
 def dflash_selftest_wait_timeout(ws, limit_ns: int, stream=None):
     _check(load().dflash_selftest_wait_timeout(_p(ws), ws.numel(), limit_ns, _stream(stream)))
 
@@ -395,7 +409,10 @@ def dflash_draft_step(cfg: Config, w: DeviceWeights, buf: StepBuffers,
                       new_off: Optional[torch.Tensor] = None,
                       ctx_cached: Optional[torch.Tensor] = None, verify: bool = False,
                       stream=None, confidence: bool = False, sample: bool = False,
-                      seed: int = 0, rng_offset: int = 0):
+                      seed: int = 0, rng_offset: int = 0,
+                      ctx_len: Optional[torch.Tensor] = None,
+                      new_count: Optional[torch.Tensor] = None,
+                      max_ctx_len: Optional[int] = None):
     """One draft step over ``buf``'s blocks.  ``new_states`` [n_new][T][H]
     holds the target states of the context rows to (re)compute: all rows
     (``ctx_cached`` None) or rows [cached_r, L_r) of every request."""
@@ -404,7 +421,7 @@ def dflash_draft_step(cfg: Config, w: DeviceWeights, buf: StepBuffers,
     a.n_req = buf.R
     a.n_blocks = buf.nb
     a.n_ctx_new = n_new
-    a.max_ctx_len = buf.max_L
+    a.max_ctx_len = buf.max_L if max_ctx_len is None else max_ctx_len
     a.block_req = buf.block_req.data_ptr()
     a.block_tokens = buf.block_tokens.data_ptr()
     a.known_len = buf.known_len.data_ptr()
@@ -422,6 +439,8 @@ def dflash_draft_step(cfg: Config, w: DeviceWeights, buf: StepBuffers,
     a.n_acc = buf.n_acc.data_ptr()
     a.best_k = buf.best_k.data_ptr()
     a.out_tok = buf.out_tok.data_ptr()
+    a.ctx_len = None if ctx_len is None else ctx_len.data_ptr()
+    a.new_count = None if new_count is None else new_count.data_ptr()
     if sample:
         a.sample = 1
         a.seed = seed

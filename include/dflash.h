@@ -362,6 +362,17 @@ typedef struct {
   float* draft_logits;         /* out [nb][B][V] fp32 (required with sample = 1) */
   float* draft_logq;           /* out [nb][B] (nullable): log q of each drafted token */
   const float* target_logp;    /* [nb][B][V] fp32 (nullable: no verification) */
+  /* Device-resident lengths, for a decode loop that never reads back to the
+   * host between steps (see dflash_advance).  ctx_len (nullable): request r's
+   * context is the ctx_len[r] rows starting at cache row ctx_off[r], and
+   * ctx_off[r+1] - ctx_off[r] is its capacity; max_ctx_len must bound every
+   * ctx_len (it sizes the attention split).  new_count (nullable, needs
+   * ctx_len): new_states then holds B slots per request ([n_req][B][T][H],
+   * n_ctx_new = n_req * B), of which the first new_count[r] are the context
+   * rows ctx_len[r] - new_count[r] .. ctx_len[r] - 1; the other slots are
+   * skipped (new_off and ctx_cached are then unused). */
+  const int32_t* ctx_len;
+  const int32_t* new_count;
 } dflash_step_args;
 
 /* One draft step (DFlash summary, methodology step 2; DFLARE sections
@@ -377,6 +388,29 @@ dflash_status dflash_draft_step(const dflash_config* cfg,
                                 const dflash_weights* w,
                                 const dflash_step_args* a, void* ws,
                                 size_t ws_bytes, void* stream);
+
+/* Roll the speculative window forward on the device (DFlash summary,
+ * methodology step 4; D2SD summary, methodology step 5), after verification
+ * and before the next dflash_draft_step, with no host round trip.  For
+ * request r with n = n_acc[r] accepted tokens of candidate k = best_k[r]
+ * (best_k nullable = 0):
+ *   new_states[r][j] = verify_states[r][k][j]   for j = 0 .. n
+ *     (the target's hidden states of the verified block's anchor and
+ *     accepted slots, [T][H] each; layouts [R][K][B][T][H] and [R][B][T][H])
+ *   new_count[r] = n + 1;  ctx_len[r] += n + 1  (in place)
+ *   block_tokens[r] = (out_tok[r][n], mask, ..., mask);  known_len[r] = 1
+ * so that the next draft step, given ctx_len and new_count, fuses and
+ * projects exactly the n + 1 new rows and drafts from the new anchor.
+ * ctx_off [R+1] gives each request's cache capacity; a context that would
+ * outgrow it is clipped there and DFLASH_EINVAL is recorded in the
+ * workspace header (dflash_check reports it). */
+dflash_status dflash_advance(const dflash_config* cfg, int32_t R, int32_t K,
+                             const int32_t* n_acc, const int32_t* best_k,
+                             const int32_t* out_tok, const void* verify_states,
+                             int32_t* ctx_len, const int64_t* ctx_off,
+                             void* new_states, int32_t* new_count,
+                             int32_t* block_tokens, int32_t* known_len, void* ws,
+                             size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * Failure-detection self test
