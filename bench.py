@@ -58,8 +58,11 @@ def parse():
                     help="launch the step eagerly instead of replaying a CUDA graph")
     ap.add_argument("--profile", action="store_true",
                     help="eager steps inside an NVTX range 'dflash_step' (for ncu launch lists)")
-    ap.add_argument("--op", choices=["lmhead", "mlp", "ctxproj", "attn", "fuse"],
+    ap.add_argument("--op", choices=["lmhead", "mlp", "ctxproj", "attn", "fuse", "fcfuse",
+                                     "sample"],
                     help="time one entry point alone at the workload's shapes")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="--op: context rows (default: the workload's own sum of lengths)")
     return ap.parse_args()
 
 
@@ -654,6 +657,8 @@ def run_op(args):
     nb = cfg.n_req * cfg.n_cand
     M = nb * cfg.block
     lens = synth.ctx_lengths(cfg, args.seed)
+    if args.rows > 0:   # same shapes, fewer rows (small ncu captures)
+        lens = [max(1, args.rows // len(lens))] * len(lens)
     N = int(sum(lens))
     g = torch.Generator(device="cuda").manual_seed(args.seed)
 
@@ -697,6 +702,23 @@ def run_op(args):
         algo = 2 * N * kvd * e + 2 * M * qd * e + 2 * M * kvd * e
         flops = 4.0 * cfg.n_cand * N * cfg.block * qd
         kernel = "attn_mma_kernel<d, CS> (split-KV block attention, cluster merge)"
+    elif args.op == "fcfuse":
+        st = rnd(N, T, H)
+        wfc = rnd(H, T * H, scale=0.02)
+        gfc = torch.ones(H, device="cuda")
+        fused = torch.empty(N, H, dtype=dt, device="cuda")
+        ws = DF.alloc_workspace(DF.dflash_workspace_size(cc, cfg.n_req, nb, N, max(lens)))
+        call = lambda: DF.dflash_fc_fuse_ctx(cc, st, wfc, gfc, fused, ws)
+        algo = N * T * H * e + H * T * H * e + N * H * (e + 8)
+        flops = 2.0 * N * T * H * H
+        kernel = "FC fusion GEMM (fp32 epilogue) + rmsnorm_kernel"
+    elif args.op == "sample":
+        z = torch.randn(M, V, device="cuda", generator=g)
+        tok = torch.empty(M, dtype=torch.int32, device="cuda")
+        lq = torch.empty(M, device="cuda")
+        call = lambda: DF.dflash_sample(cc, z, 1, 0, tok, lq, None)
+        algo = M * V * 4 + M * 8
+        kernel = "sample_rows_kernel (Gumbel-max over stored logits)"
     else:  # fuse
         st = rnd(N, T, H)
         wf = torch.randn(D, T, device="cuda", generator=g)

@@ -21,6 +21,9 @@
 namespace dfl {
 
 struct AttnParams {
+  CUtensorMap tm_k;          // bf16 context cache [rows][Hkv][d] (3-D TMA map)
+  CUtensorMap tm_v;
+  uint32_t* status;
   const void* q;
   const void* kb;
   const void* vb;
@@ -202,30 +205,81 @@ __device__ __forceinline__ float4 dsmem_ld4(uint32_t addr) {
   return v;
 }
 
+// Context K/V tiles of 64 keys stream through TMA (cp.async.bulk.tensor on a
+// 3-D map [rows][Hkv][d] of the packed cache, one 64-dim box per 128-byte
+// swizzled sub-tile) into a 2-stage mbarrier ring; every full 64-key tile of
+// a split comes this way.  The split's ragged tail tile (fewer than 64
+// context keys) and, for split 0, the B block keys are gathered with
+// cp.async into a separate buffer with the same swizzled layout, so the TMA
+// never reads past the request's last row.  Sub-tile s of a 64-key tile is
+// 64 keys x 64 dims (8 KB); 16-byte chunk c of key k sits at chunk
+// c ^ (k & 7) of its 128-byte row (the TMA 128-byte swizzle), which keeps
+// the ldmatrix reads conflict-free.
+//
+// Splits: the CS CTAs of one (block, kv head, row chunk) divide THIS
+// request's context into CS near-equal 64-key-aligned slices, so ragged
+// requests spread their keys over all CTAs of their cluster.
+//
 // CS = 0: partials to global memory for the combine kernel.  CS = 1: one
 // split, normalised in registers.  CS >= 2: the grid's y extent is CS and
 // each cluster of CS CTAs (one per split) merges through shared memory.
+constexpr int kAttnStages = 2;
+constexpr uint64_t kMaxCacheRows = 1ull << 28;   // row extent of the K/V tensor maps
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+        "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// byte offset of 16-byte chunk `ch` of key `kk` in a swizzled 64-key tile
+__device__ __forceinline__ uint32_t tile_off(int kk, int ch) {
+  return static_cast<uint32_t>((ch >> 3) * 8192 + kk * 128 + (((ch & 7) ^ (kk & 7)) << 4));
+}
+
 template <int D, int CS>
-__global__ void __launch_bounds__(128) attn_mma_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ AttnParams p) {
   constexpr int CH = D / 8;                 // 16-byte chunks per key row
   constexpr int NT = kMmaKeys / 8;          // n-tiles of S per key tile
   constexpr int KS = D / 16;                // k-steps of Q K^T
   constexpr int DT = D / 8;                 // n-tiles of O
-  extern __shared__ __align__(128) uint8_t smraw[];
-  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smraw);        // [2][64][D]
-  __nv_bfloat16* sV = sK + 2 * kMmaKeys * D;                          // [2][64][D]
+  constexpr int TILE = kMmaKeys * D * 2;    // bytes of one K (or V) tile
+  constexpr int SUB = D / 64;               // 64-dim TMA boxes per tile
+  extern __shared__ __align__(1024) uint8_t smraw_[];
+  uint8_t* smraw = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smraw_) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smraw;                                // [stage][K tile | V tile]
+  uint8_t* man = smraw + kAttnStages * 2 * TILE;        // [K tile | V tile], cp.async
+  __shared__ __align__(8) uint64_t full[kAttnStages];
+  __shared__ volatile int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int i = 0; i < kAttnStages; ++i) mbar_init(&full[i], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+  }
+  __syncthreads();
   pdl_wait();
-  if (threadIdx.x == 0) pdl_launch();
+  if (tid == 0) pdl_launch();
   const int b = blockIdx.x / p.Hkv, g = blockIdx.x % p.Hkv;
   const int split = blockIdx.y;
+  const int nsplit = CS >= 1 ? CS : p.splits;
   const int r = p.block_req[b];
   const int64_t c_begin = p.ctx_off[r];
   const int64_t L = p.ctx_len ? static_cast<int64_t>(p.ctx_len[r]) : p.ctx_off[r + 1] - c_begin;
-  const int64_t k_lo = static_cast<int64_t>(split) * p.chunk;
-  const int n_ctx = static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(L, k_lo + p.chunk) - k_lo));
-  const int total = n_ctx + (split == 0 ? p.B : 0);
+  const int64_t chunk = ((L + nsplit - 1) / nsplit + kMmaKeys - 1) / kMmaKeys * kMmaKeys;
+  const int64_t k_lo = static_cast<int64_t>(split) * chunk;
+  const int n_ctx = static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(L, k_lo + chunk) - k_lo));
+  const int n_full = n_ctx / kMmaKeys;                 // TMA tiles
+  const int n_tail = n_ctx - n_full * kMmaKeys;        // keys of the gathered tail tile
+  const int n_blk = split == 0 ? p.B : 0;
   const int nrows_all = p.B * p.G;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, tq = lane & 3;
   const int rbase = blockIdx.z * kMmaRows + warp * 16;
   const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(p.q);
@@ -233,34 +287,43 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnParams p) {
   const __nv_bfloat16* VC = static_cast<const __nv_bfloat16*>(p.vc);
   const __nv_bfloat16* KB = static_cast<const __nv_bfloat16*>(p.kb);
   const __nv_bfloat16* VB = static_cast<const __nv_bfloat16*>(p.vb);
+  const int row0 = static_cast<int>(c_begin + k_lo);
 
-  auto load_tile = [&](int t, int buf) {
+  auto issue = [&](int t) {   // TMA of full tile t into stage t % kAttnStages
+    const int st = t % kAttnStages;
+    uint8_t* dst = ring + st * 2 * TILE;
+    mbar_arrive_expect_tx(&full[st], 2 * TILE);
+#pragma unroll
+    for (int sb = 0; sb < SUB; ++sb) {
+      tma_load_3d(dst + sb * 8192, &p.tm_k, &full[st], sb * 64, g, row0 + t * kMmaKeys);
+      tma_load_3d(dst + TILE + sb * 8192, &p.tm_v, &full[st], sb * 64, g, row0 + t * kMmaKeys);
+    }
+  };
+  // gather n keys (context rows from `first`, or block rows) into `man`
+  auto gather = [&](bool block_keys, int n) {
     for (int c = tid; c < kMmaKeys * CH; c += 128) {
       const int kk = c / CH, ch = c % CH;
-      const int key = t * kMmaKeys + kk;
-      const __nv_bfloat16* sk = KC;
-      const __nv_bfloat16* sv = VC;
+      const bool valid = kk < n;
+      const __nv_bfloat16* sk = KB;   // any valid address when nothing is read
+      const __nv_bfloat16* sv = VB;
       size_t off = 0;
-      const bool valid = key < total;
-      if (key < n_ctx) {
-        off = (static_cast<size_t>(c_begin + k_lo + key) * p.Hkv + g) * D + ch * 8;
+      if (valid && !block_keys) {
+        sk = KC;
+        sv = VC;
+        off = (static_cast<size_t>(row0 + n_full * kMmaKeys + kk) * p.Hkv + g) * D + ch * 8;
       } else if (valid) {
-        sk = KB;
-        sv = VB;
-        off = ((static_cast<size_t>(b) * p.B + (key - n_ctx)) * p.Hkv + g) * D + ch * 8;
-      } else {
-        sk = KB;   // any valid address; zero bytes are read
-        sv = VB;
+        off = ((static_cast<size_t>(b) * p.B + kk) * p.Hkv + g) * D + ch * 8;
       }
-      const int sw = (ch ^ (kk & 7)) * 8;
-      cp_async16(sK + (buf * kMmaKeys + kk) * D + sw, sk + off, valid);
-      cp_async16(sV + (buf * kMmaKeys + kk) * D + sw, sv + off, valid);
+      cp_async16(man + tile_off(kk, ch), sk + off, valid);
+      cp_async16(man + TILE + tile_off(kk, ch), sv + off, valid);
     }
     cp_async_commit();
   };
 
-  const int ntiles = (total + kMmaKeys - 1) / kMmaKeys;
-  if (ntiles > 0) load_tile(0, 0);
+  if (tid == 0)
+    for (int t = 0; t < n_full && t < kAttnStages; ++t) issue(t);
+  if (n_tail > 0) gather(false, n_tail);
+  else if (n_blk > 0) gather(true, n_blk);
 
   // Q fragments of this warp's 16 rows (rows past B*G read as zero)
   uint32_t qf[KS][4];
@@ -292,18 +355,8 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnParams p) {
   for (int i = 0; i < DT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
-  for (int t = 0; t < ntiles; ++t) {
-    const int buf = t & 1;
-    if (t + 1 < ntiles) {
-      load_tile(t + 1, buf ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const uint32_t kbase = smem_u32(sK + buf * kMmaKeys * D);
-    const uint32_t vbase = smem_u32(sV + buf * kMmaKeys * D);
-    // S = Q K^T  (16 rows x 64 keys per warp)
+  // one 64-key tile (K at kbase, V at vbase, swizzled), keys < nvalid count
+  auto process = [&](uint32_t kbase, uint32_t vbase, int nvalid) {
     float sc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -313,19 +366,17 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnParams p) {
         const int kk = nt * 8 + (lane & 7);
         const int ch = k2 * 2 + (lane >> 3);
         uint32_t b0, b1, b2, b3;
-        ldsm_x4(kbase + (kk * D + ((ch ^ (kk & 7)) * 8)) * 2, b0, b1, b2, b3);
+        ldsm_x4(kbase + tile_off(kk, ch), b0, b1, b2, b3);
         mma_bf16(sc[nt], qf[k2], b0, b1);
         mma_bf16(sc[nt], qf[k2 + 1], b2, b3);
       }
     }
-    // online softmax (rows gq and gq + 8 of the warp's 16)
-    const int key0 = t * kMmaKeys;
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const bool ok = key0 + nt * 8 + 2 * tq + e < total;
+        const bool ok = nt * 8 + 2 * tq + e < nvalid;
         sc[nt][e] = ok ? sc[nt][e] * sl2 : -INFINITY;
         sc[nt][e + 2] = ok ? sc[nt][e + 2] * sl2 : -INFINITY;
         mx0 = fmaxf(mx0, sc[nt][e]);
@@ -368,10 +419,48 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const AttnParams p) {
         const int key = kk * 16 + (mi & 1) * 8 + (lane & 7);
         const int ch = dt + (mi >> 1);
         uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vbase + (key * D + ((ch ^ (key & 7)) * 8)) * 2, b0, b1, b2, b3);
+        ldsm_x4_t(vbase + tile_off(key, ch), b0, b1, b2, b3);
         mma_bf16(o[dt], a, b0, b1);
         mma_bf16(o[dt + 1], a, b2, b3);
       }
+    }
+  };
+
+  // full context tiles through the TMA ring
+  int t = 0;
+  for (; t < n_full; ++t) {
+    const int st = t % kAttnStages;
+    // every thread waits (bounded); all reach the barrier, then leave together
+    if (!mbar_wait(&full[st], static_cast<uint32_t>((t / kAttnStages) & 1), p.status, 71))
+      abort_flag = 1;
+    __syncthreads();
+    if (abort_flag) break;
+    const uint32_t base = smem_u32(ring + st * 2 * TILE);
+    process(base, base + TILE, kMmaKeys);
+    __syncthreads();   // every warp is done with the stage before it is refilled
+    if (tid == 0 && t + kAttnStages < n_full) issue(t + kAttnStages);
+  }
+  if (abort_flag) {
+    // let TMA copies still in flight land before the CTA's shared memory goes away
+    if (tid == 0)
+      for (int q = t; q < n_full && q < t + kAttnStages; ++q)
+        mbar_wait(&full[q % kAttnStages], static_cast<uint32_t>((q / kAttnStages) & 1),
+                  p.status, 72);
+    cp_async_wait<0>();
+    __syncthreads();
+  } else {
+    // the gathered tail tile, then (split 0) the block keys
+    if (n_tail > 0) {
+      cp_async_wait<0>();
+      __syncthreads();
+      process(smem_u32(man), smem_u32(man + TILE), n_tail);
+      __syncthreads();
+      if (n_blk > 0) gather(true, n_blk);
+    }
+    if (n_blk > 0) {
+      cp_async_wait<0>();
+      __syncthreads();
+      process(smem_u32(man), smem_u32(man + TILE), n_blk);
     }
     __syncthreads();
   }
@@ -525,6 +614,12 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   out[idx] = from_f<T>(num / den);
 }
 
+// Dynamic shared memory of the bf16 kernel: the TMA ring, the gather buffer
+// and 1 KB of slack for the 1024-byte alignment of the swizzled tiles.
+static size_t attn_smem_bytes(int d) {
+  return static_cast<size_t>(kAttnStages * 2 + 2) * kMmaKeys * d * 2 + 1024;
+}
+
 // Opt every attention kernel into large dynamic shared memory once (on the
 // first call, which must come before any stream capture), allow the
 // 16-CTA clusters, and record the largest cluster the device can schedule.
@@ -562,7 +657,7 @@ static cudaError_t allow_smem() {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(1, 16, 1);
       cfg.blockDim = dim3(128);
-      cfg.dynamicSmemBytes = 2 * 2 * kMmaKeys * 128 * sizeof(__nv_bfloat16);
+      cfg.dynamicSmemBytes = attn_smem_bytes(128);
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
       attr[0].val.clusterDim.x = 1;
@@ -597,8 +692,11 @@ AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d, int64_t max
       p.chunk = 64;
       return p;
     }
+    // enough CTAs to fill the GPU twice, and at most ~512 context keys per
+    // CTA for the longest request (each request divides its own context)
     const int64_t max_splits = std::min<int64_t>(16, (max_ctx_len + 127) / 128);
-    const int64_t n = std::max<int64_t>(1, std::min(want, max_splits));
+    const int64_t by_keys = (max_ctx_len + 511) / 512;
+    const int64_t n = std::max<int64_t>(1, std::min(std::max(want, by_keys), max_splits));
     while (p.cluster < n) p.cluster *= 2;
     int64_t chunk = (max_ctx_len + p.cluster - 1) / p.cluster;
     p.chunk = static_cast<int>((chunk + 63) / 64 * 64);
@@ -668,7 +766,6 @@ cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq, 
                         const void* vc, const int64_t* ctx_off, const int32_t* block_req,
                         void* out, float* ws, uint32_t* status, cudaStream_t st,
                         const int32_t* ctx_len) {
-  (void)status;
   if (nb <= 0) return cudaSuccess;
   AttnParams p{};
   p.q = q; p.kb = kb; p.vb = vb; p.kc = kc; p.vc = vc;
@@ -681,6 +778,7 @@ cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq, 
   p.rows_per_cta = plan.rows_per_cta;
   p.scale = 1.0f / sqrtf(static_cast<float>(d));
   p.out = out;
+  p.status = status;
   const int64_t n_rows = static_cast<int64_t>(nb) * B * Hq;
   p.part_o = ws;
   p.part_ml = ws + static_cast<size_t>(n_rows) * plan.splits * d;
@@ -690,7 +788,15 @@ cudaError_t launch_attn(int dtype, const AttnPlan& plan, int nb, int B, int Hq, 
   int cs = 0;   // 0: partials through global memory + combine kernel
   if (dtype == DFLASH_BF16) {
     cs = plan.cluster <= g_max_cluster ? plan.cluster : 0;
-    const size_t smem = 2 * 2 * static_cast<size_t>(kMmaKeys) * d * sizeof(__nv_bfloat16);
+    // context K/V as 3-D tensors [rows][Hkv][d]; only rows of the requests'
+    // contexts are ever loaded, so the row extent is an upper bound
+    // (kMaxCacheRows, far above any cache this path is sized for)
+    const void* kbase = kc ? kc : kb;
+    const void* vbase = vc ? vc : vb;
+    if (!encode_tmap_bf16_3d(&p.tm_k, kbase, d, Hkv, kMaxCacheRows, 64, 1, kMmaKeys) ||
+        !encode_tmap_bf16_3d(&p.tm_v, vbase, d, Hkv, kMaxCacheRows, 64, 1, kMmaKeys))
+      return cudaErrorInvalidValue;
+    const size_t smem = attn_smem_bytes(d);
     e = d == 64 ? launch_bf16<64>(p, cs, grid, smem, st) : launch_bf16<128>(p, cs, grid, smem, st);
     if (e != cudaSuccess || cs != 0) return e;
   } else {

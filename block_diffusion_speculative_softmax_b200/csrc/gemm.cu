@@ -263,7 +263,8 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
   const bool ok = mbar_wait(&acc_bar, 0, p.status, 14);
   tc_fence_after();
   pdl_wait();
-  const bool live = ok && !abort_flag;
+  // warp-uniform: the tcgen05.ld below is a warp-wide instruction
+  const bool live = __all_sync(0xffffffffu, ok && !abort_flag);
   const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
 
   if constexpr (ARGMAX) {
@@ -806,7 +807,8 @@ __global__ void __launch_bounds__(128, 1) gemm_tok_kernel(const __grid_constant_
   const bool ok = mbar_wait(&acc_bar, 0, p.status, 34);
   tc_fence_after();
   pdl_wait();
-  const bool live = ok && !abort_flag;
+  // warp-uniform: the tcgen05.ld below is a warp-wide instruction
+  const bool live = __all_sync(0xffffffffu, ok && !abort_flag);
   const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
   const int t = tok0 + tid;
   const bool tv = t < p.M;
@@ -1063,7 +1065,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tokp_kernel(const __grid_constant
       const int tok = (2 * tp + static_cast<int>(rank)) * BM + r;
       const bool tv = tok < p.M;
       const uint32_t acc = lane_addr + static_cast<uint32_t>(b * BW);
-      if (ok && !abort_flag) {
+      if (__all_sync(0xffffffffu, ok && !abort_flag)) {   // warp-wide tcgen05.ld below
         auto cols = [&](int c, float* v) { tmem_ld16(acc + c, v); };
         tok_row_epilogue<BW, ARGMAX>(p, S, ftile, f0, tok, tv, cols);
       }
@@ -1896,6 +1898,21 @@ bool encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner,
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                         uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  EncodeFn fn = get_encode();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

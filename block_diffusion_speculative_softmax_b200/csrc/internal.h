@@ -192,5 +192,8 @@ cudaError_t launch_wait_selftest(uint32_t* status, int64_t limit_ns,
 // Tensor maps (driver entry point fetched through the runtime).
 bool encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner,
                          uint64_t outer, uint32_t box_inner, uint32_t box_outer);
+// 3-D bf16 map, dims (d0 fastest, d1, d2), dense strides, 128-byte swizzle.
+bool encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                         uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2);
 
 }  // namespace dfl

@@ -190,7 +190,9 @@ dflash_status dflash_kv_project(const dflash_config* cfg, const void* x,
  * q, out [nb*B][Hq][d]; k_blk, v_blk [nb*B][Hkv][d]; k_ctx, v_ctx packed
  * [sum L][Hkv][d]; ctx_off device [R+1] int64 row offsets of each request's
  * context (L_r = ctx_off[r+1] - ctx_off[r], may be 0); block_req device [nb]
- * int32; max_ctx_len = max_r L_r (host, sizes the split-KV grid). */
+ * int32; max_ctx_len = max_r L_r (host, sizes the split-KV grid).  The
+ * packed caches may hold at most 2^28 rows (bf16 path: the TMA tensor maps
+ * over them span that many rows). */
 dflash_status dflash_block_attn(const dflash_config* cfg, int32_t n_blocks,
                                 const void* q, const void* k_blk,
                                 const void* v_blk, const void* k_ctx,
