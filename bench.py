@@ -508,7 +508,7 @@ def run_ours(args):
             steps2 = max(5, min(args.steps, 30))
             ms2, g2, _ = measure_step(w2, args, stream, steps2, max(3, args.warmup), 1)
             del g2
-            t2, _ = accepted_tokens(w2, stream, n2, 4)
+            t2, _ = accepted_tokens(w2, stream, n2, 16)
             r2 = kernel_table(w2, c2, DF, peaks, stream, 10, ms2)
             d2 = dominant(r2)
             per_config[name] = {"ms_per_step": ms2, "blocks_s": w2.final_buf.nb / (ms2 / 1e3),

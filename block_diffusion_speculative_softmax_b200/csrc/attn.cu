@@ -210,8 +210,8 @@ __device__ __forceinline__ float4 dsmem_ld4(uint32_t addr) {
 // swizzled sub-tile) into a 2-stage mbarrier ring; every full 64-key tile of
 // a split comes this way.  The split's ragged tail tile (fewer than 64
 // context keys) and, for split 0, the B block keys are gathered with
-// cp.async into a separate buffer with the same swizzled layout, so the TMA
-// never reads past the request's last row.  Sub-tile s of a 64-key tile is
+// cp.async, in the same swizzled layout, into ring stages that no TMA will
+// write again, so the TMA never reads past the request's last row.  Sub-tile s of a 64-key tile is
 // 64 keys x 64 dims (8 KB); 16-byte chunk c of key k sits at chunk
 // c ^ (k & 7) of its 128-byte row (the TMA 128-byte swizzle), which keeps
 // the ldmatrix reads conflict-free.
@@ -242,7 +242,7 @@ __device__ __forceinline__ uint32_t tile_off(int kk, int ch) {
 }
 
 template <int D, int CS>
-__global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(128, 3) attn_mma_kernel(const __grid_constant__ AttnParams p) {
   constexpr int CH = D / 8;                 // 16-byte chunks per key row
   constexpr int NT = kMmaKeys / 8;          // n-tiles of S per key tile
   constexpr int KS = D / 16;                // k-steps of Q K^T
@@ -253,7 +253,6 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
   uint8_t* smraw = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smraw_) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smraw;                                // [stage][K tile | V tile]
-  uint8_t* man = smraw + kAttnStages * 2 * TILE;        // [K tile | V tile], cp.async
   __shared__ __align__(8) uint64_t full[kAttnStages];
   __shared__ volatile int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -299,8 +298,12 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
       tma_load_3d(dst + TILE + sb * 8192, &p.tm_v, &full[st], sb * 64, g, row0 + t * kMmaKeys);
     }
   };
-  // gather n keys (context rows from `first`, or block rows) into `man`
-  auto gather = [&](bool block_keys, int n) {
+  // gather n keys (the ragged context tail, or the block rows) into ring
+  // stage `st` once no TMA is pending on it: the tail goes to the stage that
+  // tile n_full would use (free after tile n_full - 2), the block keys to the
+  // other one (free after tile n_full - 1)
+  auto gather = [&](bool block_keys, int n, int st) {
+    uint8_t* man = ring + st * 2 * TILE;
     for (int c = tid; c < kMmaKeys * CH; c += 128) {
       const int kk = c / CH, ch = c % CH;
       const bool valid = kk < n;
@@ -320,10 +323,11 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
     cp_async_commit();
   };
 
+  const int st_tail = n_full & 1, st_blk = (n_full + 1) & 1;
   if (tid == 0)
     for (int t = 0; t < n_full && t < kAttnStages; ++t) issue(t);
-  if (n_tail > 0) gather(false, n_tail);
-  else if (n_blk > 0) gather(true, n_blk);
+  if (n_tail > 0 && n_full <= 1) gather(false, n_tail, st_tail);
+  if (n_blk > 0 && n_full == 0) gather(true, n_blk, st_blk);
 
   // Q fragments of this warp's 16 rows (rows past B*G read as zero)
   uint32_t qf[KS][4];
@@ -426,24 +430,30 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
     }
   };
 
-  // full context tiles through the TMA ring
+  // full context tiles through the TMA ring; one block barrier per tile
   int t = 0;
   for (; t < n_full; ++t) {
     const int st = t % kAttnStages;
-    // every thread waits (bounded); all reach the barrier, then leave together
-    if (!mbar_wait(&full[st], static_cast<uint32_t>((t / kAttnStages) & 1), p.status, 71))
-      abort_flag = 1;
-    __syncthreads();
-    if (abort_flag) break;
-    const uint32_t base = smem_u32(ring + st * 2 * TILE);
-    process(base, base + TILE, kMmaKeys);
+    // every thread waits (bounded); a warp computes only if all its lanes saw
+    // the tile, and every warp reaches the barrier below either way
+    const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((t / kAttnStages) & 1),
+                              p.status, 71);
+    if (!ok) abort_flag = 1;
+    if (__all_sync(0xffffffffu, ok)) {
+      const uint32_t base = smem_u32(ring + st * 2 * TILE);
+      process(base, base + TILE, kMmaKeys);
+    }
     __syncthreads();   // every warp is done with the stage before it is refilled
+    if (abort_flag) break;
     if (tid == 0 && t + kAttnStages < n_full) issue(t + kAttnStages);
+    // the stages freed for good take the gathered tiles
+    if (t == n_full - 2 && n_tail > 0) gather(false, n_tail, st_tail);
+    if (t == n_full - 1 && n_blk > 0) gather(true, n_blk, st_blk);
   }
   if (abort_flag) {
     // let TMA copies still in flight land before the CTA's shared memory goes away
     if (tid == 0)
-      for (int q = t; q < n_full && q < t + kAttnStages; ++q)
+      for (int q = t; q < n_full && q <= t + 1; ++q)   // tiles t, t + 1 may be in flight
         mbar_wait(&full[q % kAttnStages], static_cast<uint32_t>((q / kAttnStages) & 1),
                   p.status, 72);
     cp_async_wait<0>();
@@ -451,16 +461,17 @@ __global__ void __launch_bounds__(128) attn_mma_kernel(const __grid_constant__ A
   } else {
     // the gathered tail tile, then (split 0) the block keys
     if (n_tail > 0) {
-      cp_async_wait<0>();
+      if (n_blk > 0) cp_async_wait<1>();   // the block keys may still be landing
+      else cp_async_wait<0>();
       __syncthreads();
-      process(smem_u32(man), smem_u32(man + TILE), n_tail);
-      __syncthreads();
-      if (n_blk > 0) gather(true, n_blk);
+      process(smem_u32(ring + st_tail * 2 * TILE), smem_u32(ring + st_tail * 2 * TILE + TILE),
+              n_tail);
     }
     if (n_blk > 0) {
       cp_async_wait<0>();
       __syncthreads();
-      process(smem_u32(man), smem_u32(man + TILE), n_blk);
+      process(smem_u32(ring + st_blk * 2 * TILE), smem_u32(ring + st_blk * 2 * TILE + TILE),
+              n_blk);
     }
     __syncthreads();
   }
@@ -614,10 +625,11 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   out[idx] = from_f<T>(num / den);
 }
 
-// Dynamic shared memory of the bf16 kernel: the TMA ring, the gather buffer
-// and 1 KB of slack for the 1024-byte alignment of the swizzled tiles.
+// Dynamic shared memory of the bf16 kernel: the TMA ring (which also takes
+// the gathered tiles) and 1 KB of slack for the 1024-byte alignment of the
+// swizzled tiles.
 static size_t attn_smem_bytes(int d) {
-  return static_cast<size_t>(kAttnStages * 2 + 2) * kMmaKeys * d * 2 + 1024;
+  return static_cast<size_t>(kAttnStages * 2) * kMmaKeys * d * 2 + 1024;
 }
 
 // Opt every attention kernel into large dynamic shared memory once (on the

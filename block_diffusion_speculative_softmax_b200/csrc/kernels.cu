@@ -27,7 +27,7 @@ struct FuseGains {
 };
 
 constexpr int kFuseThreads = 512;
-constexpr int kFuseSmemBudget = 200 * 1024;
+constexpr int kFuseSmemBudget = 221 * 1024;
 
 template <typename T, int MAXD>
 __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ __align__(8) uint64_t full[8];
   __shared__ float alpha[kMaxLayers][kMaxTargetLayers];
-  __shared__ float red[2][32][MAXD];
+  __shared__ __align__(16) float red[2][MAXD][32];   // per-warp partial sums, layer-major
   __shared__ volatile int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nwarps = (blockDim.x + 31) >> 5;
@@ -128,7 +128,25 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
     for (int i = 0; i < MAXD; ++i) {
       if (i < D) {
         const float v = warp_sum(ss[i]);
-        if (lane == 0) red[par][warp][i] = v;
+        if (lane == 0) red[par][i][warp] = v;
+      }
+    }
+    // the gain does not enter the norm: apply it now, so its loads overlap
+    // the reductions and the barrier instead of following them
+    if (active && !abort_flag) {
+#pragma unroll
+      for (int i = 0; i < MAXD; ++i) {
+        if (i < D) {
+          const float4* g4 = reinterpret_cast<const float4*>(gains.g[i] + col);
+#pragma unroll
+          for (int q = 0; q < VE / 4; ++q) {
+            const float4 gv = __ldg(g4 + q);
+            u[i][4 * q] *= gv.x;
+            u[i][4 * q + 1] *= gv.y;
+            u[i][4 * q + 2] *= gv.z;
+            u[i][4 * q + 3] *= gv.w;
+          }
+        }
       }
     }
     __syncthreads();   // the slot is consumed and the per-warp sums are visible
@@ -143,19 +161,25 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
 #pragma unroll
       for (int i = 0; i < MAXD; ++i) {
         if (i < D) {
-          // all per-warp partials loaded first, then a short add tree
-          float part[32];
+          // the per-warp partials of layer i as float4 loads (warps past
+          // nwarps wrote nothing: their slots are masked), then a short tree
+          const float4* r4 = reinterpret_cast<const float4*>(red[par][i]);
+          float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int w = 0; w < 32; ++w) part[w] = w < nwarps ? red[par][w][i] : 0.f;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-            for (int w = 0; w < o; ++w) part[w] += part[w + o];
-          const float sc = rsqrtf(part[0] / static_cast<float>(H) + eps);
-          const float* g = gains.g[i] + col;
+          for (int w4 = 0; w4 < 8; ++w4) {
+            if (4 * w4 < nwarps) {
+              float4 t = r4[w4];
+              if (4 * w4 + 1 >= nwarps) t.y = 0.f;
+              if (4 * w4 + 2 >= nwarps) t.z = 0.f;
+              if (4 * w4 + 3 >= nwarps) t.w = 0.f;
+              acc4.x += t.x; acc4.y += t.y; acc4.z += t.z; acc4.w += t.w;
+            }
+          }
+          const float sc = rsqrtf(((acc4.x + acc4.y) + (acc4.z + acc4.w)) /
+                                  static_cast<float>(H) + eps);
           float o[VE];
 #pragma unroll
-          for (int e = 0; e < VE; ++e) o[e] = u[i][e] * sc * __ldg(g + e);
+          for (int e = 0; e < VE; ++e) o[e] = u[i][e] * sc;
           V::store(fused + (static_cast<size_t>(i) * N + n) * H + col, o);
         }
       }
@@ -168,176 +192,15 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
   }
 }
 
-// ---------------------------------------------------------------------------
-// Tensor-core variant (bf16, D <= 8, T <= 16).  For one context row the D
-// fused vectors are U = alpha (D x T) * states (T x H): a product with K = T,
-// run on mma.sync m16n8k16 over n-tiles of 8 columns.  alpha is split into
-// bf16 halves hi + lo (hi = bf16(alpha), lo = bf16(alpha - hi)); rows 0..7
-// of the A operand hold hi and rows 8..15 hold lo, so one MMA yields both
-// halves and u = C[i] + C[i + 8] carries alpha to ~2^-17 while every product
-// of bf16 values is exact in the fp32 accumulator.  K rows past T read
-// state row 0 against zero A columns.
-//
-// The T state rows of a context row land in the ring by T bulk copies at a
-// padded stride (H*2 + 16 bytes) so the 8 rows an ldmatrix reads sit in
-// different banks.  Pass 1 forms u and the per-layer sums of squares; one
-// block barrier combines them; pass 2 forms u again (the MMAs are cheap),
-// scales by rsqrt(mean(u^2) + eps) and the gain, and stores bf16 pairs.  A
-// warp owns a contiguous run of n-tiles, so its stores of one layer row are
-// contiguous across consecutive n-tiles.  Gains sit in shared memory when
-// they fit beside the ring.
-// ---------------------------------------------------------------------------
-constexpr int kFuseMmaThreads = 256;
-
-template <bool GAINS_SMEM>
-__global__ void __launch_bounds__(kFuseMmaThreads) fuse_mma_kernel(
-    const __nv_bfloat16* __restrict__ states, int64_t N, int nT, int H, int D,
-    const float* __restrict__ w_fuse, const FuseGains gains, __nv_bfloat16* __restrict__ fused,
-    float eps, int slots, uint32_t* status) {
-  extern __shared__ __align__(128) uint8_t fsm[];
-  __shared__ __align__(8) uint64_t full[8];
-  __shared__ float alpha_s[kMaxLayers][kMaxTargetLayers];
-  __shared__ float red[2][8][kFuseMmaThreads / 32];
-  __shared__ volatile int abort_flag;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gq = lane >> 2, tq = lane & 3;
-  const uint32_t rs = static_cast<uint32_t>(H) * 2 + 16;       // padded state-row stride
-  const uint32_t slot_bytes = rs * static_cast<uint32_t>(nT);
-  const uint32_t row_bytes = static_cast<uint32_t>(H) * 2;
-  float* gs = reinterpret_cast<float*>(fsm + static_cast<size_t>(slots) * slot_bytes);
-  if (tid == 0) {
-    for (int s = 0; s < slots; ++s) mbar_init(&full[s], 1);
-    abort_flag = 0;
-    fence_mbar_init();
-  }
-  pdl_wait();
-  if (tid == 0) pdl_launch();
-  if (tid < D) {
-    float mx = -INFINITY;
-    for (int j = 0; j < nT; ++j) mx = fmaxf(mx, w_fuse[tid * nT + j]);
-    float sum = 0.f;
-    for (int j = 0; j < nT; ++j) {
-      const float e = expf(w_fuse[tid * nT + j] - mx);
-      alpha_s[tid][j] = e;
-      sum += e;
-    }
-    for (int j = 0; j < nT; ++j) alpha_s[tid][j] /= sum;
-  }
-  if constexpr (GAINS_SMEM) {
-    for (int e = tid; e < D * H; e += blockDim.x) gs[e] = __ldg(gains.g[e / H] + e % H);
-  }
-  __syncthreads();
-  // A fragments: rows 0..7 = bf16(alpha), rows 8..15 = bf16(alpha - bf16(alpha))
-  uint32_t af[4];
-  {
-    auto a_el = [&](int row, int col) -> __nv_bfloat16 {
-      const int i = row & 7;
-      if (i >= D || col >= nT) return __float2bfloat16_rn(0.f);
-      const float a = alpha_s[i][col];
-      const __nv_bfloat16 hi = __float2bfloat16_rn(a);
-      return row < 8 ? hi : __float2bfloat16_rn(a - __bfloat162float(hi));
-    };
-    auto pk = [&](int row, int col) {
-      __nv_bfloat162 v;
-      v.x = a_el(row, col);
-      v.y = a_el(row, col + 1);
-      return *reinterpret_cast<uint32_t*>(&v);
-    };
-    af[0] = pk(gq, 2 * tq);
-    af[1] = pk(gq + 8, 2 * tq);
-    af[2] = pk(gq, 2 * tq + 8);
-    af[3] = pk(gq + 8, 2 * tq + 8);
-  }
-  const int64_t my_rows = N > blockIdx.x ? (N - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  auto load_row = [&](int64_t k, int slot) {
-    const int64_t n = blockIdx.x + k * static_cast<int64_t>(gridDim.x);
-    uint8_t* dst = fsm + static_cast<size_t>(slot) * slot_bytes;
-    mbar_arrive_expect_tx(&full[slot], row_bytes * nT);
-    for (int j = 0; j < nT; ++j)
-      bulk_load(dst + j * rs, states + (n * nT + j) * H, row_bytes, &full[slot]);
-  };
-  if (tid == 0)
-    for (int k = 0; k < slots && k < my_rows; ++k) load_row(k, k);
-  // this warp's n-tiles (8 columns each): a contiguous run
-  const int ntiles = H >> 3;
-  const int per = (ntiles + 7) >> 3;
-  const int nt0 = warp * per, nt1 = min(ntiles, nt0 + per);
-  // ldmatrix.x2.trans row address of lane l (K row l & 15; rows >= T -> row 0)
-  const int krow = (lane & 15) < nT ? (lane & 15) : 0;
-  const float inv_h = 1.f / static_cast<float>(H);
-
-  int64_t k = 0;
-  for (; k < my_rows; ++k) {
-    const int slot = static_cast<int>(k % slots);
-    const int64_t n = blockIdx.x + k * static_cast<int64_t>(gridDim.x);
-    // every thread waits (bounded), then all leave together: the warp-wide
-    // ldmatrix / mma below must never run in a diverged warp
-    if (!mbar_wait(&full[slot], static_cast<uint32_t>((k / slots) & 1), status, 23))
-      abort_flag = 1;
-    __syncthreads();
-    if (abort_flag) break;
-    const uint32_t base = smem_u32(fsm + static_cast<size_t>(slot) * slot_bytes) + krow * rs;
-    auto mma_tile = [&](int nt, float* c) {
-      uint32_t b0, b1;
-      asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-                   : "=r"(b0), "=r"(b1) : "r"(base + nt * 16));
-      c[0] = c[1] = c[2] = c[3] = 0.f;
-      asm volatile(
-          "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-          "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-          : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-          : "r"(af[0]), "r"(af[1]), "r"(af[2]), "r"(af[3]), "r"(b0), "r"(b1));
-    };
-    // pass 1: sums of squares of layer gq over this warp's columns
-    float ss = 0.f;
-#pragma unroll 4
-    for (int nt = nt0; nt < nt1; ++nt) {
-      float c[4];
-      mma_tile(nt, c);
-      const float u0 = c[0] + c[2], u1 = c[1] + c[3];
-      ss = fmaf(u0, u0, fmaf(u1, u1, ss));
-    }
-    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-    const int par = static_cast<int>(k & 1);
-    if (tq == 0) red[par][gq][warp] = ss;
-    __syncthreads();
-    float tot = 0.f;
-#pragma unroll
-    for (int w = 0; w < kFuseMmaThreads / 32; ++w) tot += red[par][gq][w];
-    const float sc = rsqrtf(tot * inv_h + eps);
-    // pass 2: scale, gain, store (lanes of layers gq < D; every lane runs
-    // the warp-wide ldmatrix / mma)
-    const bool st_lane = gq < D;
-    __nv_bfloat16* out = fused + (static_cast<size_t>(st_lane ? gq : 0) * N + n) * H + 2 * tq;
-    const float* gp = (GAINS_SMEM ? gs + (st_lane ? gq : 0) * H : gains.g[st_lane ? gq : 0]) +
-                      2 * tq;
-#pragma unroll 4
-    for (int nt = nt0; nt < nt1; ++nt) {
-      float c[4];
-      mma_tile(nt, c);
-      if (st_lane) {
-        const float2 gv = GAINS_SMEM ? *reinterpret_cast<const float2*>(gp + nt * 8)
-                                     : __ldg(reinterpret_cast<const float2*>(gp + nt * 8));
-        const float f0 = (c[0] + c[2]) * sc * gv.x, f1 = (c[1] + c[3]) * sc * gv.y;
-        *reinterpret_cast<__nv_bfloat162*>(out + nt * 8) = __floats2bfloat162_rn(f0, f1);
-      }
-    }
-    __syncthreads();   // every warp is done with the slot
-    if (tid == 0 && k + slots < my_rows) load_row(k + slots, slot);
-  }
-  if (abort_flag && tid == 0) {
-    for (int64_t q = k; q < my_rows && q < k + slots; ++q)
-      mbar_wait(&full[q % slots], static_cast<uint32_t>((q / slots) & 1), status, 24);
-  }
-}
-
 // Ring depth: rows of up to ~96 KB in flight per CTA (two CTAs per SM fit
 // when the ring is small), never fewer than two rows.
 template <typename T>
 static int fuse_slots(int nT, int H) {
   const int rb = nT * H * static_cast<int>(sizeof(T));
-  return std::max(2, std::min(8, (96 * 1024) / rb));
+  const int two_per_sm = (96 * 1024) / rb;          // rows that keep two CTAs per SM
+  if (two_per_sm >= 2) return std::min(8, two_per_sm);
+  // one CTA per SM anyway: as many rows in flight as the budget holds
+  return std::max(2, std::min(8, kFuseSmemBudget / rb));
 }
 
 template <typename T, int MAXD>
@@ -372,62 +235,11 @@ static int fuse_max_hidden(int nT) {
   return std::min(by_threads, by_smem / 16 * 16);
 }
 
-// Tensor-core fusion launch: ring slots and gain placement from the shared
-// memory the row size leaves (two CTAs per SM when both fit in half an SM).
-static cudaError_t fuse_mma_go(const void* states, int64_t N, int nT, int H, int D,
-                               const float* w_fuse, const FuseGains& g, void* fused, float eps,
-                               uint32_t* status, cudaStream_t st) {
-  constexpr size_t kBudget = 222 * 1024;
-  const size_t slot = static_cast<size_t>(nT) * (static_cast<size_t>(H) * 2 + 16);
-  const size_t gbytes = static_cast<size_t>(D) * H * 4;
-  int per_sm = 1, slots = 0;
-  bool gsm = false;
-  if (2 * slot + gbytes <= kBudget / 2) {          // two CTAs, two slots + gains each
-    per_sm = 2;
-    slots = 2;
-    gsm = true;
-  } else if (2 * slot + gbytes <= kBudget) {
-    slots = static_cast<int>(std::min<size_t>(8, (kBudget - gbytes) / slot));
-    gsm = true;
-  } else {
-    slots = static_cast<int>(std::min<size_t>(8, kBudget / slot));
-  }
-  if (slots < 2) return cudaErrorInvalidValue;
-  const size_t smem = slots * slot + (gsm ? gbytes : 0);
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    for (const void* k : {reinterpret_cast<const void*>(fuse_mma_kernel<true>),
-                          reinterpret_cast<const void*>(fuse_mma_kernel<false>)}) {
-      const cudaError_t e =
-          cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kBudget);
-      if (e != cudaSuccess && attr == cudaSuccess) attr = e;
-    }
-  });
-  if (attr != cudaSuccess) return attr;
-  const int grid = static_cast<int>(std::min<int64_t>(N, kNumSMs * per_sm));
-  auto* st_ = static_cast<const __nv_bfloat16*>(states);
-  auto* fu = static_cast<__nv_bfloat16*>(fused);
-  if (gsm)
-    return launch_k(fuse_mma_kernel<true>, dim3(grid), dim3(kFuseMmaThreads), smem, st, st_, N,
-                    nT, H, D, w_fuse, g, fu, eps, slots, status);
-  return launch_k(fuse_mma_kernel<false>, dim3(grid), dim3(kFuseMmaThreads), smem, st, st_, N, nT,
-                  H, D, w_fuse, g, fu, eps, slots, status);
-}
-
-static bool fuse_mma_ok(int dtype, int nT, int H, int D) {
-  if (dtype != DFLASH_BF16 || D > 8 || nT > 16 || H % 8 != 0) return false;
-  if (const char* e = std::getenv("DFLASH_FUSE_SIMT")) return e[0] == '0';
-  return static_cast<size_t>(2) * nT * (static_cast<size_t>(H) * 2 + 16) <= 222 * 1024;
-}
-
 template <typename T>
 static cudaError_t launch_fuse_t(const void* states, int64_t N, int nT, int H, int D,
                                  const float* w_fuse, const FuseGains& g, void* fused, float eps,
                                  uint32_t* status, cudaStream_t st) {
   if (H > fuse_max_hidden<T>(nT)) return cudaErrorInvalidValue;
-  if (fuse_mma_ok(sizeof(T) == 2 ? DFLASH_BF16 : DFLASH_FP32, nT, H, D))
-    return fuse_mma_go(states, N, nT, H, D, w_fuse, g, fused, eps, status, st);
   if (D <= 4) return fuse_go<T, 4>(states, N, nT, H, D, w_fuse, g, fused, eps, status, st);
   if (D <= 8) return fuse_go<T, 8>(states, N, nT, H, D, w_fuse, g, fused, eps, status, st);
   return fuse_go<T, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, status, st);
