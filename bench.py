@@ -497,11 +497,14 @@ def run_ours(args):
     # dominant-kernel roofline of each
     per_config = {}
     if world == 1 and not args.no_per_config:
-        for name in synth.CONFIG_ORDER:
-            if name == cfg.name:
-                continue
+        # every other workload in this mode, and the main workload in the
+        # other mode (steady: only the newly accepted rows fused/projected)
+        other = "steady" if args.mode == "full" else "full"
+        runs = [(n, args.mode) for n in synth.CONFIG_ORDER if n != cfg.name]
+        runs.append((cfg.name, other))
+        for name, mode2 in runs:
             c2 = synth.get_config(name)
-            w2 = workload.Workload(c2, seed=args.seed, mode=args.mode)
+            w2 = workload.Workload(c2, seed=args.seed, mode=mode2)
             w2.step(verify=False)
             torch.cuda.synchronize()
             n2 = w2.plant_targets()
@@ -511,7 +514,8 @@ def run_ours(args):
             t2, _ = accepted_tokens(w2, stream, n2, 16)
             r2 = kernel_table(w2, c2, DF, peaks, stream, 10, ms2)
             d2 = dominant(r2)
-            per_config[name] = {"ms_per_step": ms2, "blocks_s": w2.final_buf.nb / (ms2 / 1e3),
+            key = name if mode2 == args.mode else f"{name}/{mode2}"
+            per_config[key] = {"ms_per_step": ms2, "blocks_s": w2.final_buf.nb / (ms2 / 1e3),
                                 "accepted_tok_s": t2 / (ms2 / 1e3), "steps": steps2,
                                 "dominant_kernel": d2["kernel"], "dominant_bound": d2["bound"],
                                 "dominant_frac": d2["frac"],
