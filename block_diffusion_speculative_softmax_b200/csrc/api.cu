@@ -249,21 +249,31 @@ struct Needs {
   }
 };
 
+// Scratch of the GEMMs of one step.  A workspace sized for (M, n_new) must
+// also serve every smaller call (a D2SD first pass drafts fewer blocks than
+// its second, a steady step fuses fewer rows), and smaller token counts can
+// need MORE split-K scratch, so every smaller block count and a dense sample
+// of smaller row counts are planned too.
 Needs step_needs(const dflash_config* c, int64_t M, int64_t n_new) {
   Needs n;
   dflash_layer_weights l{};
+  auto ctx_rows = [&](int64_t r) {
+    n.take(plan_gemm(job_kv(c, nullptr, r, nullptr, nullptr, 0, 0, 0, 0)));
+    n.take(plan_gemm(job_fc(c, nullptr, r, nullptr, nullptr)));
+  };
   if (n_new > 0) {
-    n.take(plan_gemm(job_kv(c, nullptr, n_new, nullptr, nullptr, 0, 0, 0, 0)));
-    n.take(plan_gemm(job_fc(c, nullptr, n_new, nullptr, nullptr)));
+    ctx_rows(n_new);
+    for (int64_t r = 1; r < n_new && r <= 4096; r += (r < 128 ? 1 : 64)) ctx_rows(r);
   }
-  if (M > 0) {
-    n.take(plan_gemm(job_kv(c, nullptr, M, nullptr, nullptr, 0, 0, 0, 0)));
-    n.take(plan_gemm(job_qkv(c, l, nullptr, M, nullptr, 0, 0, 0)));
-    n.take(plan_gemm(job_resid(c, nullptr, nullptr, M, c->n_q_heads * c->head_dim, 0)));
-    n.take(plan_gemm(job_swiglu(c, nullptr, nullptr, nullptr, M, 0)));
-    n.take(plan_gemm(job_resid(c, nullptr, nullptr, M, c->ffn, 0)));
-    n.take(plan_lmhead(c->dtype, c->vocab, M, c->hidden));
-    n.take(plan_gemm(job_logits(c, nullptr, M, nullptr, nullptr)));
+  for (int64_t m = std::min<int64_t>(M, c->block); m > 0 && m <= M;
+       m = (m == M) ? M + 1 : std::min<int64_t>(M, m + c->block)) {
+    n.take(plan_gemm(job_kv(c, nullptr, m, nullptr, nullptr, 0, 0, 0, 0)));
+    n.take(plan_gemm(job_qkv(c, l, nullptr, m, nullptr, 0, 0, 0)));
+    n.take(plan_gemm(job_resid(c, nullptr, nullptr, m, c->n_q_heads * c->head_dim, 0)));
+    n.take(plan_gemm(job_swiglu(c, nullptr, nullptr, nullptr, m, 0)));
+    n.take(plan_gemm(job_resid(c, nullptr, nullptr, m, c->ffn, 0)));
+    n.take(plan_lmhead(c->dtype, c->vocab, m, c->hidden));
+    n.take(plan_gemm(job_logits(c, nullptr, m, nullptr, nullptr)));
   }
   return n;
 }
@@ -296,7 +306,15 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
   // context behind its fp32 product [N][H] in the same region
   L.fused = take(std::max(static_cast<size_t>(c->n_draft_layers) * e, 4 + e) * n_new * H);
   L.partial = take(nd.partial_floats * 4);
-  L.attn_ws = take(attn_ws_bytes(ap, nb, c->block, c->n_q_heads, c->head_dim));
+  // fewer blocks can mean more splits (and more partials): size for all
+  size_t attn_bytes = 0;
+  for (int b = 1; b <= nb; ++b)
+    attn_bytes = std::max(
+        attn_bytes, attn_ws_bytes(plan_attn(c->dtype, b, c->block, c->n_q_heads, c->n_kv_heads,
+                                            c->head_dim, max_ctx),
+                                  b, c->block, c->n_q_heads, c->head_dim));
+  (void)ap;
+  L.attn_ws = take(attn_bytes);
   const size_t ncount = nd.counters;
   // the context branch runs on a second stream: its own split-K scratch
   Needs side;
@@ -306,17 +324,17 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
   }
   L.partial_side = take(side.partial_floats * 4);
   size_t chain_pf = 0, chain_cn = 0;
-  if (use_chain(c, M)) {
-    // the chain with a QKV stage is the larger one
-    chain_needs(job_chain(c, nullptr, 0, M, nullptr, nullptr, nullptr, nullptr, nullptr,
-                          nullptr, nullptr, nullptr, nullptr, 0),
-                &chain_pf, &chain_cn);
-    size_t pf2 = 0, cn2 = 0;
-    chain_needs(job_chain(c, nullptr, c->n_draft_layers - 1, M, nullptr, nullptr, nullptr,
-                          nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0),
-                &pf2, &cn2);
-    chain_pf = std::max(chain_pf, pf2);
-    chain_cn = std::max(chain_cn, cn2);
+  // any call with up to min(M, 64) block rows may run the layer chain
+  const int64_t Mc = std::min<int64_t>(M, 64);
+  if (use_chain(c, Mc)) {
+    for (int i : {0, c->n_draft_layers - 1}) {   // with and without the QKV stage
+      size_t pf2 = 0, cn2 = 0;
+      chain_needs(job_chain(c, nullptr, i, Mc, nullptr, nullptr, nullptr, nullptr, nullptr,
+                            nullptr, nullptr, nullptr, nullptr, 0),
+                  &pf2, &cn2);
+      chain_pf = std::max(chain_pf, pf2);
+      chain_cn = std::max(chain_cn, cn2);
+    }
   }
   L.chain_part = take(chain_pf * 4);
   L.zero = off;
@@ -329,7 +347,10 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
   L.blk_pos = take(M * 4);
   L.new_pos = take(n_new * 4);
   L.new_dst = take(n_new * 8);
-  L.lse = take(static_cast<size_t>(lmhead_tiles(c->dtype, c->vocab, M)) * M * 8);
+  // (fewer tokens can mean more, narrower vocabulary tiles: size for both)
+  const int64_t Ms = std::min<int64_t>(M, 64);
+  L.lse = take(std::max(static_cast<size_t>(lmhead_tiles(c->dtype, c->vocab, M)) * M,
+                        static_cast<size_t>(lmhead_tiles(c->dtype, c->vocab, Ms)) * Ms) * 8);
   L.row_lse = take(M * 4);   // temperature-1 mode: logsumexp of each logit row
   L.rope_len = static_cast<int>(max_ctx + c->block);
   L.rope = take(static_cast<size_t>(L.rope_len) * (c->head_dim / 2) * 8);

@@ -143,7 +143,6 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
   __shared__ int s_last, s_post;
-  __shared__ float s_red[EPI / 32];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.grid;
@@ -231,6 +230,7 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
           const uint64_t t0 = globaltimer_ns();
           uint32_t it = 0;
           while (ld_acquire(p.ready + si) == 0u) {
+            __nanosleep(32);
             if ((++it & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
               report(p.status, DFLASH_ETIMEOUT, 82);
               abort_flag = 1;
@@ -448,25 +448,32 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
         if (s_post) {
           __threadfence();
           if (S.norm_g != nullptr) {
-            // x[m] = h[m] / sqrt(mean(h[m]^2) + eps) * g, one row at a time
-            for (int m = 0; m < p.M; ++m) {
-              const float* hr = p.h + static_cast<int64_t>(m) * p.H;
+            // x[m] = h[m] / sqrt(mean(h[m]^2) + eps) * g: one warp per row,
+            // float4 loads (the row is read twice, from L2)
+            const int nv = p.H >> 2;
+            const float4* g4 = reinterpret_cast<const float4*>(S.norm_g);
+            for (int m = et >> 5; m < p.M; m += EPI / 32) {
+              const float4* hr = reinterpret_cast<const float4*>(p.h + static_cast<int64_t>(m) * p.H);
               float ss = 0.f;
-              for (int e = et; e < p.H; e += EPI) {
-                const float hv = __ldcg(hr + e);
-                ss = fmaf(hv, hv, ss);
+#pragma unroll 4
+              for (int e = lane; e < nv; e += 32) {
+                const float4 hv = __ldcg(hr + e);
+                ss = fmaf(hv.x, hv.x, fmaf(hv.y, hv.y, fmaf(hv.z, hv.z, fmaf(hv.w, hv.w, ss))));
               }
               ss = warp_sum(ss);
-              if (lane == 0) s_red[et >> 5] = ss;
-              named_sync(1, EPI);
-              float tot = 0.f;
-#pragma unroll
-              for (int w = 0; w < EPI / 32; ++w) tot += s_red[w];
-              const float sc = rsqrtf(tot / static_cast<float>(p.H) + p.eps);
-              for (int e = et; e < p.H; e += EPI)
-                p.x[static_cast<int64_t>(m) * p.H + e] =
-                    __float2bfloat16_rn(__ldcg(hr + e) * sc * __ldg(S.norm_g + e));
-              named_sync(1, EPI);
+              const float sc = rsqrtf(ss / static_cast<float>(p.H) + p.eps);
+              uint2* xr = reinterpret_cast<uint2*>(p.x + static_cast<int64_t>(m) * p.H);
+#pragma unroll 4
+              for (int e = lane; e < nv; e += 32) {
+                const float4 hv = __ldcg(hr + e);
+                const float4 gv = __ldg(g4 + e);
+                __nv_bfloat162 lo = __floats2bfloat162_rn(hv.x * sc * gv.x, hv.y * sc * gv.y);
+                __nv_bfloat162 hi = __floats2bfloat162_rn(hv.z * sc * gv.z, hv.w * sc * gv.w);
+                uint2 pk;
+                pk.x = *reinterpret_cast<uint32_t*>(&lo);
+                pk.y = *reinterpret_cast<uint32_t*>(&hi);
+                xr[e] = pk;
+              }
             }
             fence_proxy_async_global();
             named_sync(1, EPI);

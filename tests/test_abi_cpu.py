@@ -143,3 +143,24 @@ def test_misaligned_index_and_output_pointers_rejected(lib):
     st = lib.dflash_draft_step(C.byref(cfg), C.byref(w), C.byref(a), ok, 1 << 30, None)
     assert st == DF.EINVAL and b"ctx_off is not 8-byte aligned" in lib.dflash_last_error()
     assert DF.dflash_launch_count() == 0
+
+
+def test_workspace_size_is_monotone_in_blocks_and_rows():
+    """A workspace sized for (n_blocks, n_ctx_new) must serve every call with
+    fewer blocks or rows (a D2SD first pass drafts fewer blocks than its
+    second pass; a steady step fuses fewer rows than a full one)."""
+    from block_diffusion_speculative_softmax_b200 import dflash as DF
+    DF.load()
+    for kw in (dict(hidden=640, n_q_heads=16, n_kv_heads=2, head_dim=64, ffn=704,
+                    n_draft_layers=2, n_target_layers=5, block=16, vocab=3001),
+               dict(hidden=2560, n_q_heads=32, n_kv_heads=8, head_dim=128, ffn=9728,
+                    n_draft_layers=5, n_target_layers=5, block=16, vocab=151936)):
+        cc = DF.make_config(**kw)
+        sizes = {}
+        for nb in (1, 2, 3, 4, 5, 8, 12, 32):
+            for n_new in (0, 7, 100, 2048):
+                sizes[nb, n_new] = DF.dflash_workspace_size(cc, nb, nb, n_new, 4096)
+        for (nb, n_new), v in sizes.items():
+            for (nb2, n2), v2 in sizes.items():
+                if nb2 <= nb and n2 <= n_new:
+                    assert v2 <= v, ((nb, n_new, v), (nb2, n2, v2))
