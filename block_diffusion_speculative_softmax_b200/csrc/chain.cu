@@ -405,12 +405,17 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
               }
             }
           } else if (g.op == EPI_RESID) {
+            // all of the column's residual loads first, then the adds
             const int f = row0 + et;
             float* hp = static_cast<float*>(g.out) + f;
+            const bool fv = f < g.rows;
+            float hv[BN];
 #pragma unroll
             for (int j = 0; j < BN; ++j)
-              if (f < g.rows && j < p.M)
-                hp[static_cast<int64_t>(j) * g.out_stride] += stg[j * SROW + et];
+              hv[j] = (fv && j < p.M) ? __ldcg(hp + static_cast<int64_t>(j) * g.out_stride) : 0.f;
+#pragma unroll
+            for (int j = 0; j < BN; ++j)
+              if (fv && j < p.M) hp[static_cast<int64_t>(j) * g.out_stride] = hv[j] + stg[j * SROW + et];
           } else {
             const int f = row0 + et;
             const int half = p.head_dim >> 1;
@@ -418,16 +423,29 @@ __global__ void __launch_bounds__(THREADS, 1) chain_kernel(const __grid_constant
             const int prt = i < half ? et + half : et - half;
             const int fi = i < half ? i : i - half;
             __nv_bfloat16* o = static_cast<__nv_bfloat16*>(g.out);
-#pragma unroll 4
-            for (int j = 0; j < BN; ++j) {
-              if (f >= g.rows || j >= p.M) continue;
-              float xv = stg[j * SROW + et];
+            // 16 tokens at a time: their positions, then their (cos, sin),
+            // each as one batch of independent loads
+#pragma unroll 1
+            for (int j0 = 0; j0 < BN; j0 += 16) {
+              float2 cs[16];
               if (g.rope) {
-                const float2 cs = rope_cs(p, p.pos[j], fi);
-                const float pv = stg[j * SROW + prt];
-                xv = i < half ? xv * cs.x - pv * cs.y : xv * cs.x + pv * cs.y;
+                int ps[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) ps[q] = __ldg(p.pos + min(j0 + q, p.M - 1));
+#pragma unroll
+                for (int q = 0; q < 16; ++q) cs[q] = rope_cs(p, ps[q], fi);
               }
-              o[static_cast<int64_t>(j) * g.out_stride + f] = __float2bfloat16_rn(xv);
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                const int j = j0 + q;
+                if (f >= g.rows || j >= p.M) continue;
+                float xv = stg[j * SROW + et];
+                if (g.rope) {
+                  const float pv = stg[j * SROW + prt];
+                  xv = i < half ? xv * cs[q].x - pv * cs[q].y : xv * cs[q].x + pv * cs[q].y;
+                }
+                o[static_cast<int64_t>(j) * g.out_stride + f] = __float2bfloat16_rn(xv);
+              }
             }
           }
           // the next stage reads these outputs through TMA (async proxy)

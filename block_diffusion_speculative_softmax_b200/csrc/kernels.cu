@@ -26,6 +26,20 @@ struct FuseGains {
   const float* g[kMaxLayers];
 };
 
+// Paired fp32 arithmetic (one instruction for two lanes of a .b64 pair):
+// d = a * b + d and d = a * b, elementwise on (0, 1).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{.reg .b64 A, B, D;\n\tmov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+      "mov.b64 D, {%0, %1};\n\tfma.rn.f32x2 D, A, B, D;\n\tmov.b64 {%0, %1}, D;}"
+      : "+f"(d0), "+f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void fmul2(float& d0, float& d1, float b0, float b1) {
+  asm("{.reg .b64 B, D;\n\tmov.b64 B, {%2, %3};\n\tmov.b64 D, {%0, %1};\n\t"
+      "mul.rn.f32x2 D, D, B;\n\tmov.b64 {%0, %1}, D;}"
+      : "+f"(d0), "+f"(d1) : "f"(b0), "f"(b1));
+}
+
 constexpr int kFuseThreads = 512;
 constexpr int kFuseSmemBudget = 221 * 1024;
 
@@ -38,7 +52,7 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
   constexpr int VE = V::N;
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ __align__(8) uint64_t full[8];
-  __shared__ float alpha[kMaxLayers][kMaxTargetLayers];
+  __shared__ __align__(16) float alpha[kMaxTargetLayers][MAXD];   // [j][i], zero past D
   __shared__ __align__(16) float red[2][MAXD][32];   // per-warp partial sums, layer-major
   __shared__ volatile int abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -51,16 +65,20 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (tid < D) {
-    float mx = -INFINITY;
-    for (int j = 0; j < nT; ++j) mx = fmaxf(mx, w_fuse[tid * nT + j]);
-    float sum = 0.f;
-    for (int j = 0; j < nT; ++j) {
-      const float e = expf(w_fuse[tid * nT + j] - mx);
-      alpha[tid][j] = e;
-      sum += e;
+  if (tid < MAXD) {
+    if (tid < D) {
+      float mx = -INFINITY;
+      for (int j = 0; j < nT; ++j) mx = fmaxf(mx, w_fuse[tid * nT + j]);
+      float sum = 0.f;
+      for (int j = 0; j < nT; ++j) {
+        const float e = expf(w_fuse[tid * nT + j] - mx);
+        alpha[j][tid] = e;
+        sum += e;
+      }
+      for (int j = 0; j < nT; ++j) alpha[j][tid] /= sum;
+    } else {
+      for (int j = 0; j < nT; ++j) alpha[j][tid] = 0.f;
     }
-    for (int j = 0; j < nT; ++j) alpha[tid][j] /= sum;
   }
   __syncthreads();
   // rows of this CTA: blockIdx.x, blockIdx.x + gridDim.x, ...
@@ -109,19 +127,28 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
 #pragma unroll
           for (int q = 0; q < VE; ++q) h[q] = fp[q];
         }
+        // alpha[j][0..MAXD) as float4 loads, paired FMAs over column pairs
+        float a[MAXD];
+#pragma unroll
+        for (int q = 0; q < MAXD / 4; ++q) {
+          const float4 av = *reinterpret_cast<const float4*>(&alpha[j][4 * q]);
+          a[4 * q] = av.x; a[4 * q + 1] = av.y; a[4 * q + 2] = av.z; a[4 * q + 3] = av.w;
+        }
 #pragma unroll
         for (int i = 0; i < MAXD; ++i) {
           if (i < D) {
-            const float a = alpha[i][j];
 #pragma unroll
-            for (int e = 0; e < VE; ++e) u[i][e] = fmaf(a, h[e], u[i][e]);
+            for (int e = 0; e < VE; e += 2) ffma2(u[i][e], u[i][e + 1], a[i], a[i], h[e], h[e + 1]);
           }
         }
       }
 #pragma unroll
-      for (int i = 0; i < MAXD; ++i)
+      for (int i = 0; i < MAXD; ++i) {
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < VE; ++e) ss[i] = fmaf(u[i][e], u[i][e], ss[i]);
+        for (int e = 0; e < VE; e += 2) ffma2(s0, s1, u[i][e], u[i][e + 1], u[i][e], u[i][e + 1]);
+        ss[i] = s0 + s1;
+      }
     }
     const int par = static_cast<int>(k & 1);
 #pragma unroll
@@ -141,10 +168,8 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
 #pragma unroll
           for (int q = 0; q < VE / 4; ++q) {
             const float4 gv = __ldg(g4 + q);
-            u[i][4 * q] *= gv.x;
-            u[i][4 * q + 1] *= gv.y;
-            u[i][4 * q + 2] *= gv.z;
-            u[i][4 * q + 3] *= gv.w;
+            fmul2(u[i][4 * q], u[i][4 * q + 1], gv.x, gv.y);
+            fmul2(u[i][4 * q + 2], u[i][4 * q + 3], gv.z, gv.w);
           }
         }
       }
@@ -179,7 +204,11 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
                                   static_cast<float>(H) + eps);
           float o[VE];
 #pragma unroll
-          for (int e = 0; e < VE; ++e) o[e] = u[i][e] * sc;
+          for (int e = 0; e < VE; e += 2) {
+            o[e] = u[i][e];
+            o[e + 1] = u[i][e + 1];
+            fmul2(o[e], o[e + 1], sc, sc);
+          }
           V::store(fused + (static_cast<size_t>(i) * N + n) * H + col, o);
         }
       }
