@@ -38,7 +38,12 @@ ACCEPT_DRAWS = 32          # planted target draws averaged for accepted tok/s
 # (summarised under profiles/), valid only for the source file it was taken
 # with (digest of the file without comments); any later change of that code
 # nulls it.  Key: (workload, mode, kernel-table name).
-TRAFFIC = {}
+TRAFFIC = {
+    # one serving32 context K/V projection (1 pass: dram__bytes_read.sum +
+    # dram__bytes_write.sum of gemm_tokp_kernel, profiles/gemm_tokp_ctxproj_serving32.md)
+    ("serving32", "full", "ctx_kv_proj"): {"bytes": 1188603392 + 534270976, "file": "gemm.cu",
+                                          "sha256": "7821341021342553"},
+}
 
 
 def parse():
