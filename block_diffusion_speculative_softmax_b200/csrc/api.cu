@@ -168,74 +168,11 @@ GemmJob job_swiglu(const dflash_config* c, const void* wg, const void* wu, const
   return j;
 }
 
-// Layer chain i (bf16, <= 64 block rows): O_i -> RMSNorm_mlp -> gate/up_i ->
-// down_i -> RMSNorm (next layer's attention norm, or the final norm) ->
-// next layer's QKV (absent after the last layer).  Buffers as in the step.
-// DFLASH_NO_CHAIN=1 runs the layer as separate GEMM launches instead (the
-// same arithmetic; kept so the two schedules can be compared on one build).
-bool chain_disabled() {
-  const char* e = std::getenv("DFLASH_NO_CHAIN");
-  return e != nullptr && e[0] == '1';
-}
-
-bool use_chain(const dflash_config* c, int64_t M) {
-  return c->dtype == DFLASH_BF16 && M >= 1 && chain_bn(M) > 0;
-}
-
-ChainJob job_chain(const dflash_config* c, const dflash_weights* w, int i, int64_t M, float* h,
-                   void* x, void* attn, void* act, void* q, void* kb, void* vb,
-                   const int32_t* pos, const float2* rope_tab, int rope_len) {
-  const int D = c->n_draft_layers, H = c->hidden, F = c->ffn;
-  const int qd = c->n_q_heads * c->head_dim, kvd = c->n_kv_heads * c->head_dim;
-  const dflash_layer_weights* l = w ? &w->layers[i] : nullptr;
-  const dflash_layer_weights* ln = (w && i + 1 < D) ? &w->layers[i + 1] : nullptr;
-  ChainJob j;
-  j.M = M;
-  j.h = h;
-  j.H = H;
-  j.eps = c->rms_eps;
-  j.x_out = x;
-  j.pos = pos;
-  j.rope_tab = rope_tab;
-  j.rope_len = rope_len;
-  j.head_dim = c->head_dim;
-  ChainStageJob& o = j.st[0];
-  o.nseg = 1;
-  o.seg[0] = {l ? l->w_o : nullptr, nullptr, H, EPI_RESID, 0, h, H, 0};
-  o.x = attn;
-  o.K = qd;
-  o.norm_g = l ? l->g_mlp : nullptr;
-  ChainStageJob& gu = j.st[1];
-  gu.nseg = 1;
-  gu.seg[0] = {l ? l->w_gate : nullptr, l ? l->w_up : nullptr, F, EPI_SWIGLU, 0, act, F, 0};
-  gu.x = x;
-  gu.K = H;
-  ChainStageJob& dn = j.st[2];
-  dn.nseg = 1;
-  dn.seg[0] = {l ? l->w_down : nullptr, nullptr, H, EPI_RESID, 0, h, H, 0};
-  dn.x = act;
-  dn.K = F;
-  dn.norm_g = w ? (ln ? ln->g_attn : w->g_final) : nullptr;
-  j.nst = 3;
-  if (i + 1 < D) {
-    ChainStageJob& qs = j.st[3];
-    qs.nseg = 3;
-    qs.seg[0] = {ln ? ln->w_q : nullptr, nullptr, qd, EPI_STORE, 1, q, qd, 0};
-    qs.seg[1] = {ln ? ln->w_kd : nullptr, nullptr, kvd, EPI_STORE, 1, kb, kvd, 0};
-    qs.seg[2] = {ln ? ln->w_vd : nullptr, nullptr, kvd, EPI_STORE, 0, vb, kvd, 0};
-    qs.x = x;
-    qs.K = H;
-    j.nst = 4;
-  }
-  return j;
-}
-
 // ------------------------------------------------------------------ layout
 struct Layout {
   size_t h = 0, x = 0, q = 0, kb = 0, vb = 0, attn = 0, act = 0, fused = 0, partial = 0,
          attn_ws = 0, zero = 0, keys = 0, counters = 0, blk_pos = 0, new_pos = 0, new_dst = 0,
-         rope = 0, partial_side = 0, counters_side = 0, lse = 0, row_lse = 0, chain_part = 0,
-         chain_cnt = 0, chain_flags = 0, total = 0;
+         rope = 0, partial_side = 0, counters_side = 0, lse = 0, row_lse = 0, total = 0;
   int rope_len = 0;
   size_t zero_bytes = 0;   // [keys | counters], zeroed at the start of a step
 };
@@ -323,26 +260,10 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
     side.take(plan_gemm(job_fc(c, nullptr, n_new, nullptr, nullptr)));
   }
   L.partial_side = take(side.partial_floats * 4);
-  size_t chain_pf = 0, chain_cn = 0;
-  // any call with up to min(M, 64) block rows may run the layer chain
-  const int64_t Mc = std::min<int64_t>(M, 64);
-  if (use_chain(c, Mc)) {
-    for (int i : {0, c->n_draft_layers - 1}) {   // with and without the QKV stage
-      size_t pf2 = 0, cn2 = 0;
-      chain_needs(job_chain(c, nullptr, i, Mc, nullptr, nullptr, nullptr, nullptr, nullptr,
-                            nullptr, nullptr, nullptr, nullptr, 0),
-                  &pf2, &cn2);
-      chain_pf = std::max(chain_pf, pf2);
-      chain_cn = std::max(chain_cn, cn2);
-    }
-  }
-  L.chain_part = take(chain_pf * 4);
   L.zero = off;
   L.keys = take(M * 8);
   L.counters = take(ncount * 4);
   L.counters_side = take(side.counters * 4);
-  L.chain_cnt = take(chain_cn * 4);
-  L.chain_flags = take(static_cast<size_t>(c->n_draft_layers) * 2 * kChainMaxStages * 4);
   L.zero_bytes = off - L.zero;
   L.blk_pos = take(M * 4);
   L.new_pos = take(n_new * 4);
@@ -954,33 +875,19 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
            "slot embedding");
   const AttnPlan ap = plan_attn(dt, a->n_blocks, c->block, c->n_q_heads, c->n_kv_heads,
                                 c->head_dim, a->max_ctx_len);
-  const bool chained = use_chain(c, M) && !chain_disabled();
   for (int i = 0; i < D; ++i) {
     const dflash_layer_weights& l = w->layers[i];
-    // block: RMSNorm -> Q (RoPE), K^d (RoPE), V^d (from layer 1 on, the
-    // previous layer's chain already produced them)
-    if (!chained || i == 0) {
-      DFL_CUDA(launch_rmsnorm(dt, h, M, H, l.g_attn, c->rms_eps, x, st), "attention rmsnorm");
-      GemmJob jq = job_qkv(c, l, x, M, blk_pos, q, kb, vb);
-      jq.rope_tab = rope_tab;
-      jq.rope_len = L.rope_len;
-      if ((s = run_job(jq, partial, counters, status, st, "QKV GEMM")) != DFLASH_OK) return s;
-    }
+    // block: RMSNorm -> Q (RoPE), K^d (RoPE), V^d
+    DFL_CUDA(launch_rmsnorm(dt, h, M, H, l.g_attn, c->rms_eps, x, st), "attention rmsnorm");
+    GemmJob jq = job_qkv(c, l, x, M, blk_pos, q, kb, vb);
+    jq.rope_tab = rope_tab;
+    jq.rope_len = L.rope_len;
+    if ((s = run_job(jq, partial, counters, status, st, "QKV GEMM")) != DFLASH_OK) return s;
     if (side) DFL_CUDA(cudaStreamWaitEvent(st, side->done[i], 0), "join context");
     DFL_CUDA(launch_attn(dt, ap, a->n_blocks, c->block, c->n_q_heads, c->n_kv_heads,
                          c->head_dim, q, kb, vb, a->k_cache[i], a->v_cache[i], a->ctx_off,
                          a->block_req, attn, at<float>(ws, L.attn_ws), status, st, a->ctx_len),
              "attention");
-    if (chained) {
-      // O, MLP and the next layer's QKV (or the final norm) in one launch
-      const ChainJob jc = job_chain(c, w, i, M, h, x, attn, act, q, kb, vb, blk_pos, rope_tab,
-                                    L.rope_len);
-      DFL_CUDA(launch_chain(jc, at<float>(ws, L.chain_part), at<uint32_t>(ws, L.chain_cnt),
-                            at<uint32_t>(ws, L.chain_flags) + i * 2 * kChainMaxStages, status,
-                            st),
-               "layer chain");
-      continue;
-    }
     if ((s = run_job(job_resid(c, l.w_o, attn, M, qd, h), partial, counters, status, st,
                      "O GEMM")) != DFLASH_OK)
       return s;
@@ -992,8 +899,7 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
                      "down GEMM")) != DFLASH_OK)
       return s;
   }
-  if (!chained)   // (the last chain ends with the final norm)
-    DFL_CUDA(launch_rmsnorm(dt, h, M, H, w->g_final, c->rms_eps, x, st), "final rmsnorm");
+  DFL_CUDA(launch_rmsnorm(dt, h, M, H, w->g_final, c->rms_eps, x, st), "final rmsnorm");
   if (sampling) {
     // temperature 1: logits to the caller's buffer, a Gumbel-max draw per
     // slot, then (optionally) stochastic verification

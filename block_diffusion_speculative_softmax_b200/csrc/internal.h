@@ -93,38 +93,6 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V,
                                  cudaStream_t st, float* partial = nullptr,
                                  uint32_t* counters = nullptr, float2* lse = nullptr);
 
-// ---------------------------------------------------------------- layer chain
-// Persistent weight-streaming chain of GEMM stages for M <= 64 bf16 rows
-// (chain.cu): stage s reads x [M][K] (the previous stage's output or the
-// post-norm x_out), streams its weights and applies its segments' ops; a
-// stage with norm_g writes x_out = RMSNorm_{norm_g}(h) after it completes.
-constexpr int kChainMaxStages = 4;
-struct ChainStageJob {
-  GemmOut seg[kMaxSegs];
-  int nseg = 0;
-  const void* x = nullptr;
-  int K = 0;
-  const float* norm_g = nullptr;
-};
-struct ChainJob {
-  ChainStageJob st[kChainMaxStages];
-  int nst = 0;
-  int64_t M = 0;
-  float* h = nullptr;
-  int H = 0;
-  float eps = 0.f;
-  void* x_out = nullptr;
-  const int32_t* pos = nullptr;
-  const float2* rope_tab = nullptr;
-  int rope_len = 0;
-  int head_dim = 0;
-};
-int chain_bn(int64_t M);   // token tile for M rows (0: M too large for the chain)
-void chain_needs(const ChainJob& job, size_t* partial_floats, size_t* counters);
-// flags: 2 * kChainMaxStages zeroed words per launch; counters zero (left zero)
-cudaError_t launch_chain(const ChainJob& job, float* partial, uint32_t* counters,
-                         uint32_t* flags, uint32_t* status, cudaStream_t st);
-
 // ---------------------------------------------------------------- others
 cudaError_t launch_fuse(int dtype, const void* states, int64_t N, int T, int H,
                         int D, const float* w_fuse, const float* const* g_fuse,
