@@ -41,8 +41,8 @@ ACCEPT_DRAWS = 32          # planted target draws averaged for accepted tok/s
 TRAFFIC = {
     # one serving32 context K/V projection (1 pass: dram__bytes_read.sum +
     # dram__bytes_write.sum of gemm_tokp_kernel, profiles/gemm_tokp_ctxproj_serving32.md)
-    ("serving32", "full", "ctx_kv_proj"): {"bytes": 1188603392 + 534270976, "file": "gemm.cu",
-                                          "sha256": "7821341021342553"},
+    ("serving32", "full", "ctx_kv_proj"): {"bytes": 1192218112 + 533901312, "file": "gemm.cu",
+                                          "sha256": "17615a7f2c849ec7"},
 }
 
 
@@ -63,8 +63,8 @@ def parse():
                     help="launch the step eagerly instead of replaying a CUDA graph")
     ap.add_argument("--profile", action="store_true",
                     help="eager steps inside an NVTX range 'dflash_step' (for ncu launch lists)")
-    ap.add_argument("--op", choices=["lmhead", "mlp", "ctxproj", "attn", "fuse", "fcfuse",
-                                     "sample"],
+    ap.add_argument("--op", choices=["lmhead", "mlp", "ctxproj", "attn", "fuse", "fusenorm",
+                                     "fcfuse", "sample"],
                     help="time one entry point alone at the workload's shapes")
     ap.add_argument("--rows", type=int, default=0,
                     help="--op: context rows (default: the workload's own sum of lengths)")
@@ -396,10 +396,22 @@ def kernel_table(wl, cfg, DF, peaks, stream, reps, ms_step):
     if n_new > 0 and wl.w.w_fc is None:
         fused = torch.empty(D, n_new, H, dtype=dt, device="cuda")
         gl = [l["g_fuse"] for l in wl.w.layers]
-        sec = time_calls(lambda: DF.dflash_fuse_ctx(cc, wl.new_states, wl.w.w_fuse, gl, fused),
-                         stream, reps)
-        rows.append(_entry("fuse", "fuse_rows_kernel", sec, 1,
-                           n_new * T * H * e + D * n_new * H * e, 0.0, peaks, ms_step))
+        if cfg.dtype == "bf16":
+            # the step's form: unnormalised rows + per-row partial sums of
+            # squares (the norm is applied in the context projection)
+            P = DF.dflash_fuse_rss_parts(H)
+            rss = torch.empty(D, n_new, P, device="cuda")
+            sec = time_calls(lambda: DF.dflash_fuse_ctx_rss(cc, wl.new_states, wl.w.w_fuse, gl,
+                                                            fused, rss, ws), stream, reps)
+            rows.append(_entry("fuse", "fuse_rows_unnorm_kernel", sec, 1,
+                               n_new * T * H * e + D * n_new * H * e + D * n_new * P * 4, 0.0,
+                               peaks, ms_step))
+            del rss
+        else:
+            sec = time_calls(lambda: DF.dflash_fuse_ctx(cc, wl.new_states, wl.w.w_fuse, gl,
+                                                        fused), stream, reps)
+            rows.append(_entry("fuse", "fuse_rows_kernel", sec, 1,
+                               n_new * T * H * e + D * n_new * H * e, 0.0, peaks, ms_step))
         pos = torch.arange(n_new, dtype=torch.int32, device="cuda")
         lay = wl.w.layers[0]
         kc, vc = fb.k_cache[0], fb.v_cache[0]
@@ -728,14 +740,21 @@ def run_op(args):
         call = lambda: DF.dflash_sample(cc, z, 1, 0, tok, lq, None)
         algo = M * V * 4 + M * 8
         kernel = "sample_rows_kernel (Gumbel-max over stored logits)"
-    else:  # fuse
+    else:  # fuse (the step's split form for bf16), fusenorm (normalised output)
         st = rnd(N, T, H)
         wf = torch.randn(D, T, device="cuda", generator=g)
         gl = [torch.ones(H, device="cuda") for _ in range(D)]
         fused = torch.empty(D, N, H, dtype=dt, device="cuda")
-        call = lambda: DF.dflash_fuse_ctx(cc, st, wf, gl, fused)
-        algo = N * T * H * e + D * N * H * e
-        kernel = "fuse_rows_kernel (fusion + RMSNorm, all draft layers)"
+        if args.op == "fuse" and cfg.dtype == "bf16":
+            P = DF.dflash_fuse_rss_parts(H)
+            rss = torch.empty(D, N, P, device="cuda")
+            call = lambda: DF.dflash_fuse_ctx_rss(cc, st, wf, gl, fused, rss, ws)
+            algo = N * T * H * e + D * N * H * e + D * N * P * 4
+            kernel = "fuse_rows_unnorm_kernel (fusion, row sums of squares, all draft layers)"
+        else:
+            call = lambda: DF.dflash_fuse_ctx(cc, st, wf, gl, fused)
+            algo = N * T * H * e + D * N * H * e
+            kernel = "fuse_rows_kernel (fusion + RMSNorm, all draft layers)"
     for _ in range(args.warmup):
         call()
     torch.cuda.synchronize()

@@ -1,10 +1,15 @@
 """Build libdflash.so in-tree with nvcc for sm_100a.
 
-    python -m block_diffusion_speculative_softmax_b200.build [--verbose]
+    python -m block_diffusion_speculative_softmax_b200.build [--verbose] [--debug-bounds]
 
 Each .cu under csrc/ is compiled to an object in _build/ (in parallel), then
 linked into block_diffusion_speculative_softmax_b200/libdflash.so with the
 static CUDA runtime, so the library needs only the driver at run time.
+
+--debug-bounds builds libdflash_debug.so instead (objects in _build_debug/):
+the same kernels compiled with -DDFLASH_DEBUG_BOUNDS, whose device-side index
+checks report DFLASH_EBOUNDS through the status word instead of reading or
+writing outside a buffer.  Load it with DFLASH_LIB=<path> (see dflash.py).
 """
 from __future__ import annotations
 
@@ -21,6 +26,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libdflash.so")
+BUILD_DEBUG = os.path.join(ROOT, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libdflash_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
@@ -35,8 +42,8 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _compile(src: str, extra, verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src: str, extra, verbose: bool, build_dir: str = BUILD) -> str:
+    obj = os.path.join(build_dir, os.path.basename(src) + ".o")
     cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
     if verbose:
         print(" ".join(cmd), flush=True)
@@ -48,31 +55,35 @@ def _compile(src: str, extra, verbose: bool) -> str:
     return obj
 
 
-def _stale(srcs) -> bool:
-    if not os.path.exists(LIB):
+def _stale(srcs, lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = srcs + glob.glob(os.path.join(CSRC, "*.cuh")) + \
         glob.glob(os.path.join(CSRC, "*.h")) + \
         glob.glob(os.path.join(ROOT, "include", "*.h")) + [__file__]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          debug_bounds: bool = False) -> str:
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    if not force and not ptxas_info and not _stale(srcs):
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    lib, bdir = (LIB_DEBUG, BUILD_DEBUG) if debug_bounds else (LIB, BUILD)
+    if not force and not ptxas_info and not _stale(srcs, lib):
+        return lib
+    os.makedirs(bdir, exist_ok=True)
     extra = ["-Xptxas", "-v"] if ptxas_info else []
+    if debug_bounds:
+        extra.append("-DDFLASH_DEBUG_BOUNDS")
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, extra, verbose or ptxas_info), srcs))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, extra, verbose or ptxas_info, bdir), srcs))
+    tmp = lib + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
@@ -81,6 +92,9 @@ if __name__ == "__main__":
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true",
                     help="print registers / spills / shared memory per kernel")
+    ap.add_argument("--debug-bounds", action="store_true",
+                    help="build libdflash_debug.so with the device-side index checks")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose, ptxas_info=a.ptxas_info))
+    print(build(force=a.force, verbose=a.verbose, ptxas_info=a.ptxas_info,
+                debug_bounds=a.debug_bounds))
     sys.exit(0)

@@ -172,7 +172,7 @@ GemmJob job_swiglu(const dflash_config* c, const void* wg, const void* wu, const
 struct Layout {
   size_t h = 0, x = 0, q = 0, kb = 0, vb = 0, attn = 0, act = 0, fused = 0, partial = 0,
          attn_ws = 0, zero = 0, keys = 0, counters = 0, blk_pos = 0, new_pos = 0, new_dst = 0,
-         rope = 0, partial_side = 0, counters_side = 0, lse = 0, row_lse = 0, total = 0;
+         rope = 0, partial_side = 0, counters_side = 0, lse = 0, row_lse = 0, rss = 0, total = 0;
   int rope_len = 0;
   size_t zero_bytes = 0;   // [keys | counters], zeroed at the start of a step
 };
@@ -273,6 +273,9 @@ Layout make_layout(const dflash_config* c, int32_t n_req, int32_t nb, int64_t n_
   L.lse = take(std::max(static_cast<size_t>(lmhead_tiles(c->dtype, c->vocab, M)) * M,
                         static_cast<size_t>(lmhead_tiles(c->dtype, c->vocab, Ms)) * Ms) * 8);
   L.row_lse = take(M * 4);   // temperature-1 mode: logsumexp of each logit row
+  // per (draft layer, new row) partial sums of squares of the unnormalised
+  // bf16 fusion
+  L.rss = take(static_cast<size_t>(c->n_draft_layers) * n_new * fuse_unnorm_parts(c->hidden) * 4);
   L.rope_len = static_cast<int>(max_ctx + c->block);
   L.rope = take(static_cast<size_t>(L.rope_len) * (c->head_dim / 2) * 8);
   L.total = off;
@@ -369,6 +372,7 @@ dflash_status dflash_check(void* ws, void* stream) {
     DFL_CUDA(cudaMemset(ws, 0, sizeof(hdr)), "clear status");
     const char* what = hdr[0] == DFLASH_ETIMEOUT ? "a bounded device wait ran out"
                        : hdr[0] == DFLASH_ENUMERIC ? "non-finite logit"
+                       : hdr[0] == DFLASH_EBOUNDS  ? "device index out of its buffer"
                                                    : "device error";
     return fail(static_cast<dflash_status>(hdr[0]), "%s (kernel tag %u)", what, hdr[1]);
   }
@@ -390,6 +394,31 @@ dflash_status dflash_fuse_ctx(const dflash_config* cfg, const void* states, int6
   DFL_CUDA(launch_fuse(cfg->dtype, states, n_rows, cfg->n_target_layers, cfg->hidden,
                        cfg->n_draft_layers, w_fuse, g_fuse, fused, cfg->rms_eps, nullptr,
                        static_cast<cudaStream_t>(stream)),
+           "fusion kernel");
+  return DFLASH_OK;
+}
+
+int32_t dflash_fuse_rss_parts(int32_t hidden) { return hidden > 0 ? fuse_unnorm_parts(hidden) : 0; }
+
+dflash_status dflash_fuse_ctx_rss(const dflash_config* cfg, const void* states, int64_t n_rows,
+                                  const float* w_fuse, const float* const* g_fuse, void* fused,
+                                  float* rss, void* ws, size_t ws_bytes, void* stream) {
+  dflash_status s = check_config(cfg);
+  if (s != DFLASH_OK) return s;
+  DFL_CHECK(cfg->dtype == DFLASH_BF16, DFLASH_EUNSUPPORTED, "the split fusion is bf16 only");
+  DFL_CHECK(n_rows >= 0, DFLASH_EINVAL, "n_rows must be >= 0");
+  if ((s = check_ws(ws, ws_bytes, sizeof(DevStatus))) != DFLASH_OK) return s;
+  if (n_rows == 0) return DFLASH_OK;
+  DFL_PTR(states, "states");
+  DFL_PTR(fused, "fused");
+  DFL_CHECK(rss != nullptr, DFLASH_EINVAL, "rss is NULL");
+  DFL_ALIGNED(rss, 4, "rss");
+  DFL_CHECK(w_fuse != nullptr, DFLASH_EINVAL, "w_fuse is NULL");
+  DFL_CHECK(g_fuse != nullptr, DFLASH_EINVAL, "g_fuse is NULL");
+  for (int i = 0; i < cfg->n_draft_layers; ++i) DFL_PTR(g_fuse[i], "g_fuse[i]");
+  DFL_CUDA(launch_fuse_unnorm(states, n_rows, cfg->n_target_layers, cfg->hidden,
+                              cfg->n_draft_layers, w_fuse, g_fuse, fused, rss, status_word(ws),
+                              static_cast<cudaStream_t>(stream)),
            "fusion kernel");
   return DFLASH_OK;
 }
@@ -595,7 +624,7 @@ dflash_status dflash_sample(const dflash_config* cfg, int64_t M, const float* lo
   DFL_ALIGNED(logq, 4, "logq");
   DFL_ALIGNED(lse, 4, "lse");
   DFL_CUDA(launch_sample_rows(logits, M, cfg->vocab, seed, offset, cfg->block, nullptr, nullptr,
-                              tok, logq, lse, static_cast<cudaStream_t>(stream)),
+                              tok, logq, lse, nullptr, static_cast<cudaStream_t>(stream)),
            "sampling kernel");
   return DFLASH_OK;
 }
@@ -623,7 +652,7 @@ dflash_status dflash_accept_stochastic(int32_t R, int32_t B, int32_t V, const in
   DFL_CUDA(launch_accept_stochastic(R, B, V, draft, draft_logits, draft_lse, target_logp, seed,
                                     offset, n_acc, out_tok,
                                     at<unsigned long long>(ws, sizeof(DevStatus)),
-                                    static_cast<cudaStream_t>(stream)),
+                                    status_word(ws), static_cast<cudaStream_t>(stream)),
            "stochastic accept");
   return DFLASH_OK;
 }
@@ -824,7 +853,8 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
   DFL_CUDA(launch_prep_rows(a->n_req, a->n_blocks, c->block, a->block_req, a->ctx_off,
                             a->new_off, a->ctx_cached, a->ctx_len, a->new_count, a->n_ctx_new,
                             blk_pos, new_pos, new_dst,
-                            at<uint32_t>(ws, L.zero), static_cast<int64_t>(L.zero_bytes / 4), st),
+                            at<uint32_t>(ws, L.zero), static_cast<int64_t>(L.zero_bytes / 4),
+                            status, st),
            "row bookkeeping");
   float2* rope_tab = at<float2>(ws, L.rope);
   DFL_CUDA(launch_rope_table(rope_tab, L.rope_len, c->head_dim, c->rope_theta, st), "RoPE table");
@@ -843,6 +873,10 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
     // FC variant: fp32 product at the start of the fused region, the one
     // shared context right behind it
     uint8_t* fc_ctx = fused + static_cast<size_t>(a->n_ctx_new) * H * 4;
+    // bf16: the fusion leaves the norm's per-row scale to the K/V epilogue
+    const bool unnorm = !fc && dt == DFLASH_BF16;
+    float* rss = at<float>(ws, L.rss);
+    const int rss_parts = fuse_unnorm_parts(H);
     if (fc) {
       s = run_job(job_fc(c, a->new_states, a->n_ctx_new, w->w_fc, reinterpret_cast<float*>(fused)),
                   part_c, cnt_c, status, cs, "FC fusion GEMM");
@@ -853,9 +887,14 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
     } else {
       const float* gf[kMaxLayers];
       for (int i = 0; i < D; ++i) gf[i] = w->layers[i].g_fuse;
-      DFL_CUDA(launch_fuse(dt, a->new_states, a->n_ctx_new, c->n_target_layers, H, D, w->w_fuse,
-                           gf, fused, c->rms_eps, status, cs),
-               "fusion kernel");
+      if (unnorm)
+        DFL_CUDA(launch_fuse_unnorm(a->new_states, a->n_ctx_new, c->n_target_layers, H, D,
+                                    w->w_fuse, gf, fused, rss, status, cs),
+                 "fusion kernel");
+      else
+        DFL_CUDA(launch_fuse(dt, a->new_states, a->n_ctx_new, c->n_target_layers, H, D,
+                             w->w_fuse, gf, fused, c->rms_eps, status, cs),
+                 "fusion kernel");
     }
     for (int i = 0; i < D; ++i) {
       const dflash_layer_weights& l = w->layers[i];
@@ -865,13 +904,19 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
                           a->k_cache[i], a->v_cache[i]);
       jc.rope_tab = rope_tab;
       jc.rope_len = L.rope_len;
+      if (unnorm) {   // the fusion's RMSNorm, applied per row in the epilogue
+        jc.rss = rss + static_cast<size_t>(i) * a->n_ctx_new * rss_parts;
+        jc.rss_parts = rss_parts;
+        jc.rss_inv = 1.f / static_cast<float>(H);
+        jc.rss_eps = c->rms_eps;
+      }
       s = run_job(jc, part_c, cnt_c, status, cs, "context K/V GEMM");
       if (s != DFLASH_OK) return s;
       if (side) DFL_CUDA(cudaEventRecord(side->done[i], side->stream), "context done");
     }
   }
   DFL_CUDA(launch_embed(dt, w->embed, H, a->n_blocks, c->block, a->block_tokens, a->known_len,
-                        c->mask_token_id, h, st),
+                        c->mask_token_id, c->vocab, h, status, st),
            "slot embedding");
   const AttnPlan ap = plan_attn(dt, a->n_blocks, c->block, c->n_q_heads, c->n_kv_heads,
                                 c->head_dim, a->max_ctx_len);
@@ -909,12 +954,12 @@ dflash_status dflash_draft_step(const dflash_config* c, const dflash_weights* w,
     if (s != DFLASH_OK) return s;
     DFL_CUDA(launch_sample_rows(a->draft_logits, M, c->vocab, a->seed, a->rng_offset, c->block,
                                 a->block_tokens, a->known_len, a->draft_tokens, a->draft_logq,
-                                row_lse, st),
+                                row_lse, status, st),
              "sampling kernel");
     if (a->target_logp) {
       DFL_CUDA(launch_accept_stochastic(a->n_req, c->block, c->vocab, a->draft_tokens,
                                         a->draft_logits, row_lse, a->target_logp, a->seed,
-                                        a->rng_offset, a->n_acc, a->out_tok, keys, st),
+                                        a->rng_offset, a->n_acc, a->out_tok, keys, status, st),
                "stochastic accept");
     }
     return DFLASH_OK;

@@ -57,7 +57,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_simt_kernel(const AttnPa
   const int split = blockIdx.y;
   const int r = p.block_req[b];
   const int64_t c_begin = p.ctx_off[r];
-  const int64_t L = p.ctx_len ? static_cast<int64_t>(p.ctx_len[r]) : p.ctx_off[r + 1] - c_begin;
+  int64_t L = p.ctx_len ? static_cast<int64_t>(p.ctx_len[r]) : p.ctx_off[r + 1] - c_begin;
+  if (!DFL_BOUNDS(L >= 0 && L <= p.ctx_off[r + 1] - c_begin, p.status, 86)) L = 0;
   const int64_t k_lo = static_cast<int64_t>(split) * p.chunk;
   const int n_ctx = static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(L, k_lo + p.chunk) - k_lo));
   const int n_blk = split == 0 ? p.B : 0;
@@ -271,7 +272,8 @@ __global__ void __launch_bounds__(128, 3) attn_mma_kernel(const __grid_constant_
   const int nsplit = CS >= 1 ? CS : p.splits;
   const int r = p.block_req[b];
   const int64_t c_begin = p.ctx_off[r];
-  const int64_t L = p.ctx_len ? static_cast<int64_t>(p.ctx_len[r]) : p.ctx_off[r + 1] - c_begin;
+  int64_t L = p.ctx_len ? static_cast<int64_t>(p.ctx_len[r]) : p.ctx_off[r + 1] - c_begin;
+  if (!DFL_BOUNDS(L >= 0 && L <= p.ctx_off[r + 1] - c_begin, p.status, 85)) L = 0;
   const int64_t chunk = ((L + nsplit - 1) / nsplit + kMmaKeys - 1) / kMmaKeys * kMmaKeys;
   const int64_t k_lo = static_cast<int64_t>(split) * chunk;
   const int n_ctx = static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(L, k_lo + chunk) - k_lo));
@@ -704,11 +706,15 @@ AttnPlan plan_attn(int dtype, int nb, int B, int Hq, int Hkv, int d, int64_t max
       p.chunk = 64;
       return p;
     }
-    // enough CTAs to fill the GPU twice, and at most ~512 context keys per
-    // CTA for the longest request (each request divides its own context)
-    const int64_t max_splits = std::min<int64_t>(16, (max_ctx_len + 127) / 128);
-    const int64_t by_keys = (max_ctx_len + 511) / 512;
-    const int64_t n = std::max<int64_t>(1, std::min(std::max(want, by_keys), max_splits));
+    // Each request divides its own context into n splits.  Every CTA pays a
+    // fixed cost (Q fragments, ring fill, the cluster merge), so n doubles
+    // only while the grid stays within ~2.5 waves of resident CTAs (three
+    // per SM) and each split of the longest context keeps at least four
+    // 64-key tiles.
+    const int64_t slots = 3 * static_cast<int64_t>(kNumSMs);
+    int64_t n = 1;
+    while (n < 16 && base * (2 * n) * 2 <= 5 * slots && max_ctx_len / (2 * n) >= 4 * kMmaKeys)
+      n *= 2;
     while (p.cluster < n) p.cluster *= 2;
     int64_t chunk = (max_ctx_len + p.cluster - 1) / p.cluster;
     p.chunk = static_cast<int>((chunk + 63) / 64 * 64);

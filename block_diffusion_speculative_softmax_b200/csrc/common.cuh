@@ -26,6 +26,21 @@ __device__ __forceinline__ void report(uint32_t* status, uint32_t code,
   if (atomicCAS(status, 0u, code) == 0u) status[1] = where;
 }
 
+// Index checks of the debug-bounds build (-DDFLASH_DEBUG_BOUNDS): an index
+// read from device memory that falls outside its buffer records
+// DFLASH_EBOUNDS (with the site's tag) in the status word, and the caller
+// skips or clamps the access; nothing traps.  The release build compiles the
+// checks out (the macro is the constant true).
+#ifdef DFLASH_DEBUG_BOUNDS
+__device__ __forceinline__ bool bounds_check(bool ok, uint32_t* status, uint32_t where) {
+  if (!ok) report(status, DFLASH_EBOUNDS, where);
+  return ok;
+}
+#define DFL_BOUNDS(ok, status, where) (::dfl::bounds_check((ok), (status), (where)))
+#else
+#define DFL_BOUNDS(ok, status, where) (true)
+#endif
+
 // Bounded waits give up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 

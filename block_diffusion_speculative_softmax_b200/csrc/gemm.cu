@@ -98,6 +98,10 @@ struct Params {
   const float2* rope_tab;           // (cos, sin) [rope_len][head_dim / 2] or null
   int rope_len;
   double inv_freq[64];
+  const float* rss;                 // [M][rss_parts] row sums of squares, or null
+  int rss_parts;
+  float rss_inv;                    // 1 / hidden
+  float rss_eps;
   unsigned long long* keys;         // argmax mode: [M]
   float2* lse;                      // argmax mode: per (vocab tile, token) (max, sum exp)
   uint32_t* status;
@@ -113,6 +117,17 @@ __device__ __forceinline__ float2 rope_cs(const Params& p, int pos, int fi) {
   float sn, cs;
   sincosf(static_cast<float>(ang), &sn, &cs);
   return make_float2(cs, sn);
+}
+
+// RMSNorm scale of token row t when the input rows arrive unnormalised:
+// rsqrt(sum of the row's partial sums of squares / hidden + eps), the parts
+// added in a fixed order; 1 without one.
+__device__ __forceinline__ float rss_scale(const Params& p, int t) {
+  if (p.rss == nullptr) return 1.f;
+  const float* r = p.rss + static_cast<size_t>(t) * p.rss_parts;
+  float s = 0.f;
+  for (int w = 0; w < p.rss_parts; ++w) s += __ldg(r + w);
+  return rsqrtf(s * p.rss_inv + p.rss_eps);
 }
 
 // (cos, sin) of frequencies i0 .. i0 + 15 at `pos`: eight 16-byte table loads
@@ -443,11 +458,13 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
         for (int j0 = 0; j0 < BN; j0 += JU) {
           float2 cs[JU];
           int64_t orow[JU];
+          float rs[JU];
 #pragma unroll
           for (int q = 0; q < JU; ++q) {
             const int t = min(tok0 + j0 + q, p.M - 1);
             cs[q] = S.rope ? rope_cs(p, p.pos[t], fi) : make_float2(1.f, 0.f);
             orow[q] = S.use_dst ? p.dst[t] : t;
+            rs[q] = rss_scale(p, t);
           }
 #pragma unroll
           for (int q = 0; q < JU; ++q) {
@@ -458,6 +475,7 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(const __grid_constant__ Pa
               const float pv = st[(j0 + q) * SROW + prt];
               v = i < half ? v * cs[q].x - pv * cs[q].y : v * cs[q].x + pv * cs[q].y;
             }
+            v *= rs[q];
             if (S.op == EPI_STORE_F32)
               static_cast<float*>(S.out)[orow[q] * S.out_stride + f] = v;
             else
@@ -555,7 +573,12 @@ __device__ __forceinline__ void tok_row_epilogue(const Params& p, const Seg& S, 
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(S.out) + orow * S.out_stride;
     const int d = p.head_dim, half = d >> 1;
     const int pos = (tv && S.rope) ? p.pos[t] : 0;
-    auto put16 = [&](int f, const float* v) {
+    const float rs = tv ? rss_scale(p, t) : 1.f;
+    auto put16 = [&](int f, float* v) {
+      if (p.rss != nullptr) {
+#pragma unroll
+        for (int q = 0; q < 16; ++q) v[q] *= rs;
+      }
       if (S.op == EPI_STORE_F32) {
         float* of = static_cast<float*>(S.out) + orow * S.out_stride;
         if (f + 16 <= S.rows) {
@@ -1457,11 +1480,13 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
           for (int j0 = 0; j0 < BN; j0 += 8) {
             float2 cs[8];
             int64_t orow[8];
+            float rs[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const int t = min(tok0 + j0 + q, p.M - 1);
               cs[q] = S.rope ? rope_cs(p, p.pos[t], fi) : make_float2(1.f, 0.f);
               orow[q] = S.use_dst ? p.dst[t] : t;
+              rs[q] = rss_scale(p, t);
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -1472,6 +1497,7 @@ __global__ void __launch_bounds__(192, 1) gemm_sk_kernel(const __grid_constant__
                 const float pv = st[(j0 + q) * SROW + prt];
                 x = i < half ? x * cs[q].x - pv * cs[q].y : x * cs[q].x + pv * cs[q].y;
               }
+              x *= rs[q];
               if (S.op == EPI_STORE_F32)
                 static_cast<float*>(S.out)[orow[q] * S.out_stride + f] = x;
               else
@@ -1989,6 +2015,7 @@ GemmPlan plan_gemm(const GemmJob& job) {
 
 static cudaError_t launch_gemm_simt(const GemmJob& job, const GemmPlan& pl, float* partial,
                                     uint32_t* status, cudaStream_t st) {
+  if (job.rss != nullptr) return cudaErrorInvalidValue;   // bf16 paths only
   simt::Params p{};
   simt::FinishParams f{};
   int tiles = 0, col = 0, n = 0;
@@ -2089,6 +2116,10 @@ cudaError_t launch_gemm(const GemmJob& job, const GemmPlan& pl, float* partial,
   p.dst = job.dst;
   p.head_dim = job.head_dim > 0 ? job.head_dim : 128;
   p.rope_tab = job.rope_tab;
+  p.rss = job.rss;
+  p.rss_parts = job.rss_parts;
+  p.rss_inv = job.rss_inv;
+  p.rss_eps = job.rss_eps;
   p.rope_len = job.rope_len;
   fill_inv_freq(job.theta, p.head_dim, p.inv_freq);
   p.status = status;

@@ -55,6 +55,13 @@ struct GemmJob {
   double theta = 1e6;
   const float2* rope_tab = nullptr;   // (cos, sin) [rope_len][head_dim / 2]
   int rope_len = 0;
+  // EPI_STORE rows scaled by rsqrt(sum_w rss[m][w] * rss_inv + rss_eps) (the
+  // RMSNorm of an unnormalised input row; rss [M][rss_parts]; nullptr: no
+  // scale; bf16 tensor-core paths only)
+  const float* rss = nullptr;
+  int rss_parts = 0;
+  float rss_inv = 0.f;
+  float rss_eps = 0.f;
 };
 
 struct GemmPlan {
@@ -97,11 +104,19 @@ cudaError_t launch_lmhead_argmax(int dtype, const void* W, int V,
 cudaError_t launch_fuse(int dtype, const void* states, int64_t N, int T, int H,
                         int D, const float* w_fuse, const float* const* g_fuse,
                         void* fused, float eps, uint32_t* status, cudaStream_t st);
+// bf16 fusion for the step's context branch without the norm: fused[i][n] =
+// u_i * g_i and rss[i][n][w] = consumer warp w's share of sum(u_i^2), for
+// w < fuse_unnorm_parts(H); the context K/V GEMM applies rsqrt(sum / H + eps)
+// per row (GemmJob::rss).
+int fuse_unnorm_parts(int H);
+cudaError_t launch_fuse_unnorm(const void* states, int64_t N, int nT, int H, int D,
+                               const float* w_fuse, const float* const* g_fuse, void* fused,
+                               float* rss, uint32_t* status, cudaStream_t st);
 // Largest hidden size the fusion kernel covers for T target layers.
 int fuse_hidden_limit(int dtype, int nT);
 cudaError_t launch_embed(int dtype, const void* embed, int H, int nb, int B,
                          const int32_t* block_tokens, const int32_t* known_len,
-                         int mask_id, float* h, cudaStream_t st);
+                         int mask_id, int vocab, float* h, uint32_t* status, cudaStream_t st);
 cudaError_t launch_rmsnorm(int dtype, const float* h, int64_t M, int H,
                            const float* g, float eps, void* x, cudaStream_t st);
 cudaError_t launch_prep_rows(int R, int nb, int B, const int32_t* block_req,
@@ -110,7 +125,7 @@ cudaError_t launch_prep_rows(int R, int nb, int B, const int32_t* block_req,
                              const int32_t* new_count, int64_t n_new,
                              int32_t* blk_pos, int32_t* new_pos,
                              int64_t* new_dst, uint32_t* zero, int64_t n_zero,
-                             cudaStream_t st);
+                             uint32_t* status, cudaStream_t st);
 cudaError_t launch_advance(int R, int K, int B, int64_t row_bytes, const int32_t* n_acc,
                            const int32_t* best_k, const int32_t* out_tok, const void* verify_states,
                            int32_t* ctx_len, const int64_t* ctx_off, void* new_states,
@@ -179,13 +194,14 @@ cudaError_t launch_d2sd(int R, int B, int K, int mask_id, const int32_t* base,
 cudaError_t launch_sample_rows(const float* logits, int64_t M, int V, uint64_t seed,
                                uint32_t offset, int B, const int32_t* block_tokens,
                                const int32_t* known_len, int32_t* tok, float* logq,
-                               float* lse, cudaStream_t st);
+                               float* lse, uint32_t* status, cudaStream_t st);
 // Stochastic acceptance of one candidate per request; keys [R] scratch.
 cudaError_t launch_accept_stochastic(int R, int B, int V, const int32_t* draft,
                                      const float* draft_logits, const float* draft_lse,
                                      const float* target_logp, uint64_t seed, uint32_t offset,
                                      int32_t* n_acc, int32_t* out_tok,
-                                     unsigned long long* keys, cudaStream_t st);
+                                     unsigned long long* keys, uint32_t* status,
+                                     cudaStream_t st);
 cudaError_t launch_wait_selftest(uint32_t* status, int64_t limit_ns,
                                  cudaStream_t st);
 

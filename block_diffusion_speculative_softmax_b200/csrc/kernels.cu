@@ -40,6 +40,10 @@ __device__ __forceinline__ void fmul2(float& d0, float& d1, float b0, float b1) 
       : "+f"(d0), "+f"(d1) : "f"(b0), "f"(b1));
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 constexpr int kFuseThreads = 512;
 constexpr int kFuseSmemBudget = 221 * 1024;
 
@@ -221,6 +225,204 @@ __global__ void __launch_bounds__(kFuseThreads) fuse_rows_kernel(
   }
 }
 
+// Sums each of NV values over the warp (NV a power of two <= 32): afterwards
+// v[0] of lane l holds the warp total of value l / (32 / NV).  Each halving
+// step exchanges half of the values still held, so NV values take
+// NV - 1 + log2(32 / NV) shuffles instead of 5 NV.
+template <int NV>
+__device__ __forceinline__ void warp_sum_multi(float (&v)[NV], int lane) {
+#pragma unroll
+  for (int cnt = NV, off = 16; cnt > 1; cnt >>= 1, off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int k = 0; k < cnt / 2; ++k) {
+      const float send = up ? v[k] : v[k + cnt / 2];
+      const float keep = up ? v[k + cnt / 2] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+#pragma unroll
+  for (int off = 16 / NV; off >= 1; off >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+}
+
+// ---------------------------------------------------------------------------
+// Fusion for the draft step's context branch, without the norm.  RMSNorm is
+// a per-row scale: f_i = (u_i * g_i) * rsqrt(mean(u_i^2) + eps).  This
+// variant stores v_i = u_i * g_i and adds each warp's share of sum(u_i^2)
+// to rss[i][n][w] (one slot per consumer warp w, so the sum's order is
+// fixed); the context K/V GEMM applies the row's rsqrt(sum / H + eps) to its
+// accumulator row in the epilogue (K and V are
+// linear in f, and RoPE commutes with a scalar).  With no cross-warp
+// reduction per row, warps never wait for one another: the last warp done
+// reading a ring slot (a shared counter) issues the slot's next row.
+// ---------------------------------------------------------------------------
+template <typename T, int MAXD>
+__global__ void __launch_bounds__(kFuseThreads) fuse_rows_unnorm_kernel(
+    const T* __restrict__ states, int64_t N, int nT, int H, int D,
+    const float* __restrict__ w_fuse, const FuseGains gains, T* __restrict__ fused,
+    float* __restrict__ rss, int slots, uint32_t* status) {
+  using V = Vec16<T>;
+  constexpr int VE = V::N;
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ __align__(8) uint64_t full[8];
+  __shared__ int done_cnt[8];      // warps done with the slot's current row
+  __shared__ int64_t last_k[8];    // latest row loaded into the slot
+  __shared__ __align__(16) float alpha[kMaxTargetLayers][MAXD];
+  __shared__ volatile int abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ncw = blockDim.x >> 5;
+  const uint32_t row_bytes = static_cast<uint32_t>(nT) * H * sizeof(T);
+  pdl_wait();
+  if (tid == 0) pdl_launch();
+  if (tid == 0) {
+    for (int s = 0; s < slots; ++s) {
+      mbar_init(&full[s], 1);
+      done_cnt[s] = 0;
+      last_k[s] = -1;
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (tid < MAXD) {
+    if (tid < D) {
+      float mx = -INFINITY;
+      for (int j = 0; j < nT; ++j) mx = fmaxf(mx, w_fuse[tid * nT + j]);
+      float sum = 0.f;
+      for (int j = 0; j < nT; ++j) {
+        const float e = expf(w_fuse[tid * nT + j] - mx);
+        alpha[j][tid] = e;
+        sum += e;
+      }
+      for (int j = 0; j < nT; ++j) alpha[j][tid] /= sum;
+    } else {
+      for (int j = 0; j < nT; ++j) alpha[j][tid] = 0.f;
+    }
+  }
+  __syncthreads();
+  const int64_t my_rows = N > blockIdx.x ? (N - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  auto issue = [&](int64_t k) {   // row k of this CTA into slot k % slots
+    const int slot = static_cast<int>(k % slots);
+    const int64_t n = blockIdx.x + k * static_cast<int64_t>(gridDim.x);
+    last_k[slot] = k;
+    mbar_arrive_expect_tx(&full[slot], row_bytes);
+    bulk_load(ring + static_cast<size_t>(slot) * row_bytes, states + n * nT * H, row_bytes,
+              &full[slot]);
+  };
+  if (tid == 0)
+    for (int64_t k = 0; k < slots && k < my_rows; ++k) issue(k);
+  const int nvec = H / VE;
+  const bool active = tid < nvec;
+  const int col = tid * VE;
+  constexpr int GW = 3;   // layers whose gains are in flight ahead of their use
+  auto load_gain = [&](float4 (&g)[VE / 4], int i) {
+#pragma unroll
+    for (int q = 0; q < VE / 4; ++q)
+      g[q] = (active && i < D) ? __ldg(reinterpret_cast<const float4*>(gains.g[i] + col) + q)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  for (int64_t k = 0; k < my_rows; ++k) {
+    const int slot = static_cast<int>(k % slots);
+    const int64_t n = blockIdx.x + k * static_cast<int64_t>(gridDim.x);
+    // the gains are the same for every row: the first GW layers' load while
+    // the row arrives and is summed
+    float4 gq[GW][VE / 4];
+#pragma unroll
+    for (int w = 0; w < GW; ++w) load_gain(gq[w], w);
+    const bool ok = mbar_wait(&full[slot], static_cast<uint32_t>((k / slots) & 1), status, 26);
+    if (!ok) abort_flag = 1;
+    float u[MAXD][VE];
+#pragma unroll
+    for (int i = 0; i < MAXD; ++i)
+#pragma unroll
+      for (int e = 0; e < VE; ++e) u[i][e] = 0.f;
+    if (active && ok) {
+      const T* row = reinterpret_cast<const T*>(ring + static_cast<size_t>(slot) * row_bytes);
+      for (int j = 0; j < nT; ++j) {
+        float h[VE];
+        const uint4 raw = *reinterpret_cast<const uint4*>(row + static_cast<size_t>(j) * H + col);
+        if constexpr (VE == 8) {
+          const __nv_bfloat162* hp = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(hp[q]);
+            h[2 * q] = f.x;
+            h[2 * q + 1] = f.y;
+          }
+        } else {
+          const float* fp = reinterpret_cast<const float*>(&raw);
+#pragma unroll
+          for (int q = 0; q < VE; ++q) h[q] = fp[q];
+        }
+        float a[MAXD];
+#pragma unroll
+        for (int q = 0; q < MAXD / 4; ++q) {
+          const float4 av = *reinterpret_cast<const float4*>(&alpha[j][4 * q]);
+          a[4 * q] = av.x; a[4 * q + 1] = av.y; a[4 * q + 2] = av.z; a[4 * q + 3] = av.w;
+        }
+#pragma unroll
+        for (int i = 0; i < MAXD; ++i) {
+          if (i < D) {
+#pragma unroll
+            for (int e = 0; e < VE; e += 2) ffma2(u[i][e], u[i][e + 1], a[i], a[i], h[e], h[e + 1]);
+          }
+        }
+      }
+    }
+    // this warp is done with the slot: the last warp to finish refills it
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence_block();
+      if (atomicAdd(&done_cnt[slot], 1) == ncw - 1) {
+        done_cnt[slot] = 0;
+        __threadfence_block();
+        if (abort_flag == 0 && k + slots < my_rows) issue(k + slots);
+      }
+    }
+    if (__any_sync(0xffffffffu, abort_flag != 0)) break;
+    // this warp's share of every layer's sum of squares (u_i = 0 past D),
+    // all layers reduced over the warp together
+    float ss[MAXD];
+#pragma unroll
+    for (int i = 0; i < MAXD; ++i) {
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int e = 0; e < VE; e += 2) ffma2(s0, s1, u[i][e], u[i][e + 1], u[i][e], u[i][e + 1]);
+      ss[i] = s0 + s1;
+    }
+    warp_sum_multi<MAXD>(ss, lane);
+    {
+      constexpr int per = 32 / MAXD;
+      const int li = lane / per;
+      if (lane % per == 0 && li < D) rss[(static_cast<size_t>(li) * N + n) * ncw + warp] = ss[0];
+    }
+    // v_i = u_i * g_i, with layer i + GW's gains loading meanwhile
+#pragma unroll
+    for (int i = 0; i < MAXD; ++i) {
+      if (i < D) {
+        float4 gv[VE / 4];
+#pragma unroll
+        for (int q = 0; q < VE / 4; ++q) gv[q] = gq[i % GW][q];
+        if (i + GW < D) load_gain(gq[i % GW], i + GW);
+        if (active) {
+#pragma unroll
+          for (int q = 0; q < VE / 4; ++q) {
+            fmul2(u[i][4 * q], u[i][4 * q + 1], gv[q].x, gv[q].y);
+            fmul2(u[i][4 * q + 2], u[i][4 * q + 3], gv[q].z, gv[q].w);
+          }
+          V::store(fused + (static_cast<size_t>(i) * N + n) * H + col, u[i]);
+        }
+      }
+    }
+  }
+  // after a wait that ran out, let the loads still in flight land before the
+  // CTA's shared memory goes away (the latest load of each slot)
+  __syncthreads();
+  if (abort_flag && tid == 0)
+    for (int s = 0; s < slots; ++s)
+      if (last_k[s] >= 0)
+        mbar_wait(&full[s], static_cast<uint32_t>((last_k[s] / slots) & 1), status, 27);
+}
+
 // Ring depth: rows of up to ~96 KB in flight per CTA (two CTAs per SM fit
 // when the ring is small), never fewer than two rows.
 template <typename T>
@@ -274,6 +476,56 @@ static cudaError_t launch_fuse_t(const void* states, int64_t N, int nT, int H, i
   return fuse_go<T, 16>(states, N, nT, H, D, w_fuse, g, fused, eps, status, st);
 }
 
+template <int MAXD>
+static cudaError_t fuse_unnorm_go(const void* states, int64_t N, int nT, int H, int D,
+                                  const float* w_fuse, const FuseGains& g, void* fused,
+                                  float* rss, uint32_t* status, cudaStream_t st) {
+  using T = __nv_bfloat16;
+  const int nvec = H / Vec16<T>::N;
+  const int threads = ((nvec + 31) / 32) * 32;
+  const int rb = nT * H * static_cast<int>(sizeof(T));
+  int slots = fuse_slots<T>(nT, H);
+  size_t smem = static_cast<size_t>(slots) * rb;
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(fuse_rows_unnorm_kernel<T, MAXD>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kFuseSmemBudget);
+  });
+  if (attr != cudaSuccess) return attr;
+  // two CTAs per SM when registers and the small ring allow it; otherwise
+  // one, with as many rows in flight as the shared-memory budget holds
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+      &per_sm, fuse_rows_unnorm_kernel<T, MAXD>, threads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 2) {
+    per_sm = 1;
+    slots = std::max(2, std::min(8, kFuseSmemBudget / rb));
+    smem = static_cast<size_t>(slots) * rb;
+  } else {
+    per_sm = 2;
+  }
+  const int grid = static_cast<int>(std::min<int64_t>(N, kNumSMs * per_sm));
+  return launch_k(fuse_rows_unnorm_kernel<T, MAXD>, dim3(grid), dim3(threads), smem, st,
+                  static_cast<const T*>(states), N, nT, H, D, w_fuse, g, static_cast<T*>(fused),
+                  rss, slots, status);
+}
+
+int fuse_unnorm_parts(int H) { return (H / Vec16<__nv_bfloat16>::N + 31) / 32; }
+
+cudaError_t launch_fuse_unnorm(const void* states, int64_t N, int nT, int H, int D,
+                               const float* w_fuse, const float* const* g_fuse, void* fused,
+                               float* rss, uint32_t* status, cudaStream_t st) {
+  if (N <= 0) return cudaSuccess;
+  if (H > fuse_max_hidden<__nv_bfloat16>(nT)) return cudaErrorInvalidValue;
+  FuseGains g{};
+  for (int i = 0; i < D; ++i) g.g[i] = g_fuse[i];
+  if (D <= 4) return fuse_unnorm_go<4>(states, N, nT, H, D, w_fuse, g, fused, rss, status, st);
+  if (D <= 8) return fuse_unnorm_go<8>(states, N, nT, H, D, w_fuse, g, fused, rss, status, st);
+  return fuse_unnorm_go<16>(states, N, nT, H, D, w_fuse, g, fused, rss, status, st);
+}
+
 int fuse_hidden_limit(int dtype, int nT) {
   return dtype == DFLASH_BF16 ? fuse_max_hidden<__nv_bfloat16>(nT) : fuse_max_hidden<float>(nT);
 }
@@ -295,14 +547,15 @@ cudaError_t launch_fuse(int dtype, const void* states, int64_t N, int nT, int H,
 template <typename T>
 __global__ void embed_kernel(const T* __restrict__ embed, int H, int B,
                              const int32_t* __restrict__ block_tokens,
-                             const int32_t* __restrict__ known_len, int mask_id,
-                             float* __restrict__ h) {
+                             const int32_t* __restrict__ known_len, int mask_id, int vocab,
+                             float* __restrict__ h, uint32_t* status) {
   pdl_wait();
   if (threadIdx.x == 0) pdl_launch();
   const int m = blockIdx.x;
   const int b = m / B, s = m % B;
   const int kl = known_len ? known_len[b] : 1;
-  const int tok = s < kl ? block_tokens[m] : mask_id;
+  int tok = s < kl ? block_tokens[m] : mask_id;
+  if (!DFL_BOUNDS(tok >= 0 && tok < vocab, status, 87)) tok = mask_id;
   const T* src = embed + static_cast<size_t>(tok) * H;
   for (int c = threadIdx.x; c < H; c += blockDim.x)
     h[static_cast<size_t>(m) * H + c] = to_f(src[c]);
@@ -310,14 +563,15 @@ __global__ void embed_kernel(const T* __restrict__ embed, int H, int B,
 
 cudaError_t launch_embed(int dtype, const void* embed, int H, int nb, int B,
                          const int32_t* block_tokens, const int32_t* known_len, int mask_id,
-                         float* h, cudaStream_t st) {
+                         int vocab, float* h, uint32_t* status, cudaStream_t st) {
   if (nb <= 0) return cudaSuccess;
   if (dtype == DFLASH_BF16)
     return launch_k(embed_kernel<__nv_bfloat16>, dim3(nb * B), dim3(256), 0, st,
                     static_cast<const __nv_bfloat16*>(embed), H, B, block_tokens, known_len,
-                    mask_id, h);
+                    mask_id, vocab, h, status);
   return launch_k(embed_kernel<float>, dim3(nb * B), dim3(256), 0, st,
-                  static_cast<const float*>(embed), H, B, block_tokens, known_len, mask_id, h);
+                  static_cast<const float*>(embed), H, B, block_tokens, known_len, mask_id, vocab,
+                  h, status);
 }
 
 // ===========================================================================
@@ -392,7 +646,7 @@ __global__ void prep_rows_kernel(int R, int nb, int B, const int32_t* __restrict
                                  const int32_t* __restrict__ new_count, int64_t n_new,
                                  int32_t* __restrict__ blk_pos, int32_t* __restrict__ new_pos,
                                  int64_t* __restrict__ new_dst, uint32_t* __restrict__ zero,
-                                 int64_t n_zero) {
+                                 int64_t n_zero, uint32_t* status) {
   pdl_wait();
   if (threadIdx.x == 0) pdl_launch();
   const int64_t tid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
@@ -400,7 +654,12 @@ __global__ void prep_rows_kernel(int R, int nb, int B, const int32_t* __restrict
   for (int64_t i = tid; i < n_zero; i += stride) zero[i] = 0u;
   for (int64_t m = tid; m < static_cast<int64_t>(nb) * B; m += stride) {
     const int r = block_req[m / B];
+    if (!DFL_BOUNDS(r >= 0 && r < R, status, 81)) {
+      blk_pos[m] = 0;
+      continue;
+    }
     const int64_t L = ctx_len ? static_cast<int64_t>(ctx_len[r]) : ctx_off[r + 1] - ctx_off[r];
+    (void)DFL_BOUNDS(L >= 0 && L <= ctx_off[r + 1] - ctx_off[r], status, 82);
     blk_pos[m] = static_cast<int32_t>(L + m % B);
   }
   if (new_count != nullptr) {
@@ -409,8 +668,9 @@ __global__ void prep_rows_kernel(int R, int nb, int B, const int32_t* __restrict
     for (int64_t n = tid; n < n_new; n += stride) {
       const int r = static_cast<int>(n / B), j = static_cast<int>(n % B);
       const int c = new_count[r];
-      if (j < c) {
-        const int64_t p = static_cast<int64_t>(ctx_len[r]) - c + j;
+      const int64_t p = static_cast<int64_t>(ctx_len[r]) - c + j;
+      if (j < c &&
+          DFL_BOUNDS(c <= B && p >= 0 && ctx_off[r] + p < ctx_off[r + 1], status, 83)) {
         new_pos[n] = static_cast<int32_t>(p);
         new_dst[n] = ctx_off[r] + p;
       } else {
@@ -428,8 +688,9 @@ __global__ void prep_rows_kernel(int R, int nb, int B, const int32_t* __restrict
       if (off[mid] <= n) lo = mid; else hi = mid - 1;
     }
     const int64_t p = (ctx_cached ? ctx_cached[lo] : 0) + (n - off[lo]);
-    new_pos[n] = static_cast<int32_t>(p);
-    new_dst[n] = ctx_off[lo] + p;
+    const bool in = DFL_BOUNDS(p >= 0 && ctx_off[lo] + p < ctx_off[lo + 1], status, 84);
+    new_pos[n] = in ? static_cast<int32_t>(p) : 0;
+    new_dst[n] = in ? ctx_off[lo] + p : -1;
   }
 }
 
@@ -438,14 +699,14 @@ cudaError_t launch_prep_rows(int R, int nb, int B, const int32_t* block_req,
                              const int32_t* ctx_cached, const int32_t* ctx_len,
                              const int32_t* new_count, int64_t n_new, int32_t* blk_pos,
                              int32_t* new_pos, int64_t* new_dst, uint32_t* zero, int64_t n_zero,
-                             cudaStream_t st) {
+                             uint32_t* status, cudaStream_t st) {
   const int64_t work =
       std::max(std::max<int64_t>(static_cast<int64_t>(nb) * B, n_new), n_zero);
   if (work <= 0) return cudaSuccess;
   const int grid = static_cast<int>(std::min<int64_t>((work + 255) / 256, kNumSMs * 8));
   return launch_k(prep_rows_kernel, dim3(grid), dim3(256), 0, st, R, nb, B, block_req, ctx_off,
                   new_off, ctx_cached, ctx_len, new_count, n_new, blk_pos, new_pos, new_dst, zero,
-                  n_zero);
+                  n_zero, status);
 }
 
 struct InvFreq {

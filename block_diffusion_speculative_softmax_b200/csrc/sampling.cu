@@ -57,7 +57,8 @@ template <bool VEC4>
 __global__ void __launch_bounds__(kSampleThreads) sample_rows_kernel(
     const float* __restrict__ logits, int V, uint32_t k0, uint32_t k1, uint32_t offset, int B,
     const int32_t* __restrict__ block_tokens, const int32_t* __restrict__ known_len,
-    int32_t* __restrict__ tok, float* __restrict__ logq, float* __restrict__ lse_out) {
+    int32_t* __restrict__ tok, float* __restrict__ logq, float* __restrict__ lse_out,
+    uint32_t* status) {
   __shared__ unsigned long long s_key[kSampleThreads / 32];
   __shared__ float s_m[kSampleThreads / 32], s_s[kSampleThreads / 32];
   pdl_wait();
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(kSampleThreads) sample_rows_kernel(
       const int kl = known_len ? known_len[b] : 1;
       if (m % B < kl) t = block_tokens[m];
     }
+    if (!DFL_BOUNDS(t >= 0 && t < V, status, 89)) t = 0;
     tok[m] = t;
     if (logq) logq[m] = row[t] - lse;
     if (lse_out) lse_out[m] = lse;
@@ -126,16 +128,16 @@ __global__ void __launch_bounds__(kSampleThreads) sample_rows_kernel(
 cudaError_t launch_sample_rows(const float* logits, int64_t M, int V, uint64_t seed,
                                uint32_t offset, int B, const int32_t* block_tokens,
                                const int32_t* known_len, int32_t* tok, float* logq,
-                               float* lse, cudaStream_t st) {
+                               float* lse, uint32_t* status, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
   const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
   const bool vec = (V % 4) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
   const dim3 grid(static_cast<unsigned>(M));
   if (vec)
     return launch_k(sample_rows_kernel<true>, grid, dim3(kSampleThreads), 0, st, logits, V, k0,
-                    k1, offset, B, block_tokens, known_len, tok, logq, lse);
+                    k1, offset, B, block_tokens, known_len, tok, logq, lse, status);
   return launch_k(sample_rows_kernel<false>, grid, dim3(kSampleThreads), 0, st, logits, V, k0,
-                  k1, offset, B, block_tokens, known_len, tok, logq, lse);
+                  k1, offset, B, block_tokens, known_len, tok, logq, lse, status);
 }
 
 // ---------------------------------------------------------------------------
@@ -150,7 +152,7 @@ __global__ void accept_decide_kernel(int R, int B, int V, const int32_t* __restr
                                      const float* __restrict__ target_logp, uint32_t k0,
                                      uint32_t k1, uint32_t offset, int32_t* __restrict__ n_acc,
                                      int32_t* __restrict__ out_tok,
-                                     unsigned long long* __restrict__ keys) {
+                                     unsigned long long* __restrict__ keys, uint32_t* status) {
   pdl_wait();
   if (threadIdx.x == 0) pdl_launch();
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -159,7 +161,8 @@ __global__ void accept_decide_kernel(int R, int B, int V, const int32_t* __restr
   bool ok = false;
   if (lane >= 1 && lane < B) {
     const size_t row = static_cast<size_t>(r) * B + lane;
-    const int32_t d = draft[row];
+    int32_t d = draft[row];
+    if (!DFL_BOUNDS(d >= 0 && d < V, status, 88)) d = 0;
     const float lq = draft_logits[row * V + d] - draft_lse[row];
     const float lp = target_logp[(row - 1) * V + d];
     const uint4 w = philox4x32_10(make_uint4(static_cast<uint32_t>(lane),
@@ -244,13 +247,14 @@ cudaError_t launch_accept_stochastic(int R, int B, int V, const int32_t* draft,
                                      const float* draft_logits, const float* draft_lse,
                                      const float* target_logp, uint64_t seed, uint32_t offset,
                                      int32_t* n_acc, int32_t* out_tok,
-                                     unsigned long long* keys, cudaStream_t st) {
+                                     unsigned long long* keys, uint32_t* status,
+                                     cudaStream_t st) {
   if (R <= 0) return cudaSuccess;
   const uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
   const int wpb = 4;
   cudaError_t e = launch_k(accept_decide_kernel, dim3((R + wpb - 1) / wpb), dim3(wpb * 32), 0,
                            st, R, B, V, draft, draft_logits, draft_lse, target_logp, k0, k1,
-                           offset, n_acc, out_tok, keys);
+                           offset, n_acc, out_tok, keys, status);
   if (e != cudaSuccess) return e;
   // enough CTAs to stream the two rows of every request at full bandwidth
   const int nq = (V + 3) / 4;

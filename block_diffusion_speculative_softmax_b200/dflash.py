@@ -35,11 +35,13 @@ from typing import List, Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdflash.so")
+# DFLASH_LIB selects another build of the same ABI (e.g. the debug-bounds
+# libdflash_debug.so that `build --debug-bounds` writes beside this one).
+LIB_PATH = os.environ.get("DFLASH_LIB") or os.path.join(_HERE, "libdflash.so")
 
-OK, EINVAL, EUNSUPPORTED, ECUDA, ETIMEOUT, ENUMERIC = range(6)
+OK, EINVAL, EUNSUPPORTED, ECUDA, ETIMEOUT, ENUMERIC, EBOUNDS = range(7)
 STATUS_NAMES = {0: "OK", 1: "EINVAL", 2: "EUNSUPPORTED", 3: "ECUDA", 4: "ETIMEOUT",
-                5: "ENUMERIC"}
+                5: "ENUMERIC", 6: "EBOUNDS"}
 FP32, BF16 = 0, 1
 
 
@@ -98,6 +100,9 @@ SIGNATURES = {
     "dflash_version": (C.c_char_p, []),
     "dflash_fuse_ctx": (C.c_int, [_CFG, _VP, _I64, _VP, C.POINTER(_VP), _VP, _VP]),
     "dflash_fc_fuse_ctx": (C.c_int, [_CFG, _VP, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "dflash_fuse_rss_parts": (C.c_int32, [C.c_int32]),
+    "dflash_fuse_ctx_rss": (C.c_int, [_CFG, _VP, _I64, _VP, C.POINTER(_VP), _VP, _VP, _VP, _SZ,
+                                      _VP]),
     "dflash_kv_project": (C.c_int, [_CFG, _VP, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ,
                                     _VP]),
     "dflash_block_attn": (C.c_int, [_CFG, _I32, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I64, _VP,
@@ -217,6 +222,18 @@ def dflash_fuse_ctx(cfg: Config, states: torch.Tensor, w_fuse: torch.Tensor,
     arr = (C.c_void_p * len(g_fuse))(*[g.data_ptr() for g in g_fuse])
     _check(load().dflash_fuse_ctx(C.byref(cfg), _p(states), states.shape[0], _p(w_fuse), arr,
                                   _p(fused), _stream(stream)))
+
+
+def dflash_fuse_rss_parts(hidden: int) -> int:
+    return int(load().dflash_fuse_rss_parts(hidden))
+
+
+def dflash_fuse_ctx_rss(cfg: Config, states: torch.Tensor, w_fuse: torch.Tensor,
+                        g_fuse: Sequence[torch.Tensor], fused: torch.Tensor, rss: torch.Tensor,
+                        ws, stream=None):
+    arr = (C.c_void_p * len(g_fuse))(*[g.data_ptr() for g in g_fuse])
+    _check(load().dflash_fuse_ctx_rss(C.byref(cfg), _p(states), states.shape[0], _p(w_fuse), arr,
+                                      _p(fused), _p(rss), _p(ws), ws.numel(), _stream(stream)))
 
 
 def dflash_fc_fuse_ctx(cfg: Config, states: torch.Tensor, w_fc: torch.Tensor,

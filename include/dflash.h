@@ -59,7 +59,12 @@ typedef enum {
   DFLASH_EUNSUPPORTED = 2, /* valid but not covered (e.g. head_dim 96) */
   DFLASH_ECUDA = 3,        /* a CUDA runtime call failed */
   DFLASH_ETIMEOUT = 4,     /* a bounded device-side wait ran out */
-  DFLASH_ENUMERIC = 5      /* a non-finite logit reached the LM-head argmax */
+  DFLASH_ENUMERIC = 5,     /* a non-finite logit reached the LM-head argmax */
+  DFLASH_EBOUNDS = 6       /* debug-bounds build only (libdflash_debug.so, compiled
+                            * with -DDFLASH_DEBUG_BOUNDS): an index read from
+                            * device memory (a request id, a context length, a
+                            * new-row count, a token id) fell outside its
+                            * buffer; the access was skipped, no trap */
 } dflash_status;
 
 typedef enum { DFLASH_FP32 = 0, DFLASH_BF16 = 1 } dflash_dtype;
@@ -133,7 +138,8 @@ dflash_status dflash_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then read and clear the device status recorded in
  * the workspace header by earlier calls that used `ws`.  Returns DFLASH_OK,
- * DFLASH_ETIMEOUT, DFLASH_ENUMERIC or DFLASH_ECUDA. */
+ * DFLASH_ETIMEOUT, DFLASH_ENUMERIC, DFLASH_EBOUNDS (debug-bounds build) or
+ * DFLASH_ECUDA. */
 dflash_status dflash_check(void* ws, void* stream);
 
 /* Message describing the last error returned to the calling thread. */
@@ -159,6 +165,24 @@ dflash_status dflash_fuse_ctx(const dflash_config* cfg, const void* states,
                               int64_t n_rows, const float* w_fuse,
                               const float* const* g_fuse, void* fused,
                               void* stream);
+
+/* The draft step's split form of the same fusion (bf16 only).  RMSNorm is
+ * one scalar per row, and the context K/V projection and RoPE are linear, so
+ * dflash_draft_step applies the row scale in the projection's epilogue: the
+ * fusion stores the rows unnormalised and needs no cross-warp reduction per
+ * row.  Outputs:
+ *   fused[i, n, :] = u * g_fuse[i][:]                    [D][N][H] bf16
+ *   rss[i][n][w]   = partial sums of u^2, w < P          [D][N][P] fp32
+ * with P = dflash_fuse_rss_parts(hidden) and sum_w rss[i][n][w] = sum(u^2),
+ * the parts added in a fixed order, so that
+ *   dflash_fuse_ctx's fused[i, n, :] = fused[i, n, :] / sqrt(sum_w rss[i][n][w] / H + eps).
+ * ws: a workspace of at least 256 bytes (its header takes the device status;
+ * read it with dflash_check).  N may be 0 (no launch). */
+int32_t dflash_fuse_rss_parts(int32_t hidden);
+dflash_status dflash_fuse_ctx_rss(const dflash_config* cfg, const void* states,
+                                  int64_t n_rows, const float* w_fuse,
+                                  const float* const* g_fuse, void* fused, float* rss,
+                                  void* ws, size_t ws_bytes, void* stream);
 
 /* DFlash-style FC context fusion (DFLARE summary, section 1 item 1 and
  * section 2.2): states [N][T][H] (dtype), viewed as [N][T*H] ->

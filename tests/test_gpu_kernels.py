@@ -59,6 +59,40 @@ def test_fuse_ctx(DF, dtype, H, T, D, N):
     assert rel_err(out.float().cpu().numpy(), want) <= TOL[dtype]
 
 
+# The draft step's split fusion: unnormalised u * g plus per-warp partial sums
+# of u^2; applying the row scale here (test arithmetic) must give the fused
+# context of the oracle.  D up to 16 and T up to 9 (one and two CTAs per SM,
+# ragged N over the persistent grid).
+@pytest.mark.parametrize("H,T,D,N", [(576, 5, 3, 300), (2560, 5, 5, 2048), (4096, 9, 7, 301),
+                                     (2880, 5, 5, 37), (1024, 3, 16, 500)])
+def test_fuse_ctx_rss(DF, H, T, D, N):
+    cfg = _cfg("bf16", hidden=H, n_target_layers=T, n_draft_layers=D)
+    rng = np.random.default_rng(7 * H + N)
+    st = _round(cfg, rng.standard_normal((N, T, H)))
+    wf = rng.standard_normal((D, T)).astype(np.float32)
+    g = _round(cfg, 1 + 0.02 * rng.standard_normal((D, H)))
+    ccfg = DF.config_from(cfg)
+    P = DF.dflash_fuse_rss_parts(H)
+    assert P == -(-(H // 8) // 32)
+    gd = [to_dev(g[i], torch.float32) for i in range(D)]
+    v = torch.empty(D, N, H, dtype=torch.bfloat16, device="cuda")
+    rss = torch.full((D, N, P), float("nan"), device="cuda")
+    ws = DF.alloc_workspace(1 << 12)
+    DF.dflash_fuse_ctx_rss(ccfg, to_dev(st, torch.bfloat16), to_dev(wf, torch.float32), gd, v,
+                           rss, ws)
+    DF.dflash_check(ws)
+    ss = rss.double().sum(-1, keepdim=True).cpu().numpy()
+    assert np.all(np.isfinite(ss))
+    got = v.double().cpu().numpy() / np.sqrt(ss / H + cfg.rms_eps)
+    want = O.fuse_ctx(st, wf, g, cfg.rms_eps, bf16_storage=True)
+    assert rel_err(got, want) <= TOL["bf16"]
+    # the sums of squares themselves, against the oracle's weighted sum
+    a = np.exp(wf - wf.max(1, keepdims=True))
+    a /= a.sum(1, keepdims=True)
+    u = np.einsum("it,nth->inh", a.astype(np.float64), st.astype(np.float64))
+    np.testing.assert_allclose(ss[..., 0], (u * u).sum(-1), rtol=1e-4)
+
+
 # DFlash-style FC fusion: one Linear(T*H -> H) + RMSNorm shared by all layers
 @pytest.mark.parametrize("dtype,H,T,N", [("fp32", 256, 3, 37), ("bf16", 576, 5, 300),
                                          ("bf16", 2560, 5, 2048), ("bf16", 4096, 9, 65),
