@@ -164,3 +164,23 @@ def test_workspace_size_is_monotone_in_blocks_and_rows():
             for (nb2, n2), v2 in sizes.items():
                 if nb2 <= nb and n2 <= n_new:
                     assert v2 <= v, ((nb, n_new, v), (nb2, n2, v2))
+
+
+def test_fuse_rss_parts_is_one_per_warp_of_columns(lib):
+    # one partial sum of squares per 32 threads x 8 bf16 columns
+    for H, parts in [(4096, 16), (2880, 12), (2560, 10), (576, 3), (64, 1)]:
+        assert DF.dflash_fuse_rss_parts(H) == parts
+    assert DF.dflash_fuse_rss_parts(0) == 0
+
+
+def test_split_fusion_rejects_fp32_and_bad_arguments(lib):
+    cfg = DF.config_from(synth.get_config("tiny"))          # fp32 model
+    assert lib.dflash_fuse_ctx_rss(C.byref(cfg), None, 0, None, None, None, None, None, 0,
+                                   None) == DF.EUNSUPPORTED
+    cfg = DF.config_from(synth.small_config("qwen3_4b", hidden=576, n_q_heads=8, n_kv_heads=2,
+                                            head_dim=128, ffn=1000, n_draft_layers=2,
+                                            n_target_layers=3, ctx_len=64, block=16,
+                                            vocab=1000, dtype="bf16"))
+    # no workspace for the status word
+    assert lib.dflash_fuse_ctx_rss(C.byref(cfg), None, 0, None, None, None, None, None, 0,
+                                   None) == DF.EINVAL
