@@ -755,18 +755,28 @@ def run_op(args):
             call = lambda: DF.dflash_fuse_ctx(cc, st, wf, gl, fused)
             algo = N * T * H * e + D * N * H * e
             kernel = "fuse_rows_kernel (fusion + RMSNorm, all draft layers)"
-    for _ in range(args.warmup):
-        call()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        call()
-    e1.record()
-    e1.synchronize()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        e1.synchronize()
+        return e0.elapsed_time(e1) / args.steps / 1e3
+
+    sec = timed(call)
     DF.dflash_check(ws)
-    sec = e0.elapsed_time(e1) / args.steps / 1e3
+    extra = {}
+    if args.op == "lmhead" and M <= 4096:
+        # the allocation-free entry point on the same inputs (<= 64 tokens it
+        # takes the one-CTA-per-tile kernel instead of stream-K)
+        s2 = timed(lambda: DF.dflash_lmhead_argmax_noalloc(cc, x, w, tok))
+        extra = {"noalloc_us_per_call": s2 * 1e6, "noalloc_hbm_frac": algo / s2 / 1e9 / hbm}
     line = {"mode": "op", "op": args.op, "kernel": kernel, "workload": cfg.name,
             "us_per_call": sec * 1e6, "algorithmic_bytes": algo,
             "achieved_gbs": algo / sec / 1e9, "hbm_peak_gbs": hbm, "hbm_frac": algo / sec / 1e9 / hbm,
@@ -774,6 +784,7 @@ def run_op(args):
     if flops:
         line.update({"flops": flops, "achieved_tflops": flops / sec / 1e12,
                      "tensor_peak_tflops": tfb, "tensor_frac": flops / sec / 1e12 / tfb})
+    line.update(extra)
     print(json.dumps(line), flush=True)
 
 

@@ -182,8 +182,14 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
 }
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+// a register-only instruction: not volatile, so the compiler may interleave
+// independent MMAs with the fragment loads
 __device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
       "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -365,16 +371,18 @@ __global__ void __launch_bounds__(128, 3) attn_mma_kernel(const __grid_constant_
   auto process = [&](uint32_t kbase, uint32_t vbase, int nvalid) {
     float sc[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    // k-step outer, key tile inner: consecutive MMAs accumulate into
+    // different tiles
 #pragma unroll
-      for (int k2 = 0; k2 < KS; k2 += 2) {
+    for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
         const int kk = nt * 8 + (lane & 7);
-        const int ch = k2 * 2 + (lane >> 3);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kbase + tile_off(kk, ch), b0, b1, b2, b3);
-        mma_bf16(sc[nt], qf[k2], b0, b1);
-        mma_bf16(sc[nt], qf[k2 + 1], b2, b3);
+        const int ch = ks * 2 + ((lane >> 3) & 1);
+        uint32_t b0, b1;
+        ldsm_x2(kbase + tile_off(kk, ch), b0, b1);
+        mma_bf16(sc[nt], qf[ks], b0, b1);
       }
     }
     float mx0 = -INFINITY, mx1 = -INFINITY;
