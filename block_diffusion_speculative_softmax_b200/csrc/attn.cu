@@ -150,11 +150,12 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_simt_kernel(const AttnPa
 }
 
 // ---------------------------------------------------------------------------
-// bf16 tensor-core variant: 4 warps x 16 query rows, 64-key tiles streamed
-// into a double-buffered shared-memory ring by cp.async (16-byte chunks,
-// XOR-swizzled per row so ldmatrix is conflict-free), S = Q K^T and
-// O += P V on mma.sync m16n8k16 with fp32 accumulation, P kept in
-// registers, online softmax in the exp2 domain.
+// bf16 tensor-core variant: 4 warps x 16 query rows, 64-key tiles in a
+// double-buffered shared-memory ring (full tiles by TMA, the ragged tail and
+// the block keys by cp.async; 16-byte chunks XOR-swizzled per row so
+// ldmatrix is conflict-free), S = Q K^T and O += P V on mma.sync m16n8k16
+// with fp32 accumulation, P kept in registers, online softmax in the exp2
+// domain.
 // ---------------------------------------------------------------------------
 constexpr int kMmaRows = 64;
 constexpr int kMmaKeys = 64;
@@ -171,11 +172,6 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                        uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
 }
 __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1,
                                           uint32_t& r2, uint32_t& r3) {

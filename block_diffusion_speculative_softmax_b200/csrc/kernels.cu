@@ -40,10 +40,6 @@ __device__ __forceinline__ void fmul2(float& d0, float& d1, float b0, float b1) 
       : "+f"(d0), "+f"(d1) : "f"(b0), "f"(b1));
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 constexpr int kFuseThreads = 512;
 constexpr int kFuseSmemBudget = 221 * 1024;
 
