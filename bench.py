@@ -417,7 +417,8 @@ def kernel_table(wl, cfg, DF, peaks, stream, reps, ms_step):
         kc, vc = fb.k_cache[0], fb.v_cache[0]
         sec = time_calls(lambda: DF.dflash_kv_project(cc, fused[0], pos, None, lay["w_kt"],
                                                       lay["w_vt"], kc, vc, ws), stream, reps)
-        rows.append(_entry("ctx_kv_proj", "gemm_tok_kernel (RoPE epilogue)", sec, D,
+        rows.append(_entry("ctx_kv_proj", "gemm_tokp_kernel / gemm_tok_kernel (RoPE epilogue)",
+                           sec, D,
                            n_new * H * e + 2 * kvd * H * e + 2 * n_new * kvd * e,
                            2.0 * n_new * H * 2 * kvd, peaks, ms_step))
         del fused
@@ -710,7 +711,7 @@ def run_op(args):
         call = lambda: DF.dflash_kv_project(cc, x, pos, None, wk, wv, ko, vo, ws)
         algo = N * H * e + 2 * kvd * H * e + 2 * N * kvd * e
         flops = 2.0 * N * H * 2 * kvd
-        kernel = "gemm_tok_kernel<256,4> (context K/V projection, RoPE epilogue)"
+        kernel = "gemm_tokp_kernel / gemm_tok_kernel (context K/V projection, RoPE epilogue)"
     elif args.op == "attn":
         q, kb, vb = rnd(M, qd), rnd(M, kvd), rnd(M, kvd)
         kc, vc = rnd(N, kvd), rnd(N, kvd)
