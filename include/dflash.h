@@ -166,7 +166,9 @@ dflash_status dflash_fuse_ctx(const dflash_config* cfg, const void* states,
                               const float* const* g_fuse, void* fused,
                               void* stream);
 
-/* The draft step's split form of the same fusion (bf16 only).  RMSNorm is
+/* The draft step's split form of the same fusion (DFLARE summary, section
+ * 2.1; the split itself is this library's, the pages normalise before the
+ * projection of section 2.2), bf16 only.  RMSNorm is
  * one scalar per row, and the context K/V projection and RoPE are linear, so
  * dflash_draft_step applies the row scale in the projection's epilogue: the
  * fusion stores the rows unnormalised and needs no cross-warp reduction per
