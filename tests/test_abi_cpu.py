@@ -184,3 +184,29 @@ def test_split_fusion_rejects_fp32_and_bad_arguments(lib):
     # no workspace for the status word
     assert lib.dflash_fuse_ctx_rss(C.byref(cfg), None, 0, None, None, None, None, None, 0,
                                    None) == DF.EINVAL
+
+
+def test_split_fusion_pointer_checks_before_any_launch(lib):
+    # fake device addresses: every check here runs on the host and fails
+    # before the library touches CUDA
+    cfg = DF.config_from(synth.small_config("qwen3_4b", hidden=576, n_q_heads=8, n_kv_heads=2,
+                                            head_dim=128, ffn=1000, n_draft_layers=2,
+                                            n_target_layers=3, ctx_len=64, block=16,
+                                            vocab=1000, dtype="bf16"))
+    ws, big = C.c_void_p(1 << 20), 1 << 20
+    g = (C.c_void_p * 2)(1 << 21, 1 << 22)
+    good = dict(states=C.c_void_p(1 << 23), w=C.c_void_p(1 << 24), fused=C.c_void_p(1 << 25),
+                rss=C.c_void_p(1 << 26))
+
+    def call(**over):
+        a = dict(good, **over)
+        return lib.dflash_fuse_ctx_rss(C.byref(cfg), a["states"], 10, a["w"], g, a["fused"],
+                                       a["rss"], ws, big, None)
+
+    assert call(rss=C.c_void_p((1 << 26) + 2)) == DF.EINVAL      # rss not 4-byte aligned
+    assert call(rss=None) == DF.EINVAL
+    assert call(fused=C.c_void_p((1 << 25) + 8)) == DF.EINVAL   # bulk tensor not 16-byte aligned
+    assert call(states=None) == DF.EINVAL
+    assert lib.dflash_fuse_ctx_rss(C.byref(cfg), good["states"], 10, good["w"], g, good["fused"],
+                                   good["rss"], C.c_void_p((1 << 20) + 64), big,
+                                   None) == DF.EINVAL                # workspace not 256-aligned
